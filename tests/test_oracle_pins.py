@@ -1,0 +1,526 @@
+"""Pins of the CPU oracle to things other than itself (no GPU).
+
+Each test checks the oracle against what the pages print, a closed form, an
+invariant, a library routine the step reduces to, or brute force on tiny inputs.
+"""
+import itertools
+import json
+import math
+import os
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as syn
+
+H, I = 2816, 704
+
+
+def f32(x):
+    return struct.unpack("<f", struct.pack("<f", x))[0]
+
+
+def ulp_dist(a: float, b: float) -> int:
+    ia = struct.unpack("<i", struct.pack("<f", a))[0]
+    ib = struct.unpack("<i", struct.pack("<f", b))[0]
+    if ia < 0:
+        ia = -(ia & 0x7FFFFFFF)
+    if ib < 0:
+        ib = -(ib & 0x7FFFFFFF)
+    return abs(ia - ib)
+
+
+# ----------------------------------------------------------------- expert sizes
+
+def test_expert_bytes_match_the_pages(golden_dir):
+    """prain README, 'Expert formats': 11.34 / 5.69 / 3.01 MiB per expert and
+    42.5 / 21.3 / 11.3 GiB for all 30 x 128 experts."""
+    g = json.load(open(os.path.join(golden_dir, "expert_sizes.json")))
+    n = g["layers"] * g["experts_per_layer"]
+    for name, fmt in oracle.FMT_NAMES.items():
+        b = oracle.expert_bytes(fmt, H, I)
+        assert round(b / 2**20, 2) == g["formats"][name]["expert_mib"], name
+        assert round(b * n / 2**30, 1) == g["formats"][name]["all_gib"], name
+
+
+def test_expert_bytes_closed_form():
+    """3*H*I weights per expert; bf16 2 B each; int8 1 B + fp32 per row (2I + H rows);
+    int4 half a byte + one bf16 scale per 64 weights."""
+    for h, i in [(2816, 704), (256, 128), (64, 64), (1024, 192)]:
+        w = 3 * h * i
+        assert oracle.expert_bytes(oracle.BF16, h, i) == 2 * w
+        assert oracle.expert_bytes(oracle.INT8, h, i) == w + 4 * (2 * i + h)
+        assert oracle.expert_bytes(oracle.INT4, h, i) == w // 2 + 2 * (w // 64)
+    assert oracle.expert_bytes(oracle.BF16, H, I) == 11894784
+    assert oracle.expert_bytes(oracle.INT8, H, I) == 5964288
+    assert oracle.expert_bytes(oracle.INT4, H, I) == 3159552
+
+
+def test_blob_pieces_are_contiguous_and_16_byte_aligned():
+    for fmt in (0, 1, 2):
+        off = oracle.blob_offsets(fmt, H, I)
+        assert off[0] == 0 and off == sorted(off)
+        assert all(o % 256 == 0 for o in off)
+        assert oracle.expert_bytes(fmt, H, I) % 256 == 0
+
+
+# ------------------------------------------------------------------------ exp_p
+
+def test_exp_p_within_two_ulp_of_libm():
+    xs = np.concatenate([
+        np.linspace(-103.0, 88.0, 20001, dtype=np.float32),
+        -np.abs(np.random.default_rng(1).standard_normal(20000).astype(np.float32)) * 8,
+        np.float32([0.0, -0.0, -1e-30, 1e-30, -0.5 * math.log(2), 0.5 * math.log(2), -87.3, -86.0]),
+    ])
+    worst = 0
+    for x in xs:
+        ref = f32(math.exp(float(x)))
+        got = oracle.exp_p(float(x))
+        if ref == 0.0:
+            assert got == 0.0 or got < 2e-45
+            continue
+        worst = max(worst, ulp_dist(got, ref))
+    assert worst <= 2, worst
+
+
+def test_exp_p_special_values_and_monotone():
+    assert oracle.exp_p(0.0) == 1.0
+    assert oracle.exp_p(-0.0) == 1.0
+    assert oracle.exp_p(float("-inf")) == 0.0
+    assert oracle.exp_p(-200.0) == 0.0
+    assert math.isinf(oracle.exp_p(100.0))
+    assert math.isnan(oracle.exp_p(float("nan")))
+    xs = np.linspace(-20, 0, 40001, dtype=np.float32)
+    ys = oracle.exp_p_array(xs)
+    assert np.all(np.diff(ys.astype(np.float64)) >= 0)
+
+
+# ------------------------------------------------------------------------- gelu
+
+def test_gelu_tanh_matches_torch():
+    v = np.linspace(-8, 8, 4001)
+    ref = torch.nn.functional.gelu(torch.tensor(v, dtype=torch.float64), approximate="tanh").numpy()
+    got = np.array([oracle.gelu_tanh(x) for x in v])
+    np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-15)
+    assert oracle.gelu_tanh(0.0) == 0.0
+    assert abs(oracle.gelu_tanh(30.0) - 30.0) < 1e-12
+    assert abs(oracle.gelu_tanh(-30.0)) < 1e-12
+
+
+# ---------------------------------------------------------------------- routing
+
+def test_route_k1_weight_is_one_and_id_is_argmax():
+    lg = syn.router_logits(64, 128, "normal", seed=3)
+    ids, w = oracle.route_topk(lg, 1)
+    assert np.all(w == 1.0)
+    assert np.array_equal(ids[:, 0], np.argmax(lg, axis=1))
+
+
+def test_route_ids_equal_stable_descending_sort():
+    """Ties to the lower expert id: the order of a stable sort of -logit."""
+    rng = np.random.default_rng(5)
+    lg = rng.integers(-3, 4, size=(200, 16)).astype(np.float32)  # many ties
+    for k in (1, 2, 5, 16):
+        ids, _ = oracle.route_topk(lg, k)
+        ref = np.argsort(-lg, axis=1, kind="stable")[:, :k]
+        assert np.array_equal(ids, ref)
+
+
+def test_route_all_equal_logits():
+    ids, w = oracle.route_topk(np.zeros((3, 8), np.float32), 4)
+    assert np.array_equal(ids, np.tile(np.arange(4), (3, 1)))
+    assert np.all(w == 0.25)
+
+
+def test_route_brute_force_subsets():
+    """E=8: the chosen set maximises the summed logit over every k-subset."""
+    lg = syn.router_logits(50, 8, "normal", seed=11)
+    for k in (2, 3):
+        ids, _ = oracle.route_topk(lg, k)
+        for t in range(lg.shape[0]):
+            best = max(itertools.combinations(range(8), k), key=lambda s: (sum(lg[t, list(s)]),
+                                                                            [-e for e in s]))
+            assert sorted(ids[t]) == sorted(best)
+
+
+def test_route_full_k_is_softmax():
+    lg = syn.router_logits(32, 64, "normal", seed=2)
+    ids, w = oracle.route_topk(lg, 64)
+    z = lg.astype(np.float64)
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    ref = np.take_along_axis(p, ids.astype(np.int64), axis=1)
+    np.testing.assert_allclose(w, ref, rtol=2e-6, atol=1e-9)
+    np.testing.assert_allclose(w.astype(np.float64).sum(axis=1), 1.0, atol=1e-5)
+
+
+def test_route_topk_renormalised_softmax_fp64():
+    """Weights equal softmax over all E, kept to the top k and renormalised (fp64)."""
+    lg = syn.router_logits(64, 128, "biased", seed=4)
+    ids, w = oracle.route_topk(lg, 8)
+    z = lg.astype(np.float64)
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    top = np.take_along_axis(p, ids.astype(np.int64), axis=1)
+    ref = top / top.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(w, ref, rtol=3e-6, atol=0)
+    assert np.all(np.diff(w, axis=1) <= 0)  # rank order: non-increasing weights
+
+
+def test_route_nan_ranks_last():
+    lg = np.array([[np.nan, 1.0, 0.5, np.nan]], np.float32)
+    ids, _ = oracle.route_topk(lg, 4)
+    assert ids.tolist() == [[1, 2, 0, 3]]
+
+
+# ---------------------------------------------------------------------- permute
+
+def test_permute_equals_stable_argsort_and_bincount():
+    rng = np.random.default_rng(7)
+    for T, k, E in [(37, 3, 11), (1, 8, 128), (64, 8, 128), (5, 1, 2)]:
+        ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
+        counts, offsets, sr, rp = oracle.permute(ids, E)
+        flat = ids.ravel()
+        assert np.array_equal(counts, np.bincount(flat, minlength=E))
+        assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+        assert np.array_equal(sr, np.argsort(flat, kind="stable"))
+        assert np.array_equal(rp[sr], np.arange(T * k))
+        # token of a sorted row is route // k (remote_experts.cpp, begin)
+        assert np.array_equal(flat[sr], np.repeat(np.arange(E), counts))
+
+
+def test_permute_drops_out_of_range_ids():
+    ids = np.array([[0, 5], [-1, 1], [1, 9]], np.int32)
+    counts, offsets, sr, rp = oracle.permute(ids, 3)
+    assert counts.tolist() == [1, 2, 0]
+    assert offsets.tolist() == [0, 1, 3, 3]
+    assert sr.tolist() == [0, 3, 4, -1, -1, -1]
+    assert rp.tolist() == [0, -1, -1, 1, 2, -1]
+
+
+# ------------------------------------------------------------------------- hits
+
+def test_hits_page_vector(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "expert_pool_vectors.json")))["count_hits_matches_bincount"]
+    assert oracle.hits(np.array(g["ids"]), g["E"]).tolist() == g["hits"]
+
+
+def test_hits_is_bincount_ignoring_out_of_range_and_accumulates():
+    rng = np.random.default_rng(9)
+    ids = rng.integers(-5, 140, size=5000).astype(np.int32)
+    ok = ids[(ids >= 0) & (ids < 128)]
+    h = oracle.hits(ids, 128)
+    assert np.array_equal(h, np.bincount(ok, minlength=128))
+    assert np.array_equal(oracle.hits(ids, 128, h), 2 * h)
+
+
+# ------------------------------------------------------------------- quantisers
+
+def test_int8_exact_on_representable_rows():
+    rng = np.random.default_rng(1)
+    rows = []
+    for j in range(6):
+        m = rng.integers(-127, 128, size=256)
+        m[rng.integers(0, 256)] = 127 * (1 if j % 2 else -1)
+        rows.append(m * 2.0 ** (-3 - j))
+    w = syn.bf16_bits(np.array(rows, np.float32))
+    q, s = oracle.quantize_int8(w)
+    for j in range(6):
+        assert s[j] == np.float32(2.0 ** (-3 - j))
+        assert np.array_equal(q[j].astype(np.int64) * 1.0 * 2.0 ** (-3 - j), syn.bf16_to_f32(w[j]))
+
+
+def test_int8_zero_row_and_error_bound():
+    w = syn.normal_bf16((64, 512), 0.02, 3, 0)
+    w[5] = 0
+    q, s = oracle.quantize_int8(w)
+    assert s[5] == 0 and np.all(q[5] == 0)
+    wf = syn.bf16_to_f32(w).astype(np.float64)
+    err = np.abs(wf - q.astype(np.float64) * s[:, None].astype(np.float64))
+    # |w/s| <= 127, so the fp32 quotient carries at most 127 * 2^-24 of rounding
+    assert np.all(err <= s[:, None].astype(np.float64) * (0.5 + 127 * 2.0**-24) + 1e-30)
+    assert np.all(np.abs(q) <= 127)
+    assert np.all(np.abs(q).max(axis=1)[s > 0] == 127)
+
+
+def _unpack_int4(qb: np.ndarray) -> np.ndarray:
+    lo = (qb & 15).astype(np.int64) - 8
+    hi = (qb >> 4).astype(np.int64) - 8
+    out = np.empty(qb.shape[:-1] + (qb.shape[-1] * 2,), np.int64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def test_int4_nibble_layout_and_exact_groups():
+    """Groups that are m * s with |m| <= 7 (some |m| = 7) and s a bf16 value come
+    back exactly; byte j carries weight 2j low and 2j+1 high."""
+    rng = np.random.default_rng(2)
+    rows = []
+    scales = []
+    for r in range(8):
+        # a 5-bit mantissa keeps every m * s (|m| <= 7) exact in bf16
+        s = float(rng.integers(16, 32)) * 2.0 ** -int(rng.integers(8, 14))
+        m = rng.integers(-7, 8, size=128)
+        m[3] = 7
+        m[64 + 5] = -7
+        rows.append(m * s)
+        scales.append(s)
+    w = syn.bf16_bits(np.array(rows, np.float32))
+    assert np.array_equal(syn.bf16_to_f32(w).astype(np.float64), np.array(rows))
+    q, sb = oracle.quantize_int4(w)
+    sf = syn.bf16_to_f32(sb)
+    for r in range(8):
+        assert sf[r, 0] == np.float32(scales[r]) and sf[r, 1] == np.float32(scales[r])
+        deq = _unpack_int4(q[r]) * float(scales[r])
+        assert np.array_equal(deq, np.array(rows[r]))
+    # explicit nibble order on a hand example
+    s = 2.0 ** -6
+    m = np.array([(c % 15) - 7 for c in range(64)])
+    q1, _ = oracle.quantize_int4(syn.bf16_bits(np.float32(m * s))[None, :])
+    assert q1[0, 0] == ((m[0] + 8) | ((m[1] + 8) << 4))
+    assert q1[0, 31] == ((m[62] + 8) | ((m[63] + 8) << 4))
+
+
+def _exact_err(w64: np.ndarray, s: float) -> Fraction:
+    """Exact sum of squared residuals with the best codes in [-8, 7] for scale s."""
+    tot = Fraction(0)
+    sF = Fraction(s)
+    for v in w64:
+        vF = Fraction(float(v))
+        best = min((abs(vF - m * sF) for m in range(-8, 8)))
+        tot += best * best
+    return tot
+
+
+def test_int4_clip_search_is_the_mse_argmin():
+    """For each group: every candidate error is the exact error of the best codes
+    for its scale (to fp64 rounding), candidate scales are r * absmax / 7 for
+    ratios running 0.70 .. 1.00, and the stored scale is the strict argmin with
+    ties kept at the larger ratio."""
+    w = syn.normal_bf16((3, 64 * 6), 0.02, 9, 1)
+    q, sb = oracle.quantize_int4(w)
+    sf = syn.bf16_to_f32(sb)
+    for r in range(3):
+        for g in range(6):
+            w64 = w[r, g * 64:(g + 1) * 64]
+            wf = syn.bf16_to_f32(w64).astype(np.float64)
+            amax = np.abs(wf).max()
+            s_c, e_c = oracle.int4_candidates(w64)
+            ratios = s_c / (amax / 7.0)
+            assert np.all(np.diff(s_c) >= 0)
+            assert abs(ratios[0] - 0.70) < 0.01 and abs(ratios[15] - 1.0) < 0.01
+            for i in range(16):
+                ex = float(_exact_err(wf, float(s_c[i])))
+                assert abs(e_c[i] - ex) <= 1e-12 * max(ex, 1e-30) + 1e-300
+            best = min(range(15, -1, -1), key=lambda i: (e_c[i], -i))
+            assert sf[r, g] == s_c[best]
+            # stored codes are the nearest codes for the stored scale
+            deq = _unpack_int4(q[r, g * 32:(g + 1) * 32]) * float(sf[r, g])
+            assert float(sum(Fraction(float(a)) ** 2 for a in (wf - deq))) == pytest.approx(
+                float(_exact_err(wf, float(sf[r, g]))), rel=1e-12, abs=1e-300)
+    # on Gaussian weights clipping usually pays: most groups keep a ratio below 1.0,
+    # and no chosen error exceeds the unclipped (ratio 1.0) candidate's
+    wg = syn.normal_bf16((8, 64 * 44), 0.02, 9, 2)
+    _, sbg = oracle.quantize_int4(wg)
+    sfg = syn.bf16_to_f32(sbg)
+    clipped = 0
+    for r in range(8):
+        for g in range(44):
+            s_c, e_c = oracle.int4_candidates(wg[r, g * 64:(g + 1) * 64])
+            i = int(np.nonzero(s_c == sfg[r, g])[0][-1])
+            assert e_c[i] <= e_c[15]
+            clipped += sfg[r, g] < s_c[15]
+    assert clipped > 0.5 * 8 * 44
+
+
+def test_int4_zero_group():
+    w = np.zeros((1, 64), np.uint16)
+    q, s = oracle.quantize_int4(w)
+    assert s[0, 0] == 0 and np.all(q == 0x88)
+
+
+# ------------------------------------------------------------------ expert FFN
+
+def _tiny_layer(fmt, E=4, h=128, i=64, seed=0):
+    w13, w2 = syn.expert_weights(E, h, i, seed=seed)
+    blobs = []
+    deq13, deq2 = [], []
+    for e in range(E):
+        if fmt == oracle.BF16:
+            blobs.append(oracle.pack_expert(fmt, h, i, w13[e], None, w2[e], None))
+            deq13.append(syn.bf16_to_f32(w13[e]).astype(np.float64))
+            deq2.append(syn.bf16_to_f32(w2[e]).astype(np.float64))
+        elif fmt == oracle.INT8:
+            q13, s13 = oracle.quantize_int8(w13[e])
+            q2, s2 = oracle.quantize_int8(w2[e])
+            blobs.append(oracle.pack_expert(fmt, h, i, q13, s13, q2, s2))
+            deq13.append(q13.astype(np.float64) * s13[:, None].astype(np.float64))
+            deq2.append(q2.astype(np.float64) * s2[:, None].astype(np.float64))
+        else:
+            q13, s13 = oracle.quantize_int4(w13[e])
+            q2, s2 = oracle.quantize_int4(w2[e])
+            blobs.append(oracle.pack_expert(fmt, h, i, q13, s13, q2, s2))
+            deq13.append(_unpack_int4(q13) * np.repeat(syn.bf16_to_f32(s13).astype(np.float64), 64, axis=1))
+            deq2.append(_unpack_int4(q2) * np.repeat(syn.bf16_to_f32(s2).astype(np.float64), 64, axis=1))
+    home = np.concatenate(blobs)
+    return oracle.Layer(fmt, E, h, i, home), deq13, deq2
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_single_expert_ffn_is_the_textbook_gemm_gelu_gemm(fmt):
+    """One expert, k = 1: GEMM -> GELU-tanh gate * up -> GEMM in torch fp64, from
+    weights dequantised independently here (q * s with the page's scale layout)."""
+    L, d13, d2 = _tiny_layer(fmt)
+    x = syn.activations(5, L.H, seed=1)
+    xf = torch.tensor(syn.bf16_to_f32(x).astype(np.float64))
+    for e in range(L.E):
+        g = xf @ torch.tensor(d13[e]).T
+        hh = torch.nn.functional.gelu(g[:, :L.I], approximate="tanh") * g[:, L.I:]
+        ref = (hh @ torch.tensor(d2[e]).T).numpy()
+        for t in range(5):
+            y = oracle.expert_ffn(L, e, x[t])
+            np.testing.assert_allclose(y, ref[t], rtol=1e-10, atol=1e-12)
+
+
+def test_weight_accessor_matches_independent_dequant():
+    for fmt in (0, 1, 2):
+        L, d13, d2 = _tiny_layer(fmt, E=1)
+        rng = np.random.default_rng(fmt)
+        for _ in range(50):
+            r, c = rng.integers(0, 2 * L.I), rng.integers(0, L.H)
+            assert oracle.weight(fmt, L.home, L.H, L.I, 13, r, c) == d13[0][r, c]
+            r, c = rng.integers(0, L.H), rng.integers(0, L.I)
+            assert oracle.weight(fmt, L.home, L.H, L.I, 2, r, c) == d2[0][r, c]
+
+
+def test_zero_activation_gives_zero_output():
+    L, _, _ = _tiny_layer(0)
+    assert np.all(oracle.expert_ffn(L, 1, np.zeros(L.H, np.uint16)) == 0.0)
+
+
+def test_dense_all_experts_then_mask_equals_routed():
+    """Tiny layer (8 experts, hidden 256, intermediate 128, top-2, 16 tokens): every
+    expert on every token, then a dense [T, E] weight matrix that is zero off the
+    top-k, equals the routed layer."""
+    E, h, i, k, T = 8, 256, 128, 2, 16
+    L, _, _ = _tiny_layer(0, E=E, h=h, i=i)
+    x = syn.activations(T, h, seed=0)
+    lg = syn.router_logits(T, E, "normal", seed=0)
+    ids, w, rows, y = oracle.moe_layer(L, lg, x, k)
+    dense_w = np.zeros((T, E))
+    for t in range(T):
+        for j in range(k):
+            dense_w[t, ids[t, j]] = w[t, j]
+    allx = np.zeros((T, E, h))
+    for t in range(T):
+        for e in range(E):
+            allx[t, e] = oracle.expert_ffn(L, e, x[t])
+    for t in range(T):
+        for j in range(k):
+            assert np.array_equal(rows[t * k + j], allx[t, ids[t, j]])
+    ydense = np.einsum("te,teh->th", dense_w, allx)
+    np.testing.assert_allclose(y, ydense, rtol=1e-12, atol=1e-14)
+
+
+def test_combine_k1_unit_weight_is_identity():
+    rows = np.random.default_rng(0).standard_normal((7, 33))
+    ids = np.arange(7, dtype=np.int32)[:, None] % 3
+    y = oracle.combine(rows, ids, np.ones((7, 1), np.float32), 3)
+    assert np.array_equal(y, rows)
+
+
+def test_slot_table_only_moves_where_blobs_are_read():
+    """Router logits and expert ids are untouched by placement (expert_pool.rs,
+    module doc): a layer whose experts are served from cache slots gives the same
+    rows as the same layer served from home."""
+    E, h, i, k, T = 8, 128, 64, 2, 6
+    L, _, _ = _tiny_layer(2, E=E, h=h, i=i)
+    eb = L.expert_bytes
+    slot_of = np.full(E, -1, np.int32)
+    slot_of[[5, 1, 6]] = [0, 2, 1]
+    pool = np.zeros(3 * eb, np.uint8)
+    for e in (5, 1, 6):
+        pool[slot_of[e] * eb:(slot_of[e] + 1) * eb] = L.home[e * eb:(e + 1) * eb]
+    Ls = oracle.Layer(2, E, h, i, L.home, pool=pool, slot_table=slot_of)
+    x = syn.activations(T, h, seed=3)
+    lg = syn.router_logits(T, E, "normal", seed=3)
+    a = oracle.moe_layer(L, lg, x, k)
+    b = oracle.moe_layer(Ls, lg, x, k)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+    # and the slot really is what is read: corrupt home of a slotted expert
+    home2 = L.home.copy()
+    home2[5 * eb:6 * eb] = 0
+    Lc = oracle.Layer(2, E, h, i, home2, pool=pool, slot_table=slot_of)
+    assert np.array_equal(oracle.moe_layer(Lc, lg, x, k)[3], a[3])
+
+
+# -------------------------------------------------------------------- placement
+
+def test_placement_page_vectors(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "expert_pool_vectors.json")))
+    c = g["target_gpu_picks_top_by_count"]
+    assert oracle.refresh_target(np.array(c["counts"], np.uint32), c["budget"]).tolist() == c["target"]
+
+    c = g["paired_swap_limits_demotions"]
+    so = np.full(c["E"], -1, np.int32)
+    so[c["resident"]] = np.arange(len(c["resident"]))
+    so2, pr, de = oracle.apply_placement(so, c["budget"], np.array(c["target"]))
+    assert len(pr) == c["promotions"] and len(de) == c["demotions"]
+    assert sorted(np.nonzero(so2 >= 0)[0].tolist()) == c["resident_after"]
+
+    c = g["paired_swap_keeps_extra_residents"]
+    so = np.full(c["E"], -1, np.int32)
+    so[c["resident"]] = np.arange(len(c["resident"]))
+    so2, pr, de = oracle.apply_placement(so, c["budget"], np.array(c["target"]))
+    assert len(pr) == c["promotions"] and len(de) == c["demotions"]
+    assert int((so2 >= 0).sum()) == c["resident_count_after"]
+    assert all(so2[e] >= 0 for e in c["must_be_resident"])
+    assert all(so2[e] < 0 for e in c["must_not_be_resident"])
+
+    c = g["jump_steps_refresh_schedule"]
+    offload = c["budget"] < c["E"]
+    for step, prefill, want in c["cases"]:
+        assert oracle.should_refresh(offload, False, step, prefill, c["interval"]) == want
+
+    c = g["vram_budget_formula"]
+    b = oracle.budget_from_vram(c["free_bytes"], c["reserve_bytes"], c["expert_bytes"], c["layers"],
+                                c["max_per_layer"], c["E"])
+    assert 0 < b <= 128
+    assert b == min((c["free_bytes"] - c["reserve_bytes"]) // (c["expert_bytes"] * c["layers"]), 128)
+
+    c = g["per_layer_masks_differ_from_merged_union"]
+    masks = []
+    for ids in c["refresh_ids"]:
+        so = np.full(c["E"], -1, np.int32)
+        so[: c["budget"]] = np.arange(c["budget"])  # initial residents 0..budget
+        t = oracle.refresh_target(oracle.hits(np.array(ids), c["E"]), c["budget"])
+        so2, _, _ = oracle.apply_placement(so, c["budget"], t)
+        masks.append((so2 >= 0).tolist())
+    assert masks == c["per_layer"]
+    assert np.logical_or.reduce(np.array(masks)).tolist() == c["merged"]
+
+
+def test_placement_invariants_under_random_refreshes():
+    rng = np.random.default_rng(4)
+    E, n_slots = 128, 18
+    so = np.full(E, -1, np.int32)
+    so[:n_slots] = np.arange(n_slots)
+    for step in range(200):
+        ids = rng.zipf(1.3, size=64 * 8) % E
+        t = oracle.refresh_target(oracle.hits(ids.astype(np.int32), E), n_slots)
+        before = so.copy()
+        so, pr, de = oracle.apply_placement(so, n_slots, t)
+        res = np.nonzero(so >= 0)[0]
+        assert len(res) == n_slots                        # residency size stays the budget
+        assert sorted(so[res].tolist()) == list(range(n_slots))  # slots are a permutation
+        assert all(so[e] >= 0 for e in t)                 # the target is resident
+        assert len(pr) == len(de)                         # paired swaps
+        assert all(before[e] < 0 for e in pr) and all(before[e] >= 0 for e in de)
+        for p, d in zip(pr, de):
+            assert so[p] == before[d]                     # promoted takes the demoted slot

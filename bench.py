@@ -1,0 +1,533 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert MoE layer on B200.
+
+One step = one pass of the whole layer over one batch: route (top-k of fp32
+router logits) -> permute + expert-hit histogram -> grouped gated FFN over the
+routed experts (through the slot table) -> weighted combine, all in the
+library's kernels, inputs already resident in HBM.
+
+Default workload: one Gemma-shaped MoE layer, bf16 experts: 128 experts,
+hidden 2816, expert intermediate 704 (11.34 MiB per expert), top-8, decode
+batch of 64 tokens, router logits N(0,1), weights N(0,0.02), activations N(0,1).
+To keep the expert weights out of L2 (126 MB), each step reads a different one
+of 30 distinct layer copies (45.7 GB in HBM for bf16), so a layer's experts
+come back only after 29 other layers' worth of traffic.  The batches of 1 and
+8 tokens are measured in the same run and reported under "sweep".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--config decode-bf16|decode-int8|int4-decode|int4-prefill|tiny]
+                  [--tokens T]
+
+Multi-GPU (N > 1, launched by torchrun): the layer does not shard across GPUs
+in this build, so every rank runs an independent replica of the same
+workload (weak scaling, no collective on the data path); the timing is the
+max over ranks.
+
+--impl reference times the CPU oracle (plain C, every host core) on a bounded
+sample of the same workload on rank 0; it is the baseline, not the target.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# grouped-FFN kernels from one ncu capture, per workload; None until captured
+# for the kernels as they stand (see profiles/).
+NCU_TRAFFIC_BYTES = {}
+
+CONFIGS = {
+    # name: (weight format, logits kind, tokens, extra batches swept)
+    "decode-bf16": ("bf16", "normal", 64, [1, 8]),
+    "decode-int8": ("int8", "biased", 64, [1, 8]),
+    "int4-decode": ("int4", "normal", 64, []),
+    "int4-prefill": ("int4", "normal", 1024, []),
+    "tiny": ("bf16", "normal", 16, []),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=30)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="decode-bf16", choices=sorted(CONFIGS))
+    ap.add_argument("--tokens", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self._t is not None:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- workload
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def build_layers(moe, torch, fmt_name, E, H, I, n_layers, dev, seed=0):
+    """n_layers distinct copies of the layer's expert blobs in HBM."""
+    import synthetic as syn
+
+    fmt = moe.FMT[fmt_name]
+    eb = moe.moe_expert_bytes(fmt, H, I)
+    layers = []
+    for l in range(n_layers):
+        if fmt == moe.MOE_W_BF16:
+            # a bf16 blob is W13 then W2, all bf16: draw it in place
+            home = torch.empty(E * eb, dtype=torch.uint8, device=dev)
+            hv = home.view(torch.bfloat16)
+            g = torch.Generator(device=dev)
+            g.manual_seed(1000 * seed + l)
+            step = 1 << 26
+            for i in range(0, hv.numel(), step):
+                n = min(step, hv.numel() - i)
+                hv[i:i + n] = (torch.randn(n, generator=g, device=dev) * syn.WEIGHT_STD).to(torch.bfloat16)
+            layers.append(moe.MoeLayer(fmt, E, H, I, home, expert_bytes=eb))
+        else:
+            w13, w2 = syn.torch_expert_weights(E, H, I, seed=seed, layer=l, device=dev)
+            layers.append(moe.make_layer(fmt, w13, w2))
+            del w13, w2
+    torch.cuda.synchronize(dev)
+    return layers
+
+
+def make_batches(torch, kind, T, E, H, n, dev, seed=0):
+    import synthetic as syn
+
+    out = []
+    for b in range(n):
+        lg = syn.router_logits(T, E, kind, seed=seed + 17, layer=b)
+        x = syn.activations(T, H, seed=seed + 23, layer=b)
+        out.append((lg, x, torch.from_numpy(lg).to(dev),
+                    torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)))
+    return out
+
+
+class Runner:
+    """Device buffers for one batch size; step(i) runs the layer on batch i."""
+
+    def __init__(self, moe, torch, layers, batches, T, k, dev):
+        self.moe, self.torch, self.layers, self.batches, self.T, self.k = moe, torch, layers, batches, T, k
+        E, H = layers[0].E, layers[0].H
+        R = T * k
+        i32 = torch.int32
+        self.ids = torch.empty((T, k), dtype=i32, device=dev)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.perm = (torch.empty(E, dtype=i32, device=dev), torch.empty(E + 1, dtype=i32, device=dev),
+                     torch.empty(R, dtype=i32, device=dev), torch.empty(R, dtype=i32, device=dev))
+        self.hits = torch.zeros((len(layers), E), dtype=i32, device=dev)
+        self.rows = torch.empty((R, H), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(moe.moe_grouped_ffn_workspace(layers[0], T, k), 16), dtype=torch.uint8, device=dev)
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.ev = None
+
+    def step(self, i, ffn_events=None):
+        moe = self.moe
+        li = i % len(self.layers)
+        L = self.layers[li]
+        _, _, lg, x = self.batches[i % len(self.batches)]
+        moe.moe_route_topk(lg, self.k, self.ids, self.w)
+        counts, offsets, sr, rp = moe.moe_permute(self.ids, L.E, hits=self.hits[li], out=self.perm)
+        if ffn_events is not None:
+            ffn_events[0].record()
+        moe.moe_grouped_ffn(L, x, self.k, counts, offsets, sr, rows=self.rows, ws=self.ws)
+        if ffn_events is not None:
+            ffn_events[1].record()
+        moe.moe_combine(self.rows, rp, self.w, self.y)
+
+    LAUNCHES_PER_STEP = 5  # route, permute, FFN phase 1, FFN phase 2, combine
+
+    def distinct_experts(self):
+        """Distinct routed experts of each batch (read back from our own routing)."""
+        out = []
+        for i in range(len(self.batches)):
+            self.step(i)
+            self.torch.cuda.synchronize()
+            out.append(int((self.perm[0] > 0).sum().item()))
+        return out
+
+
+def _capture(torch, runner, first, n):
+    """One CUDA graph of n consecutive steps, with an external event pair around
+    each step's grouped-FFN launches (event record nodes inside the graph)."""
+    g = torch.cuda.CUDAGraph()
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(n)]
+    with torch.cuda.graph(g):
+        for j in range(n):
+            runner.step(first + j, evs[j])
+    return g, evs
+
+
+def time_steps(torch, runner, steps, warmup, dist):
+    """Exactly `steps` steps between two events, replayed from CUDA graphs of one
+    rotation over the layers (so Python launch overhead is out of the timed
+    region).  Returns (total ms, per-step FFN ms from the last replay of each graph)."""
+    G = len(runner.layers)
+    for i in range(warmup):
+        runner.step(i)
+    torch.cuda.synchronize()
+    full, rem = steps // G, steps % G
+    graphs = []
+    if full:
+        graphs.append(_capture(torch, runner, warmup, G))
+    if rem:
+        graphs.append(_capture(torch, runner, warmup, rem))
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(full):
+        graphs[0][0].replay()
+    if rem:
+        graphs[-1][0].replay()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if dist is not None:
+        dist.barrier()
+    ffn_ms = [a.elapsed_time(b) for _, evs in graphs for a, b in evs]
+    del graphs
+    return ms, ffn_ms
+
+
+def time_e2e(torch, moe, layers, batches, T, k, steps, warmup, dev):
+    """End to end through moe_layer_forward with host buffers: H2D of logits and x
+    from pinned memory, the layer, D2H of y, every step, on one stream."""
+    E, H = layers[0].E, layers[0].H
+    host_lg = [torch.from_numpy(b[0]).pin_memory() for b in batches]
+    host_x = [torch.from_numpy(b[1].view(np.int16)).pin_memory() for b in batches]
+    host_y = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    d_lg = torch.empty((T, E), dtype=torch.float32, device=dev)
+    d_x = torch.empty((T, H), dtype=torch.int16, device=dev)
+    d_y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(moe.moe_layer_forward_workspace(layers[0], T, k), dtype=torch.uint8, device=dev)
+
+    def one(i):
+        b = i % len(batches)
+        d_lg.copy_(host_lg[b], non_blocking=True)
+        d_x.copy_(host_x[b], non_blocking=True)
+        moe.moe_layer_forward(layers[i % len(layers)], d_lg, d_x.view(torch.bfloat16), k, y=d_y, ws=ws)
+        host_y.copy_(d_y.view(torch.int16), non_blocking=True)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        one(warmup + i)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    return ms, T * E * 4 + T * H * 2, T * H * 2
+
+
+def cpu_baseline(moe, torch, cfg_fmt, layers, batches, T, k, seconds, first_token_only=False):
+    """The oracle (as it stands) on a bounded sample: whole tokens of batch 0 of
+    layer 0, one at a time, until `seconds` have passed."""
+    import oracle
+
+    L = layers[0]
+    E, H, I = L.E, L.H, L.I
+    fmt = L.fmt
+    lg, x = batches[0][0], batches[0][1]
+    ids, _ = oracle.route_topk(lg, k)
+    # host copies of the experts the sample can touch (input bytes, drawn by the
+    # seeded generator); the oracle quantises bf16 weights itself for int8/int4
+    need = sorted(set(ids.ravel().tolist()))
+    eb = oracle.expert_bytes(fmt, H, I)
+    slot = np.full(E, -1, np.int32)
+    pool = np.zeros(len(need) * eb, np.uint8)
+    home_host = None
+    if fmt == 0:
+        for i, e in enumerate(need):
+            slot[e] = i
+            pool[i * eb:(i + 1) * eb] = L.home[e * eb:(e + 1) * eb].cpu().numpy()
+    else:
+        return None  # the quantised formats need the source bf16 weights; bf16 is the benchmarked config
+    OL = oracle.Layer(fmt, E, H, I, np.zeros(eb, np.uint8), pool=pool, slot_table=slot)
+    oracle.set_threads(os.cpu_count() or 1)
+    threads = oracle.get_threads()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.moe_layer(OL, lg[n:n + 1], x[n:n + 1], k)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or n >= T or first_token_only:
+            break
+    del home_host
+    return {"value": n / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of the {T} tokens of one batch ({n * k} routes), whole layer "
+                      f"(route, per-route fp64 FFN, combine), {el:.1f} s"}
+
+
+def main():
+    args = parse()
+    fmt_name, kind, T0, sweep = CONFIGS[args.config]
+    T = args.tokens or T0
+    E, H, I, k = (8, 256, 128, 2) if args.config == "tiny" else (128, 2816, 704, 8)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return reference_arm(args, fmt_name, kind, T, E, H, I, k, world, rank)
+
+    import torch
+
+    import moe_router_softmax_b200 as moe
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist = tdist
+
+    n_layers = args.layers if args.config != "tiny" else 2
+    layers = build_layers(moe, torch, fmt_name, E, H, I, n_layers, dev)
+    batches = make_batches(torch, kind, T, E, H, 8, dev)
+    runner = Runner(moe, torch, layers, batches, T, k, dev)
+    distinct = runner.distinct_experts()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms, ffn_ms = time_steps(torch, runner, args.steps, args.warmup, dist)
+    clk = clocks.stop()
+
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * T * args.steps / (ms / 1e3)
+
+    # roofline of the dominant kernel (the grouped FFN: two launches per step)
+    eb = moe.moe_expert_bytes(moe.FMT[fmt_name], H, I)
+    avg_distinct = sum(distinct[(args.warmup + i) % len(distinct)] for i in range(args.steps)) / args.steps
+    alg_bytes = avg_distinct * eb + T * H * 2
+    ffn_avg_ms = sum(ffn_ms) / len(ffn_ms)
+    achieved = alg_bytes / (ffn_avg_ms / 1e3) / 1e9
+    hbm_peak, tf_peak, peak_src = measured_peaks()
+    traffic = NCU_TRAFFIC_BYTES.get((args.config, T))
+    layer_bytes = avg_distinct * eb + T * H * 2 * 2 + T * E * 4
+
+    sweep_out = {}
+    for Ts in sweep:
+        b2 = make_batches(torch, kind, Ts, E, H, 8, dev, seed=Ts)
+        r2 = Runner(moe, torch, layers, b2, Ts, k, dev)
+        d2 = r2.distinct_experts()
+        ms2, ffn2 = time_steps(torch, r2, args.steps, args.warmup, dist)
+        if dist is not None:
+            t = torch.tensor([ms2], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms2 = float(t.item())
+        dd = sum(d2) / len(d2)
+        f2 = sum(ffn2) / len(ffn2)
+        sweep_out[f"T{Ts}"] = {
+            "tokens_per_s": round(world * Ts * args.steps / (ms2 / 1e3), 1),
+            "us_per_step": round(ms2 / args.steps * 1e3, 2),
+            "ffn_us": round(f2 * 1e3, 2),
+            "distinct_experts": round(dd, 2),
+            "ffn_hbm_gbs": round((dd * eb + Ts * H * 2) / (f2 / 1e3) / 1e9, 1),
+            "ffn_frac_of_hbm": round((dd * eb + Ts * H * 2) / (f2 / 1e3) / 1e9 / hbm_peak, 4),
+        }
+
+    e2e_ms, h2d, d2h = time_e2e(torch, moe, layers, batches, T, k, args.steps, args.warmup, dev)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(moe, torch, fmt_name, layers, batches, T, k, args.cpu_seconds)
+
+    line = {
+        "metric": "MoE layer tokens/s and expert-weight HBM GB/s (% of roofline) at decode/prefill",
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": fmt_name,
+        "data": "synthetic (seeded; Gemma-4-26B-A4B-shaped layer, random weights)",
+        "config": {
+            "workload": f"moe-layer-{fmt_name}-{'prefill' if T > 64 else 'decode'}-T{T}",
+            "experts": E, "hidden": H, "intermediate": I, "top_k": k, "tokens": T,
+            "weights": fmt_name, "logits": kind, "layers_rotated": n_layers,
+            "l2": f"inputs larger than L2: each step reads a different one of {n_layers} layer copies "
+                  f"({n_layers * E * eb / 1e9:.1f} GB of expert blobs)",
+            "parallelism": f"replicas x{world}",
+        },
+        "layer_hbm_gbs": round(layer_bytes / (ms_step / 1e3) / 1e9, 1),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "grouped FFN (w13+GELU gate, then w2; 2 launches)",
+            "achieved": round(achieved, 1),
+            "peak": hbm_peak,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": traffic,
+            "alg_bytes_per_launch": int(alg_bytes),
+            "avg_launch_us": round(ffn_avg_ms * 1e3, 2),
+        },
+        "sweep": sweep_out,
+        "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": Runner.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def reference_arm(args, fmt_name, kind, T, E, H, I, k, world, rank):
+    """The CPU oracle on the same workload: each step is one token of the batch
+    (k routes through the fp64 per-route FFN), on every host core; rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    import synthetic as syn
+
+    if fmt_name != "bf16":
+        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the bf16 layer only"}))
+        return
+    eb = oracle.expert_bytes(0, H, I)
+    lg = syn.router_logits(T, E, kind, seed=17, layer=0)
+    x = syn.activations(T, H, seed=23, layer=0)
+    ids, _ = oracle.route_topk(lg, k)
+    need = sorted(set(ids.ravel().tolist()))
+    w13, w2 = {}, {}
+    for e in need:  # the experts of this batch, drawn by the seeded host generator
+        a = syn.normal_bf16((1, 2 * I, H), syn.WEIGHT_STD, 0, syn.S_W13, 0, e)
+        b = syn.normal_bf16((1, H, I), syn.WEIGHT_STD, 0, syn.S_W2, 0, e)
+        w13[e], w2[e] = a[0], b[0]
+    slot = np.full(E, -1, np.int32)
+    pool = np.zeros(len(need) * eb, np.uint8)
+    for i, e in enumerate(need):
+        slot[e] = i
+        pool[i * eb:(i + 1) * eb] = oracle.pack_expert(0, H, I, w13[e], None, w2[e], None)
+    OL = oracle.Layer(0, E, H, I, np.zeros(eb, np.uint8), pool=pool, slot_table=slot)
+    oracle.set_threads(os.cpu_count() or 1)
+    for i in range(args.warmup):
+        t = i % T
+        oracle.moe_layer(OL, lg[t:t + 1], x[t:t + 1], k)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        t = (args.warmup + i) % T
+        oracle.moe_layer(OL, lg[t:t + 1], x[t:t + 1], k)
+    el = time.perf_counter() - t0
+    value = args.steps / el
+    cores = oracle.get_threads()
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "MoE layer tokens/s and expert-weight HBM GB/s (% of roofline) at decode/prefill",
+        "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"moe-layer-{fmt_name}-decode-T{T}", "experts": E, "hidden": H,
+                   "intermediate": I, "top_k": k, "tokens": T, "weights": fmt_name, "logits": kind},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step one token of the {T}-token batch ({k} routes), "
+                                   f"{args.steps} steps"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    main()

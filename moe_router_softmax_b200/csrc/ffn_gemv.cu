@@ -1,0 +1,424 @@
+// ffn_gemv.cu -- grouped gated FFN for decode-sized batches: a split-K,
+// warp-shuffle-reduced grouped GEMV that streams every routed expert's weights
+// from HBM exactly once, dequantising in registers.
+//
+// What it computes (prain README.md, "Expert formats", for the formats; the
+// gated GELU-tanh FFN with w13 = gate rows [0,I) stacked on up rows [I,2I)):
+//   phase 1 (k_ffn_gemv<..., 1>):  for every sorted route row s of expert e,
+//        g = W13_e x_{token(s)},  h[s][i] = bf16(gelu_tanh(g_i) * g_{I+i})
+//   phase 2 (k_ffn_gemv<..., 2>):  rows[s] = W2_e h[s]
+// with fp32 accumulation.  token(s) = sorted_route[s] / k (remote_experts.cpp,
+// RemoteExperts::begin).  An expert is reached through the slot table
+// (expert_blob()).
+//
+// Work decomposition.  A work item is (active expert, chunk of <= 8 of its
+// routes, tile of output rows).  Each CTA (8 warps) takes a contiguous range
+// of items, so consecutive items share an expert and the routes' activations
+// stay in shared memory (fp32, bank-conflict-free "sub-plane" layout).  Inside
+// a tile, a lane group of LG lanes owns RWP weight rows (phase 1: RWP/2 gate
+// rows and their RWP/2 up rows, so the GELU gate is applied in the epilogue
+// without a second pass); the lanes of a group split K into 16-byte chunks
+// (8 bf16 / 16 int8 / 32 int4 weights) and stream them with 128-bit
+// L1-bypassing loads, U chunks per row in flight; the partial dot products
+// are reduced across the group with xor shuffles.  LG is chosen so that each
+// lane streams about 11 chunks of each row (K = 2816 or 704).
+#include "common.cuh"
+
+namespace moe {
+
+struct FfnParams {
+    LayerView L;
+    const uint16_t *x;            // [T][H] bf16
+    int T, k;
+    const int32_t *counts;        // [E]
+    const int32_t *offsets;       // [E+1]
+    const int32_t *sorted_route;  // [R]
+    uint16_t *h;                  // [R][I] bf16 (phase 1 out / phase 2 in)
+    float *rows;                  // [R][H] fp32
+    int lg;                       // lanes per row group (power of two, <= 32)
+};
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kNTM = 8;  // routes per work item
+
+template <int FMT> struct Fmt;
+template <> struct Fmt<MOE_W_BF16> { static constexpr int kElems = 8; };   // per 16-byte chunk
+template <> struct Fmt<MOE_W_INT8> { static constexpr int kElems = 16; };
+template <> struct Fmt<MOE_W_INT4> { static constexpr int kElems = 32; };
+
+__device__ __forceinline__ float gelu_tanh(float v) {
+    const float c = 0.7978845608028654f;  // sqrt(2/pi)
+    const float u = c * (v + 0.044715f * v * v * v);
+    return 0.5f * v * (1.0f + tanhf(u));
+}
+
+// Decode sub-plane sp (4 consecutive weights) of a 16-byte chunk into fp32.
+// bf16: words 2sp, 2sp+1.  int8: word sp, signed bytes (value + 128 placed in
+// the mantissa of 2^23, minus 2^23 + 128).  int4: half of word sp/2, nibbles
+// (n - 8) the same way (2^23 + n, minus 2^23 + 8).
+template <int FMT>
+__device__ __forceinline__ void decode4(const uint4 &q, int sp, float w[4]) {
+    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+    if (FMT == MOE_W_BF16) {
+        const uint32_t a = words[2 * sp], b = words[2 * sp + 1];
+        w[0] = bf16_lo(a); w[1] = bf16_hi(a); w[2] = bf16_lo(b); w[3] = bf16_hi(b);
+    } else if (FMT == MOE_W_INT8) {
+        const uint32_t a = words[sp] ^ 0x80808080u;
+        w[0] = __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7540)) - 8388736.0f;
+        w[1] = __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7541)) - 8388736.0f;
+        w[2] = __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7542)) - 8388736.0f;
+        w[3] = __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7543)) - 8388736.0f;
+    } else {
+        const uint32_t word = words[sp >> 1];
+        const uint32_t lo = word & 0x0F0F0F0Fu;          // nibbles 0,2,4,6 in bytes 0..3
+        const uint32_t hi = (word >> 4) & 0x0F0F0F0Fu;   // nibbles 1,3,5,7
+        if ((sp & 1) == 0) {
+            w[0] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7540)) - 8388616.0f;
+            w[1] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7540)) - 8388616.0f;
+            w[2] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7541)) - 8388616.0f;
+            w[3] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7541)) - 8388616.0f;
+        } else {
+            w[0] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7542)) - 8388616.0f;
+            w[1] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7542)) - 8388616.0f;
+            w[2] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7543)) - 8388616.0f;
+            w[3] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7543)) - 8388616.0f;
+        }
+    }
+}
+
+// Load the activations of the item's routes into shared memory as fp32.
+// Layout: xs[((t * SP + sp) * nchunks + c) * 4 + i] = x_t[c * kElems + 4 sp + i]
+// so that lanes reading consecutive chunks of one sub-plane hit consecutive
+// 16-byte words (no bank conflicts).
+template <int FMT, int PHASE>
+__device__ void load_acts(const FfnParams &p, float *xs, int row0, int nt, int K, int nchunks) {
+    constexpr int EC = Fmt<FMT>::kElems, SP = EC / 4;
+    const int per_t = K / 8;  // 8-element (16-byte bf16) pieces per route
+    for (int idx = threadIdx.x; idx < nt * per_t; idx += kThreads) {
+        const int t = idx / per_t, piece = idx - t * per_t;
+        const uint16_t *src;
+        if (PHASE == 1) {
+            const int tok = __ldg(p.sorted_route + row0 + t) / p.k;
+            src = p.x + (size_t)tok * p.L.H + (size_t)piece * 8;
+        } else {
+            src = p.h + (size_t)(row0 + t) * p.L.I + (size_t)piece * 8;
+        }
+        const uint4 u = *reinterpret_cast<const uint4 *>(src);
+        const int e0 = piece * 8;             // element index of the piece
+        const int c = e0 / EC, sp = (e0 % EC) / 4;
+        float4 *d0 = reinterpret_cast<float4 *>(xs + ((size_t)(t * SP + sp) * nchunks + c) * 4);
+        float4 *d1 = reinterpret_cast<float4 *>(xs + ((size_t)(t * SP + sp + 1) * nchunks + c) * 4);
+        *d0 = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+        *d1 = make_float4(bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w));
+    }
+}
+
+// One work item for one lane group: RWP rows x NT routes.
+template <int FMT, int PHASE, int RWP, int U, int NT>
+__device__ __forceinline__ void run_item(const FfnParams &p, const float *xs, const uint8_t *blob, int u0,
+                                         int row0, int nt, int K, int nchunks, int li, int lg) {
+    constexpr int EC = Fmt<FMT>::kElems, SP = EC / 4;
+    constexpr int UPG = PHASE == 1 ? RWP / 2 : RWP;  // units (pairs or rows) per group
+    const int I = p.L.I, H = p.L.H;
+    const int n_units = PHASE == 1 ? I : H;
+    const uint64_t qoff = PHASE == 1 ? p.L.off.q13 : p.L.off.q2;
+    const uint64_t soff = PHASE == 1 ? p.L.off.s13 : p.L.off.s2;
+    const size_t row_bytes = (size_t)nchunks * 16;
+
+    int row[RWP];
+    bool valid[RWP];
+#pragma unroll
+    for (int q = 0; q < RWP; ++q) {
+        const int unit = u0 + (PHASE == 1 ? q / 2 : q);
+        valid[q] = unit < n_units;
+        const int uu = valid[q] ? unit : 0;
+        row[q] = PHASE == 1 ? ((q & 1) ? I + uu : uu) : uu;
+    }
+    const uint8_t *qbase = blob + qoff;
+
+    float acc[RWP][NT];
+#pragma unroll
+    for (int q = 0; q < RWP; ++q)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[q][t] = 0.0f;
+
+    for (int c0 = li; c0 < nchunks; c0 += U * lg) {
+        uint4 wq[U][RWP];
+        float sc[U][RWP];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + u * lg;
+#pragma unroll
+            for (int q = 0; q < RWP; ++q) {
+                if (c < nchunks) {
+                    wq[u][q] = ld_stream_v4(qbase + (size_t)row[q] * row_bytes + (size_t)c * 16);
+                    if (FMT == MOE_W_INT4)
+                        sc[u][q] = bf16_to_f32(__ldg(reinterpret_cast<const uint16_t *>(blob + soff) +
+                                                     (size_t)row[q] * (K / 64) + (c >> 1)));
+                } else {
+                    wq[u][q] = make_uint4(0, 0, 0, 0);
+                    sc[u][q] = 0.0f;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + u * lg;
+            if (c >= nchunks) break;
+            if (FMT == MOE_W_INT4) {
+                float part[RWP][NT];
+#pragma unroll
+                for (int q = 0; q < RWP; ++q)
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) part[q][t] = 0.0f;
+#pragma unroll
+                for (int sp = 0; sp < SP; ++sp) {
+                    float w[RWP][4];
+#pragma unroll
+                    for (int q = 0; q < RWP; ++q) decode4<FMT>(wq[u][q], sp, w[q]);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        const float4 xv = *reinterpret_cast<const float4 *>(xs + ((size_t)(t * SP + sp) * nchunks + c) * 4);
+#pragma unroll
+                        for (int q = 0; q < RWP; ++q) {
+                            part[q][t] = fmaf(w[q][0], xv.x, part[q][t]);
+                            part[q][t] = fmaf(w[q][1], xv.y, part[q][t]);
+                            part[q][t] = fmaf(w[q][2], xv.z, part[q][t]);
+                            part[q][t] = fmaf(w[q][3], xv.w, part[q][t]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < RWP; ++q)
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) acc[q][t] = fmaf(sc[u][q], part[q][t], acc[q][t]);
+            } else {
+#pragma unroll
+                for (int sp = 0; sp < SP; ++sp) {
+                    float w[RWP][4];
+#pragma unroll
+                    for (int q = 0; q < RWP; ++q) decode4<FMT>(wq[u][q], sp, w[q]);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        const float4 xv = *reinterpret_cast<const float4 *>(xs + ((size_t)(t * SP + sp) * nchunks + c) * 4);
+#pragma unroll
+                        for (int q = 0; q < RWP; ++q) {
+                            acc[q][t] = fmaf(w[q][0], xv.x, acc[q][t]);
+                            acc[q][t] = fmaf(w[q][1], xv.y, acc[q][t]);
+                            acc[q][t] = fmaf(w[q][2], xv.z, acc[q][t]);
+                            acc[q][t] = fmaf(w[q][3], xv.w, acc[q][t]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // reduce across the lane group
+#pragma unroll
+    for (int q = 0; q < RWP; ++q)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            float v = acc[q][t];
+            for (int off = lg >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            acc[q][t] = v;
+        }
+    if (FMT == MOE_W_INT8) {
+#pragma unroll
+        for (int q = 0; q < RWP; ++q) {
+            const float s = __ldg(reinterpret_cast<const float *>(blob + soff) + row[q]);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) acc[q][t] *= s;
+        }
+    }
+
+    // epilogue: every lane of the group holds every sum; lane li writes the
+    // routes t with t % lg == li
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        if ((t & (lg - 1)) != li || t >= nt) continue;
+        const size_t srow = (size_t)(row0 + t);
+        if (PHASE == 1) {
+#pragma unroll
+            for (int q = 0; q < UPG; ++q) {
+                if (!valid[2 * q]) continue;
+                const float g = acc[2 * q][t], up = acc[2 * q + 1][t];
+                p.h[srow * I + (u0 + q)] = f32_to_bf16_rne(gelu_tanh(g) * up);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < RWP; ++q) {
+                if (!valid[q]) continue;
+                p.rows[srow * H + row[q]] = acc[q][t];
+            }
+        }
+    }
+}
+
+template <int FMT, int PHASE, int RWP, int U>
+__global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
+    constexpr int UPG = PHASE == 1 ? RWP / 2 : RWP;
+    constexpr int EC = Fmt<FMT>::kElems;
+    extern __shared__ __align__(16) float xs[];
+    __shared__ int s_act[kMaxE];
+    __shared__ int s_base[kMaxE + 1];
+    __shared__ int s_nact;
+
+    const int E = p.L.E;
+    const int K = PHASE == 1 ? p.L.H : p.L.I;
+    const int nchunks = K / EC;
+    const int lg = p.lg;
+    const int n_units = PHASE == 1 ? p.L.I : p.L.H;
+    const int groups = kWarps * (32 / lg);
+    const int upi = groups * UPG;              // units per item
+    const int tiles = (n_units + upi - 1) / upi;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    // active experts and the prefix of their item counts (one warp)
+    if (warp == 0) {
+        int n_act = 0, run = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int n = (e < E) ? __ldg(p.counts + e) : 0;
+            const bool act = n > 0;
+            const unsigned m = __ballot_sync(0xffffffffu, act);
+            const int items = act ? tiles * ((n + kNTM - 1) / kNTM) : 0;
+            int inc = items;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, off);
+                if (lane >= off) inc += v;
+            }
+            if (act) {
+                const int pos = n_act + __popc(m & ((1u << lane) - 1u));
+                s_act[pos] = e;
+                s_base[pos] = run + inc - items;
+            }
+            run += __shfl_sync(0xffffffffu, inc, 31);
+            n_act += __popc(m);
+        }
+        if (lane == 0) {
+            s_nact = n_act;
+            s_base[n_act] = run;
+        }
+    }
+    __syncthreads();
+    const int n_act = s_nact;
+    const int total = s_base[n_act];
+    const int it_begin = (int)(((long long)total * blockIdx.x) / gridDim.x);
+    const int it_end = (int)(((long long)total * (blockIdx.x + 1)) / gridDim.x);
+    if (it_begin >= it_end) return;
+
+    int a = 0;
+    {   // first active expert whose items reach it_begin
+        int lo = 0, hi = n_act - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_base[mid] <= it_begin) lo = mid; else hi = mid - 1;
+        }
+        a = lo;
+    }
+    const int li = lane & (lg - 1);
+    const int gi = warp * (32 / lg) + lane / lg;
+    int cur_key = -1;
+    for (int it = it_begin; it < it_end; ++it) {
+        while (s_base[a + 1] <= it) ++a;
+        const int rem = it - s_base[a];
+        const int chunk = rem / tiles, tile = rem - chunk * tiles;
+        const int e = s_act[a];
+        const int n_e = __ldg(p.counts + e);
+        const int row0 = __ldg(p.offsets + e) + chunk * kNTM;
+        const int nt = min(kNTM, n_e - chunk * kNTM);
+        const int key = a * 65536 + chunk;
+        if (key != cur_key) {
+            __syncthreads();
+            load_acts<FMT, PHASE>(p, xs, row0, nt, K, nchunks);
+            __syncthreads();
+            cur_key = key;
+        }
+        const uint8_t *blob = expert_blob(p.L, e);
+        const int u0 = tile * upi + gi * UPG;
+        if (nt > 4) run_item<FMT, PHASE, RWP, U, 8>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
+        else if (nt > 2) run_item<FMT, PHASE, RWP, U, 4>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
+        else if (nt > 1) run_item<FMT, PHASE, RWP, U, 2>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
+        else run_item<FMT, PHASE, RWP, U, 1>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
+    }
+}
+
+// Lanes per row group: the largest power of two <= 32 that leaves every lane
+// at least `min_per_lane` chunks of a row (so a group is never mostly idle).
+int pick_lg(int nchunks) {
+    int lg = 32;
+    while (lg > 1 && nchunks < lg * 8) lg >>= 1;
+    return lg;
+}
+
+template <int FMT, int PHASE, int RWP, int U>
+cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
+    FfnParams p = p0;
+    const int K = PHASE == 1 ? p.L.H : p.L.I;
+    const int nchunks = K / Fmt<FMT>::kElems;
+    p.lg = pick_lg(nchunks);
+    const size_t smem = (size_t)kNTM * K * sizeof(float);
+    auto kern = k_ffn_gemv<FMT, PHASE, RWP, U>;
+    // one-time set-up per device and shared-memory size (kept out of stream
+    // capture: after the first call a launch is the only API call made here)
+    static int cached_smem[kMaxDevices] = {}, cached_per_sm[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if ((size_t)cached_smem[dev] < smem) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        int per_sm = 0;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+        if (err != cudaSuccess) return err;
+        cached_per_sm[dev] = per_sm < 1 ? 1 : per_sm;
+        cached_smem[dev] = (int)smem;
+    }
+    const int per_sm = cached_per_sm[dev];
+    kern<<<n_sm * per_sm, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const FfnParams &p, int n_sm, cudaStream_t s) {
+    // rows per lane group: 2 (one gate/up pair in phase 1); U chunks
+    // of each row in flight, so a lane keeps 8 x 16 bytes of weights in flight
+    constexpr int RWP = 2;
+    constexpr int U = 8 / RWP;
+    cudaError_t err = launch_phase<FMT, 1, RWP, U>(p, n_sm, s);
+    if (err != cudaSuccess) return err;
+    return launch_phase<FMT, 2, RWP, U>(p, n_sm, s);
+}
+
+}  // namespace
+
+size_t ffn_gemv_workspace(int T, int k, int I) { return (size_t)T * k * I * sizeof(uint16_t); }
+
+cudaError_t launch_ffn_gemv(const LayerView &L, const uint16_t *x, int T, int k, const int32_t *counts,
+                            const int32_t *offsets, const int32_t *sorted_route, float *rows, void *ws,
+                            cudaStream_t s) {
+    int n_sm = 0;
+    cudaError_t err = sm_count(&n_sm);
+    if (err != cudaSuccess) return err;
+    FfnParams p{};
+    p.L = L;
+    p.x = x;
+    p.T = T;
+    p.k = k;
+    p.counts = counts;
+    p.offsets = offsets;
+    p.sorted_route = sorted_route;
+    p.h = static_cast<uint16_t *>(ws);
+    p.rows = rows;
+    if (L.fmt == MOE_W_BF16) return launch_fmt<MOE_W_BF16>(p, n_sm, s);
+    if (L.fmt == MOE_W_INT8) return launch_fmt<MOE_W_INT8>(p, n_sm, s);
+    return launch_fmt<MOE_W_INT4>(p, n_sm, s);
+}
+
+}  // namespace moe

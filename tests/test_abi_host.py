@@ -1,0 +1,145 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every symbol the
+header declares, rejects bad arguments before any launch, and its host-side
+placement calls match the oracle and the pages' vectors."""
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import moe_router_softmax_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"^MOE_API[^(]*?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    syms = header_symbols()
+    assert len(syms) >= 20
+    for s in syms:
+        assert hasattr(moe._lib, s), s
+    assert sorted(moe.EXPORTS) == syms
+
+
+def test_version_and_expert_bytes_match_oracle():
+    assert "sm_100a" in moe.moe_version()
+    for fmt in (0, 1, 2):
+        for H, I in [(2816, 704), (256, 128), (1024, 192)]:
+            assert moe.moe_expert_bytes(fmt, H, I) == oracle.expert_bytes(fmt, H, I)
+            assert moe.moe_blob_offsets(fmt, H, I) == oracle.blob_offsets(fmt, H, I)
+    assert moe.moe_expert_bytes(0, 100, 704) == 0
+
+
+def _null_layer(**kw):
+    import ctypes
+    c = moe._CLayer()
+    c.fmt, c.E, c.H, c.I = kw.get("fmt", 0), kw.get("E", 8), kw.get("H", 256), kw.get("I", 128)
+    c.home = kw.get("home", 256)
+    c.pool = kw.get("pool", None)
+    c.slot_table = kw.get("slot_table", None)
+    c.expert_bytes = kw.get("expert_bytes", moe.moe_expert_bytes(c.fmt, c.H, c.I))
+    return ctypes.byref(c)
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(E=0), "E=0"), (dict(E=2000), "E=2000"), (dict(H=100), "H=100"), (dict(I=96), "I=96"),
+    (dict(fmt=7), "format"), (dict(expert_bytes=1000), "expert_bytes"), (dict(home=8), "aligned"),
+    (dict(slot_table=256), "pool"),
+])
+def test_ffn_rejects_bad_layers_before_launch(args, frag):
+    st = moe._lib.moe_grouped_ffn(_null_layer(**args), 256, 4, 2, 256, 256, 256, 256, 256, 1 << 20, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    assert frag in moe.moe_last_error()
+
+
+def test_calls_reject_bad_shapes_and_null_pointers():
+    L = moe._lib
+    assert L.moe_route_topk(256, 4, 8, 9, 256, 256, None) == moe.MOE_ERR_INVALID_ARG   # k > E
+    assert "k=9" in moe.moe_last_error()
+    assert L.moe_route_topk(256, 4, 8, 33, 256, 256, None) == moe.MOE_ERR_INVALID_ARG  # k > 32
+    assert L.moe_route_topk(None, 4, 8, 2, 256, 256, None) == moe.MOE_ERR_INVALID_ARG  # NULL logits
+    assert L.moe_route_topk(256, -1, 8, 2, 256, 256, None) == moe.MOE_ERR_INVALID_ARG  # T < 0
+    assert L.moe_route_topk(256, 1 << 28, 128, 8, 256, 256, None) == moe.MOE_ERR_INVALID_ARG  # T*k overflow
+    assert L.moe_route_topk(None, 0, 8, 2, None, None, None) == moe.MOE_OK  # T == 0: no-op
+    assert L.moe_permute(None, 4, 2, 8, 256, 256, 256, 256, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_hits(256, 10, 0, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(256, 256, 256, 4, 2, 100, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(264, 256, 256, 4, 2, 128, 256, None) == moe.MOE_ERR_INVALID_ARG  # misaligned rows
+    assert L.moe_quantize_int4(256, 4, 100, 256, 256, None) == moe.MOE_ERR_INVALID_ARG  # K % 64
+    assert L.moe_pack_expert(1, 256, None, 256, None, 256, 128, 256, None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small
+    st = L.moe_grouped_ffn(_null_layer(), 256, 4, 2, 256, 256, 256, 256, 256, 16, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "workspace" in moe.moe_last_error()
+    # forcing an unknown path
+    st = L.moe_grouped_ffn_path(_null_layer(), 256, 4, 2, 256, 256, 256, 256, 256, 1 << 30, 9, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_queries():
+    lay = _null_layer(E=128, H=2816, I=704)
+    need = moe._lib.moe_grouped_ffn_workspace(lay, 64, 8)
+    assert need >= 64 * 8 * 704 * 2
+    fw = moe._lib.moe_layer_forward_workspace(lay, 64, 8)
+    assert fw >= need + 64 * 8 * 2816 * 4
+
+
+# ------------------------------------------------------------------ placement
+
+def test_placement_matches_page_vectors(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "expert_pool_vectors.json")))
+    c = g["target_gpu_picks_top_by_count"]
+    assert moe.moe_refresh_target(np.array(c["counts"]), c["budget"]).tolist() == c["target"]
+    c = g["paired_swap_limits_demotions"]
+    so = np.full(c["E"], -1, np.int32)
+    so[c["resident"]] = np.arange(len(c["resident"]))
+    so2, pr, de = moe.moe_apply_placement(so, c["budget"], np.array(c["target"]))
+    assert (len(pr), len(de)) == (c["promotions"], c["demotions"])
+    assert sorted(np.nonzero(so2 >= 0)[0].tolist()) == c["resident_after"]
+    c = g["paired_swap_keeps_extra_residents"]
+    so = np.full(c["E"], -1, np.int32)
+    so[c["resident"]] = np.arange(len(c["resident"]))
+    so2, pr, de = moe.moe_apply_placement(so, c["budget"], np.array(c["target"]))
+    assert (len(pr), len(de)) == (c["promotions"], c["demotions"])
+    assert int((so2 >= 0).sum()) == c["resident_count_after"]
+    c = g["jump_steps_refresh_schedule"]
+    for step, prefill, want in c["cases"]:
+        assert moe.moe_should_refresh(c["budget"] < c["E"], False, step, prefill, c["interval"]) == want
+    assert not moe.moe_should_refresh(False, True, 0, True, 1)   # no offload: never
+    c = g["vram_budget_formula"]
+    b = moe.moe_budget_from_vram(c["free_bytes"], c["reserve_bytes"], c["expert_bytes"], c["layers"],
+                                 c["max_per_layer"], c["E"])
+    assert 0 < b <= 128
+    assert moe.moe_budget_from_vram(1, 2, 0, 0, 300, 128) == 128
+
+
+def test_placement_matches_oracle_on_random_refreshes():
+    rng = np.random.default_rng(0)
+    for E, n_slots in [(128, 18), (16, 5), (8, 8)]:
+        so_a = np.full(E, -1, np.int32)
+        so_a[:n_slots] = np.arange(n_slots)
+        so_b = so_a.copy()
+        for _ in range(100):
+            hits = rng.integers(0, 6, size=E).astype(np.uint32) * (rng.random(E) < 0.6)
+            ta = moe.moe_refresh_target(hits, n_slots)
+            tb = oracle.refresh_target(hits, n_slots)
+            assert np.array_equal(ta, tb)
+            so_a, pa, da = moe.moe_apply_placement(so_a, n_slots, ta)
+            so_b, pb, db = oracle.apply_placement(so_b, n_slots, tb)
+            assert np.array_equal(so_a, so_b) and np.array_equal(pa, pb) and np.array_equal(da, db)
+
+
+def test_placement_rejects_bad_input():
+    with pytest.raises(moe.MoeError):
+        moe.moe_apply_placement(np.full(8, -1, np.int32), 2, np.array([1, 2, 3]))  # target > slots
+    with pytest.raises(moe.MoeError):
+        moe.moe_apply_placement(np.full(8, -1, np.int32), 4, np.array([1, 1]))  # duplicate
+    so = np.full(8, -1, np.int32)
+    so[[0, 1]] = 0
+    with pytest.raises(moe.MoeError):
+        moe.moe_apply_placement(so, 4, np.array([2]))  # slot held twice

@@ -1,0 +1,332 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Routing ids and weights, the permutation, hit counts and the int8/int4 codes are
+compared bit for bit; the FFN rows and the combined output by
+max|gpu - oracle| / max|oracle| <= 1e-2.  Small cases compare every element and
+span several work items and a ragged tail; the full Gemma-shaped layer (128
+experts, hidden 2816, intermediate 704, top-8) compares sampled routes and
+tokens that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as syn
+import moe_router_softmax_b200 as moe
+from gpu_support import (FFN_TOL, bf16_dev_to_f64, device_weights_from_host, host_bits, oracle_blob,
+                         oracle_layer_for, rel_err)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def bits_equal(a: np.ndarray, b: np.ndarray) -> bool:
+    return np.array_equal(np.ascontiguousarray(a).view(np.uint32), np.ascontiguousarray(b).view(np.uint32))
+
+
+# ---------------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("T,E,k,kind", [
+    (1, 128, 8, "normal"), (8, 128, 8, "normal"), (64, 128, 8, "biased"), (1024, 128, 8, "normal"),
+    (16, 8, 2, "normal"), (37, 1000, 32, "normal"), (5, 3, 3, "normal"), (33, 1024, 1, "zipf"),
+    (300, 64, 64 // 2, "zipf"), (7, 33, 5, "biased"),
+])
+def test_route_topk_bit_exact(T, E, k, kind):
+    lg = syn.router_logits(T, E, kind, seed=T + E)
+    ids, w = moe.moe_route_topk(torch.from_numpy(lg).to(DEV), k)
+    oi, ow = oracle.route_topk(lg, k)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    assert bits_equal(w.cpu().numpy(), ow)
+
+
+def test_route_topk_ties_nan_inf():
+    rng = np.random.default_rng(3)
+    lg = rng.integers(-2, 3, size=(100, 40)).astype(np.float32)
+    lg[0, :] = 0.0
+    lg[1, 5] = np.nan
+    lg[2, [1, 7]] = np.inf
+    lg[3, :] = -np.inf
+    lg[3, 9] = 1.0
+    lg[4, ::3] = -0.0
+    ids, w = moe.moe_route_topk(torch.from_numpy(lg).to(DEV), 6)
+    oi, ow = oracle.route_topk(lg, 6)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    g = w.cpu().numpy()
+    assert np.array_equal(np.isnan(g), np.isnan(ow))
+    fin = ~np.isnan(ow)
+    assert bits_equal(np.where(fin, g, 0), np.where(fin, ow, 0))
+
+
+# ---------------------------------------------------------------------- permute
+
+@pytest.mark.parametrize("T,k,E", [(1, 8, 128), (64, 8, 128), (1024, 8, 128), (16, 2, 8), (37, 3, 11),
+                                   (5000, 8, 1024), (3, 1, 1), (700, 32, 64)])
+def test_permute_and_hits_bit_exact(T, k, E):
+    rng = np.random.default_rng(T * k + E)
+    ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    bad = rng.random((T, k)) < 0.03
+    ids[bad] = rng.choice([-1, E, E + 5, -100], size=int(bad.sum()))
+    hits0 = rng.integers(0, 50, size=E).astype(np.uint32)
+    hits = torch.from_numpy(hits0.view(np.int32)).to(DEV)
+    out = moe.moe_permute(torch.from_numpy(ids).to(DEV), E, hits=hits)
+    ref = oracle.permute(ids, E)
+    for g, r in zip(out, ref):
+        assert np.array_equal(g.cpu().numpy(), r)
+    assert np.array_equal(hits.cpu().numpy().view(np.uint32), oracle.hits(ids, E, hits0))
+
+
+@pytest.mark.parametrize("n,E", [(1, 4), (5, 4), (100000, 128), (33333, 1024)])
+def test_expert_hits_bit_exact(n, E):
+    rng = np.random.default_rng(n)
+    ids = rng.integers(-3, E + 3, size=n).astype(np.int32)
+    h = torch.zeros(E, dtype=torch.int32, device=DEV)
+    moe.moe_expert_hits(torch.from_numpy(ids).to(DEV), E, h)
+    moe.moe_expert_hits(torch.from_numpy(ids).to(DEV), E, h)
+    assert np.array_equal(h.cpu().numpy().view(np.uint32), 2 * oracle.hits(ids, E))
+
+
+def test_hits_page_vector_on_gpu():
+    h = torch.zeros(4, dtype=torch.int32, device=DEV)
+    moe.moe_expert_hits(torch.tensor([1, 0, 1, 2, 1], dtype=torch.int32, device=DEV), 4, h)
+    assert h.cpu().tolist() == [1, 3, 1, 0]
+
+
+# ------------------------------------------------------------------- quantisers
+
+def _special_matrix(rows, K, seed):
+    w = syn.normal_bf16((rows, K), 0.02, seed, 9)
+    w[0] = 0                                         # all-zero row / groups
+    w[1, :64] = syn.bf16_bits(np.float32(np.arange(64) - 32) * np.float32(2.0 ** -8))
+    w[2, 5] = syn.bf16_bits(np.float32([0.9]))[0]     # outlier
+    w[3, 64:128] = syn.bf16_bits(np.float32([1e-3] * 63 + [-0.5]))
+    return w
+
+
+@pytest.mark.parametrize("rows,K", [(1408, 2816), (2816, 704), (64, 256), (3, 64)])
+def test_quantize_int8_bit_exact(rows, K):
+    w = _special_matrix(rows, K, rows)
+    q, s = moe.moe_quantize_int8(torch.from_numpy(w.view(np.int16)).to(DEV))
+    oq, os_ = oracle.quantize_int8(w)
+    assert np.array_equal(q.cpu().numpy(), oq)
+    assert bits_equal(s.cpu().numpy(), os_)
+
+
+@pytest.mark.parametrize("rows,K", [(1408, 2816), (2816, 704), (64, 256), (3, 64)])
+def test_quantize_int4_bit_exact(rows, K):
+    w = _special_matrix(rows, K, rows + 1)
+    q, s = moe.moe_quantize_int4(torch.from_numpy(w.view(np.int16)).to(DEV))
+    oq, os_ = oracle.quantize_int4(w)
+    assert np.array_equal(q.cpu().numpy(), oq)
+    assert np.array_equal(host_bits(s), os_)
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_packed_blobs_bit_exact(fmt):
+    E, H, I = 3, 512, 192
+    w13, w2 = syn.expert_weights(E, H, I, seed=5)
+    d13, d2 = device_weights_from_host(w13, w2)
+    L = moe.make_layer(fmt, d13, d2)
+    home = L.home.cpu().numpy()
+    eb = L.expert_bytes
+    for e in range(E):
+        assert np.array_equal(home[e * eb:(e + 1) * eb], oracle_blob(fmt, w13[e], w2[e], H, I))
+
+
+# ------------------------------------------------------------------ FFN, small
+
+def _run_layer(L, logits, x, k, path=moe.MOE_FFN_AUTO):
+    ids, w = moe.moe_route_topk(logits, k)
+    counts, offsets, sr, rp = moe.moe_permute(ids, L.E)
+    rows = moe.moe_grouped_ffn(L, x, k, counts, offsets, sr, path=path)
+    y = moe.moe_combine(rows, rp, w)
+    torch.cuda.synchronize()
+    return ids, w, counts, offsets, sr, rp, rows, y
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("E,H,I,k,T", [(8, 256, 128, 2, 16), (8, 512, 192, 3, 37), (6, 1024, 320, 2, 61),
+                                       (4, 256, 64, 4, 9)])
+def test_layer_small_every_element(fmt, E, H, I, k, T):
+    w13, w2 = syn.expert_weights(E, H, I, seed=E + H)
+    x = syn.activations(T, H, seed=7)
+    lg = syn.router_logits(T, E, "normal", seed=11)
+    d13, d2 = device_weights_from_host(w13, w2)
+    L = moe.make_layer(fmt, d13, d2)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    ids, w, counts, offsets, sr, rp, rows, y = _run_layer(L, torch.from_numpy(lg).to(DEV), xd, k)
+    OL = oracle_layer_for(fmt, w13, w2)
+    oi, ow, orows, oy = oracle.moe_layer(OL, lg, x, k)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    assert bits_equal(w.cpu().numpy(), ow)
+    rp_h = rp.cpu().numpy()
+    g_rows = rows.cpu().numpy()[rp_h]       # back to flat route order
+    assert rel_err(g_rows, orows) <= FFN_TOL
+    assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
+
+
+def test_layer_forward_single_call_matches_steps():
+    E, H, I, k, T = 8, 256, 128, 2, 16  # the tiny layer
+    w13, w2 = syn.expert_weights(E, H, I, seed=0)
+    x = syn.activations(T, H, seed=0)
+    lg = syn.router_logits(T, E, "normal", seed=0)
+    L = moe.make_layer(0, *device_weights_from_host(w13, w2))
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    lgd = torch.from_numpy(lg).to(DEV)
+    hits = torch.zeros(E, dtype=torch.int32, device=DEV)
+    y1 = moe.moe_layer_forward(L, lgd, xd, k, hits=hits)
+    y2 = _run_layer(L, lgd, xd, k)[-1]
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    oi, ow, orows, oy = oracle.moe_layer(oracle_layer_for(0, w13, w2), lg, x, k)
+    assert rel_err(bf16_dev_to_f64(y1), oy) <= FFN_TOL
+    assert np.array_equal(hits.cpu().numpy().view(np.uint32), oracle.hits(oi, E))
+
+
+def test_slot_table_changes_where_not_what():
+    """Router logits and ids are unchanged by placement (expert_pool.rs, module
+    doc): the same layer served partly from cache slots gives bit-identical ids,
+    weights, rows and output."""
+    E, H, I, k, T = 16, 512, 128, 4, 40
+    w13, w2 = syn.expert_weights(E, H, I, seed=2)
+    L = moe.make_layer(2, *device_weights_from_host(w13, w2))
+    eb = L.expert_bytes
+    slot_of = np.full(E, -1, np.int32)
+    slot_of[[3, 9, 0, 15, 7]] = [4, 0, 2, 1, 3]
+    pool = torch.zeros(5 * eb, dtype=torch.uint8, device=DEV)
+    moe.moe_copy_to_slots(L.home, pool, eb, np.nonzero(slot_of >= 0)[0], slot_of[slot_of >= 0])
+    L2 = moe.MoeLayer(2, E, H, I, L.home, pool=pool, slot_table=torch.from_numpy(slot_of).to(DEV))
+    x = torch.from_numpy(syn.activations(T, H, seed=1).view(np.int16)).to(DEV).view(torch.bfloat16)
+    lg = torch.from_numpy(syn.router_logits(T, E, "zipf", seed=1)).to(DEV)
+    a = _run_layer(L, lg, x, k)
+    b = _run_layer(L2, lg, x, k)
+    for u, v in zip(a, b):
+        assert torch.equal(u.view(torch.int32) if u.dtype == torch.float32 else u, v.view(torch.int32) if v.dtype == torch.float32 else v)
+    # the pool really is what is read: wipe the home blobs of slotted experts
+    home2 = L.home.clone()
+    for e in np.nonzero(slot_of >= 0)[0]:
+        home2[e * eb:(e + 1) * eb] = 0
+    L3 = moe.MoeLayer(2, E, H, I, home2, pool=pool, slot_table=torch.from_numpy(slot_of).to(DEV))
+    c = _run_layer(L3, lg, x, k)
+    assert torch.equal(a[-1].view(torch.int16), c[-1].view(torch.int16))
+
+
+def test_empty_batch_and_dropped_routes():
+    E, H, I, k = 8, 256, 128, 2
+    w13, w2 = syn.expert_weights(E, H, I, seed=4)
+    L = moe.make_layer(0, *device_weights_from_host(w13, w2))
+    # T == 0 is a no-op everywhere
+    x0 = torch.empty((0, H), dtype=torch.bfloat16, device=DEV)
+    y0 = moe.moe_layer_forward(L, torch.empty((0, E), device=DEV), x0, k)
+    assert y0.shape == (0, H)
+    # routes with ids outside [0, E) are dropped from the groups and from the sum
+    T = 6
+    x = syn.activations(T, H, seed=4)
+    ids = np.array([[0, 3], [9, 1], [2, -1], [5, 5 + 8], [7, 6], [-4, 4]], np.int32)
+    w = np.full((T, k), 0.5, np.float32)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    counts, offsets, sr, rp = moe.moe_permute(torch.from_numpy(ids).to(DEV), E)
+    rows = moe.moe_grouped_ffn(L, xd, k, counts, offsets, sr)
+    y = moe.moe_combine(rows, rp, torch.from_numpy(w).to(DEV))
+    OL = oracle_layer_for(0, w13, w2)
+    orows = oracle.ffn_routes(OL, x, ids)
+    oy = oracle.combine(orows, ids, w, E)
+    assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
+    assert int(offsets[-1]) == int((ids >= 0).sum() - ((ids >= E).sum()))
+
+
+def test_one_expert_takes_every_token():
+    """Degenerate routing: every token routes to the same k experts (k = E)."""
+    E, H, I, T = 4, 256, 128, 70
+    w13, w2 = syn.expert_weights(E, H, I, seed=8)
+    for fmt in (0, 2):
+        L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
+        x = syn.activations(T, H, seed=8)
+        lg = syn.router_logits(T, E, "normal", seed=8)
+        ids, w, counts, offsets, sr, rp, rows, y = _run_layer(
+            L, torch.from_numpy(lg).to(DEV), torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16), E)
+        assert counts.cpu().tolist() == [T] * E
+        oi, ow, orows, oy = oracle.moe_layer(oracle_layer_for(fmt, w13, w2), lg, x, E)
+        assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
+
+
+# ------------------------------------------------------- FFN, Gemma-shaped layer
+
+_FULL = {}
+
+
+def _full_layer(fmt):
+    """128 experts, hidden 2816, intermediate 704: weights drawn on the device by a
+    seeded torch generator; the oracle reads the bf16 bytes back per expert."""
+    if fmt not in _FULL:
+        E, H, I = 128, 2816, 704
+        w13, w2 = syn.torch_expert_weights(E, H, I, seed=0, layer=0, device=DEV)
+        L = moe.make_layer(fmt, w13, w2)
+        _FULL.clear()
+        _FULL[fmt] = (w13, w2, L)
+    return _FULL[fmt]
+
+
+@pytest.mark.parametrize("fmt,kind", [(0, "normal"), (1, "biased"), (2, "normal")])
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_gemma_layer_decode_sampled(fmt, kind, T):
+    E, H, I, k = 128, 2816, 704, 8
+    w13, w2, L = _full_layer(fmt)
+    x = syn.activations(T, H, seed=100 + T)
+    lg = syn.router_logits(T, E, kind, seed=200 + T)
+    ids, w, counts, offsets, sr, rp, rows, y = _run_layer(
+        L, torch.from_numpy(lg).to(DEV), torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16), k)
+    oi, ow = oracle.route_topk(lg, k)
+    assert np.array_equal(ids.cpu().numpy(), oi) and bits_equal(w.cpu().numpy(), ow)
+    for g, r in zip((counts, offsets, sr, rp), oracle.permute(oi, E)):
+        assert np.array_equal(g.cpu().numpy(), r)
+    # sample tokens (all their k routes) for the oracle
+    rng = np.random.default_rng(T)
+    toks = np.unique(np.r_[0, T - 1, rng.integers(0, T, size=min(T, 3))])
+    routes = np.concatenate([np.arange(t * k, (t + 1) * k) for t in toks]).astype(np.int32)
+    experts = oi.ravel()[routes]
+    h13 = {e: host_bits(w13[e]) for e in set(experts.tolist())}
+    h2 = {e: host_bits(w2[e]) for e in set(experts.tolist())}
+    w13h = np.zeros((E, 2, H), np.uint16)  # placeholder shape; only sampled experts are packed
+    OL = _sparse_oracle_layer(fmt, E, H, I, h13, h2)
+    orows = oracle.ffn_some_routes(OL, x, oi, routes)
+    g_rows = rows.cpu().numpy()[rp.cpu().numpy()[routes]]
+    assert rel_err(g_rows, orows) <= FFN_TOL
+    full_rows = np.zeros((T * k, H))
+    full_rows[routes] = orows
+    oy = oracle.combine(full_rows, oi, ow, E)[toks]
+    assert rel_err(bf16_dev_to_f64(y)[toks], oy) <= FFN_TOL
+    del w13h
+
+
+def _sparse_oracle_layer(fmt, E, H, I, h13, h2):
+    eb = oracle.expert_bytes(fmt, H, I)
+    slot = np.full(E, -1, np.int32)
+    ex = sorted(h13)
+    pool = np.zeros(len(ex) * eb, np.uint8)
+    for i, e in enumerate(ex):
+        slot[e] = i
+        pool[i * eb:(i + 1) * eb] = oracle_blob(fmt, h13[e], h2[e], H, I)
+    return oracle.Layer(fmt, E, H, I, np.zeros(eb, np.uint8), pool=pool, slot_table=slot)
+
+
+def test_gemma_layer_prefill_sampled():
+    """int4 layer, 1024 tokens (the prefill batch): sampled routes and tokens."""
+    E, H, I, k, T = 128, 2816, 704, 8, 1024
+    w13, w2, L = _full_layer(2)
+    x = syn.activations(T, H, seed=5)
+    lg = syn.router_logits(T, E, "normal", seed=5)
+    ids, w, counts, offsets, sr, rp, rows, y = _run_layer(
+        L, torch.from_numpy(lg).to(DEV), torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16), k)
+    oi, ow = oracle.route_topk(lg, k)
+    assert np.array_equal(ids.cpu().numpy(), oi) and bits_equal(w.cpu().numpy(), ow)
+    toks = np.array([0, 1, 511, 1023])
+    routes = np.concatenate([np.arange(t * k, (t + 1) * k) for t in toks]).astype(np.int32)
+    experts = sorted(set(oi.ravel()[routes].tolist()))
+    OL = _sparse_oracle_layer(2, E, H, I, {e: host_bits(w13[e]) for e in experts}, {e: host_bits(w2[e]) for e in experts})
+    orows = oracle.ffn_some_routes(OL, x, oi, routes)
+    assert rel_err(rows.cpu().numpy()[rp.cpu().numpy()[routes]], orows) <= FFN_TOL
+    full_rows = np.zeros((T * k, H))
+    full_rows[routes] = orows
+    oy = oracle.combine(full_rows, oi, ow, E)[toks]
+    assert rel_err(bf16_dev_to_f64(y)[toks], oy) <= FFN_TOL

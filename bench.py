@@ -45,7 +45,10 @@ import numpy as np  # noqa: E402
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # grouped-FFN kernels from one ncu capture, per workload; None until captured
 # for the kernels as they stand (see profiles/).
-NCU_TRAFFIC_BYTES = {}
+NCU_TRAFFIC_BYTES = {
+    # profiles/ffn_gemv_bf16_T64.md: phase 1 1.0059 GB + 4.04 MB, phase 2 0.5027 GB + 5.28 MB
+    ("decode-bf16", 64): 1.5180e9,
+}
 
 CONFIGS = {
     # name: (weight format, logits kind, tokens, extra batches swept)
@@ -68,6 +71,7 @@ def parse():
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--quick", action="store_true", help="main batch only: no sweep, no e2e, no CPU baseline")
     return ap.parse_args()
 
 
@@ -398,7 +402,7 @@ def main():
     layer_bytes = avg_distinct * eb + T * H * 2 * 2 + T * E * 4
 
     sweep_out = {}
-    for Ts in sweep:
+    for Ts in ([] if args.quick else sweep):
         b2 = make_batches(torch, kind, Ts, E, H, 8, dev, seed=Ts)
         r2 = Runner(moe, torch, layers, b2, Ts, k, dev)
         d2 = r2.distinct_experts()
@@ -418,14 +422,15 @@ def main():
             "ffn_frac_of_hbm": round((dd * eb + Ts * H * 2) / (f2 / 1e3) / 1e9 / hbm_peak, 4),
         }
 
-    e2e_ms, h2d, d2h = time_e2e(torch, moe, layers, batches, T, k, args.steps, args.warmup, dev)
+    e2e_ms, h2d, d2h = (float("nan"), 0, 0) if args.quick else time_e2e(torch, moe, layers, batches, T, k,
+                                                                         args.steps, args.warmup, dev)
     if dist is not None:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
         cpu = cpu_baseline(moe, torch, fmt_name, layers, batches, T, k, args.cpu_seconds)
 
     line = {

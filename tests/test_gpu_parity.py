@@ -99,7 +99,8 @@ def _special_matrix(rows, K, seed):
     w[0] = 0                                         # all-zero row / groups
     w[1, :64] = syn.bf16_bits(np.float32(np.arange(64) - 32) * np.float32(2.0 ** -8))
     w[2, 5] = syn.bf16_bits(np.float32([0.9]))[0]     # outlier
-    w[3, 64:128] = syn.bf16_bits(np.float32([1e-3] * 63 + [-0.5]))
+    if rows > 3 and K >= 128:
+        w[3, 64:128] = syn.bf16_bits(np.float32([1e-3] * 63 + [-0.5]))
     return w
 
 

@@ -167,6 +167,25 @@ MOE_API moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *
                                 int32_t path, moe_stream_t stream);
 
 /*
+ * Grouped FFN without a caller-provided workspace, for callers that cannot
+ * allocate device memory (a plugin or serving runtime that passes the library
+ * only its input and output buffers, or a loop that must never call
+ * cudaMalloc).  Same arguments and results as moe_grouped_ffn, minus ws.  The
+ * pages have no counterpart: this is a library convenience.
+ * Scratch: a fixed 16 MiB device array inside the library, reserved on every
+ * GPU that loads it until the process exits.  Calls needing more
+ * (moe_grouped_ffn_workspace() > 16 MiB, i.e. T*k*I*2 bytes) are rejected with
+ * MOE_ERR_INVALID_ARG before any launch.  The first call on a device looks up
+ * the array's device address (once per device, that device current); make that
+ * first call before any stream capture.  Every call shares the array and leaves
+ * its contents behind; calls that overlap on the GPU race on it.  No
+ * allocation is made by this call.
+ */
+MOE_API moe_status moe_grouped_ffn_noalloc(const moe_layer *layer, const uint16_t *x, int32_t T, int32_t k,
+                                           const int32_t *counts, const int32_t *offsets,
+                                           const int32_t *sorted_route, float *rows, moe_stream_t stream);
+
+/*
  * Weighted combine back to token order (remote_experts.cpp,
  * RemoteExperts::finish copies each row back to its route's position; the
  * weighting is the router's):  y[t] = sum_{j<k} w[t][j] * rows[route_pos[t*k+j]]

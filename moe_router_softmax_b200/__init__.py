@@ -35,7 +35,7 @@ EXPORTS = [
     "moe_expert_hits", "moe_grouped_ffn_workspace", "moe_grouped_ffn", "moe_grouped_ffn_path", "moe_combine",
     "moe_layer_forward_workspace", "moe_layer_forward", "moe_quantize_int8", "moe_quantize_int4",
     "moe_pack_expert", "moe_copy_to_slots", "moe_refresh_target", "moe_apply_placement",
-    "moe_should_refresh", "moe_budget_from_vram",
+    "moe_should_refresh", "moe_budget_from_vram", "moe_grouped_ffn_noalloc",
 ]
 
 
@@ -77,6 +77,7 @@ _SIG = {
     "moe_apply_placement": (i32, [P, i32, i32, P, i32, P, P, P, P]),
     "moe_should_refresh": (i32, [i32, i32, i64, i32, i64]),
     "moe_budget_from_vram": (i64, [i64, i64, i64, i64, i64, i64]),
+    "moe_grouped_ffn_noalloc": (i32, [LP, P, i32, i32, P, P, P, P, P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -307,6 +308,20 @@ def moe_should_refresh(offload_enabled: bool, mode_refresh: bool, step: int, is_
 
 def moe_budget_from_vram(free_bytes, reserve_bytes, expert_bytes, layers, max_per_layer, E) -> int:
     return int(_lib.moe_budget_from_vram(free_bytes, reserve_bytes, expert_bytes, layers, max_per_layer, E))
+
+
+def moe_grouped_ffn_noalloc(layer: MoeLayer, x: torch.Tensor, k: int, counts, offsets, sorted_route,
+                            rows: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """moe_grouped_ffn for callers that cannot allocate: the library's fixed
+    16 MiB device scratch replaces the workspace (see include/moe.h)."""
+    T = x.shape[0]
+    if rows is None:
+        rows = torch.empty((max(T * k, 1), layer.H), dtype=torch.float32, device=x.device)
+    _check(_lib.moe_grouped_ffn_noalloc(layer.ref(), _dev(x, BF16, "x"), T, k, _dev(counts, torch.int32, "counts"),
+                                        _dev(offsets, torch.int32, "offsets"),
+                                        _dev(sorted_route, torch.int32, "sorted_route"),
+                                        _dev(rows, torch.float32, "rows"), _stream(stream)))
+    return rows
 
 
 # ------------------------------------------------------------------ helpers

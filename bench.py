@@ -47,7 +47,7 @@ import numpy as np  # noqa: E402
 # for the kernels as they stand (see profiles/).
 NCU_TRAFFIC_BYTES = {
     # profiles/ffn_gemv_bf16_T64.md: phase 1 1.0059 GB + 4.04 MB, phase 2 0.5027 GB + 5.28 MB
-    ("decode-bf16", 64): 1.5180e9,
+    ("decode-bf16", 64, "gemv"): 1.5180e9,
 }
 
 CONFIGS = {
@@ -72,6 +72,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--quick", action="store_true", help="main batch only: no sweep, no e2e, no CPU baseline")
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"],
+                    help="grouped-FFN kernels: AUTO picks by routes per call")
     return ap.parse_args()
 
 
@@ -136,11 +138,13 @@ class ClockSampler:
 # --------------------------------------------------------------- workload
 
 def measured_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 def build_layers(moe, torch, fmt_name, E, H, I, n_layers, dev, seed=0):
@@ -185,8 +189,9 @@ def make_batches(torch, kind, T, E, H, n, dev, seed=0):
 class Runner:
     """Device buffers for one batch size; step(i) runs the layer on batch i."""
 
-    def __init__(self, moe, torch, layers, batches, T, k, dev):
+    def __init__(self, moe, torch, layers, batches, T, k, dev, path=0):
         self.moe, self.torch, self.layers, self.batches, self.T, self.k = moe, torch, layers, batches, T, k
+        self.path = path
         E, H = layers[0].E, layers[0].H
         R = T * k
         i32 = torch.int32
@@ -209,12 +214,17 @@ class Runner:
         counts, offsets, sr, rp = moe.moe_permute(self.ids, L.E, hits=self.hits[li], out=self.perm)
         if ffn_events is not None:
             ffn_events[0].record()
-        moe.moe_grouped_ffn(L, x, self.k, counts, offsets, sr, rows=self.rows, ws=self.ws)
+        moe.moe_grouped_ffn(L, x, self.k, counts, offsets, sr, rows=self.rows, ws=self.ws, path=self.path)
         if ffn_events is not None:
             ffn_events[1].record()
         moe.moe_combine(self.rows, rp, self.w, self.y)
 
-    LAUNCHES_PER_STEP = 5  # route, permute, FFN phase 1, FFN phase 2, combine
+    def launches_per_step(self):
+        """route, permute, FFN (2 GEMV launches, or gather + 2 tensor-core launches), combine"""
+        R = self.T * self.k
+        auto_tc = R >= (65 if self.layers[0].fmt == self.moe.MOE_W_INT4 else 32)
+        tc = self.path == self.moe.MOE_FFN_TC or (self.path == self.moe.MOE_FFN_AUTO and auto_tc)
+        return 4 + (3 if tc else 2)
 
     def distinct_experts(self):
         """Distinct routed experts of each batch (read back from our own routing)."""
@@ -376,7 +386,8 @@ def main():
     n_layers = args.layers if args.config != "tiny" else 2
     layers = build_layers(moe, torch, fmt_name, E, H, I, n_layers, dev)
     batches = make_batches(torch, kind, T, E, H, 8, dev)
-    runner = Runner(moe, torch, layers, batches, T, k, dev)
+    path = {"auto": moe.MOE_FFN_AUTO, "gemv": moe.MOE_FFN_GEMV, "tc": moe.MOE_FFN_TC}[args.path]
+    runner = Runner(moe, torch, layers, batches, T, k, dev, path)
     distinct = runner.distinct_experts()
 
     clocks = ClockSampler(local)
@@ -397,14 +408,17 @@ def main():
     alg_bytes = avg_distinct * eb + T * H * 2
     ffn_avg_ms = sum(ffn_ms) / len(ffn_ms)
     achieved = alg_bytes / (ffn_avg_ms / 1e3) / 1e9
-    hbm_peak, tf_peak, peak_src = measured_peaks()
-    traffic = NCU_TRAFFIC_BYTES.get((args.config, T))
+    hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
+    flops = 2.0 * T * k * 3 * H * I
+    tflops = flops / (ffn_avg_ms / 1e3) / 1e12
+    tensor_bound = T > 64
+    traffic = NCU_TRAFFIC_BYTES.get((args.config, T, args.path))
     layer_bytes = avg_distinct * eb + T * H * 2 * 2 + T * E * 4
 
     sweep_out = {}
     for Ts in ([] if args.quick else sweep):
         b2 = make_batches(torch, kind, Ts, E, H, 8, dev, seed=Ts)
-        r2 = Runner(moe, torch, layers, b2, Ts, k, dev)
+        r2 = Runner(moe, torch, layers, b2, Ts, k, dev, path)
         d2 = r2.distinct_experts()
         ms2, ffn2 = time_steps(torch, r2, args.steps, args.warmup, dist)
         if dist is not None:
@@ -448,6 +462,7 @@ def main():
         "data": "synthetic (seeded; Gemma-4-26B-A4B-shaped layer, random weights)",
         "config": {
             "workload": f"moe-layer-{fmt_name}-{'prefill' if T > 64 else 'decode'}-T{T}",
+            "ffn_path": args.path,
             "experts": E, "hidden": H, "intermediate": I, "top_k": k, "tokens": T,
             "weights": fmt_name, "logits": kind, "layers_rotated": n_layers,
             "l2": f"inputs larger than L2: each step reads a different one of {n_layers} layer copies "
@@ -455,9 +470,21 @@ def main():
             "parallelism": f"replicas x{world}",
         },
         "layer_hbm_gbs": round(layer_bytes / (ms_step / 1e3) / 1e9, 1),
-        "roofline": {
+        "roofline": ({
+            "bound": "tensor",
+            "kernel": "grouped FFN on tcgen05 (gather, w13+GELU gate, w2; 3 launches)",
+            "achieved": round(tflops, 1),
+            "peak": tf_sust,
+            "peak_source": f"{peak_src} sustained bf16 (MEASURED_PEAKS.json bf16_tflops_sustained)",
+            "unit": "TFLOP/s",
+            "frac": round(tflops / tf_sust, 4),
+            "traffic": traffic,
+            "alg_flops_per_launch": flops,
+            "hbm": {"achieved_gbs": round(achieved, 1), "peak": hbm_peak, "frac": round(achieved / hbm_peak, 4)},
+            "avg_launch_us": round(ffn_avg_ms * 1e3, 2),
+        } if tensor_bound else {
             "bound": "hbm",
-            "kernel": "grouped FFN (w13+GELU gate, then w2; 2 launches)",
+            "kernel": "grouped FFN (tcgen05: gather, w13+GELU gate, w2; GEMV: w13+GELU gate, w2)",
             "achieved": round(achieved, 1),
             "peak": hbm_peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
@@ -466,11 +493,11 @@ def main():
             "traffic": traffic,
             "alg_bytes_per_launch": int(alg_bytes),
             "avg_launch_us": round(ffn_avg_ms * 1e3, 2),
-        },
+        }),
         "sweep": sweep_out,
         "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": Runner.LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": runner.launches_per_step() * args.steps,
         "clocks": clk,
         "cpu_baseline": cpu,
     }

@@ -19,7 +19,7 @@ size_t ffn_gemv_workspace(int T, int k, int I);
 cudaError_t launch_ffn_gemv(const LayerView &, const uint16_t *, int, int, const int32_t *, const int32_t *,
                             const int32_t *, float *, void *, cudaStream_t);
 size_t ffn_tc_workspace(int T, int k, int E, int H, int I);
-bool ffn_tc_supports(int fmt, int H, int I);
+bool ffn_tc_supports(int fmt, int H, int I, uint64_t stride);
 cudaError_t launch_ffn_tc(const LayerView &, const uint16_t *, int, int, const int32_t *, const int32_t *,
                           const int32_t *, float *, void *, cudaStream_t);
 
@@ -161,15 +161,22 @@ moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *x, int32
     if (T == 0) return MOE_OK;
     CHECK_ARG(x && counts && offsets && sorted_route && rows && ws, "moe_grouped_ffn: NULL pointer");
     CHECK_ARG(aligned16(x) && aligned16(rows) && aligned16(ws), "x, rows and ws must be 16-byte aligned");
-    const size_t need = moe_grouped_ffn_workspace(layer, T, k);
-    CHECK_ARG(ws_bytes >= need, "workspace %zu bytes < %zu needed", ws_bytes, need);
     const int R = T * k;
     int use = path;
-    if (use == MOE_FFN_AUTO) use = (R > 1024 && ffn_tc_supports(v.fmt, v.H, v.I)) ? MOE_FFN_TC : MOE_FFN_GEMV;
+    if (use == MOE_FFN_AUTO) {
+        // measured on B200 (Gemma-shaped layer): the tensor-core kernels win from
+        // 4 tokens x top-8 for bf16/int8 weights and above 8 tokens for int4; one
+        // token stays on the GEMV kernels
+        const int min_routes = v.fmt == MOE_W_INT4 ? 65 : 32;
+        use = (R >= min_routes && ffn_tc_supports(v.fmt, v.H, v.I, v.stride)) ? MOE_FFN_TC : MOE_FFN_GEMV;
+    }
+    if (use == MOE_FFN_TC && !ffn_tc_supports(v.fmt, v.H, v.I, v.stride))
+        return set_error(MOE_ERR_UNSUPPORTED, "tensor-core path does not handle format %d at H=%d I=%d stride=%llu",
+                         v.fmt, v.H, v.I, (unsigned long long)v.stride);
+    // the workspace the chosen path needs (moe_grouped_ffn_workspace() covers both)
+    const size_t need = align256(use == MOE_FFN_TC ? ffn_tc_workspace(T, k, v.E, v.H, v.I) : ffn_gemv_workspace(T, k, v.I));
+    CHECK_ARG(ws_bytes >= need, "workspace %zu bytes < %zu needed", ws_bytes, need);
     if (use == MOE_FFN_TC) {
-        if (!ffn_tc_supports(v.fmt, v.H, v.I))
-            return set_error(MOE_ERR_UNSUPPORTED, "tensor-core path does not handle format %d at H=%d I=%d",
-                             v.fmt, v.H, v.I);
         return cuda_status(launch_ffn_tc(v, x, T, k, counts, offsets, sorted_route, rows, ws, (cudaStream_t)stream),
                            "moe_grouped_ffn (tensor-core) launch");
     }

@@ -19,6 +19,10 @@
 
 #include "common.cuh"
 
+namespace moe {
+size_t ffn_gemv_workspace(int T, int k, int I);
+}
+
 namespace {
 
 // 16 MiB: the bf16 intermediate of T*k routes must fit, T*k*I*2 bytes
@@ -63,7 +67,8 @@ moe_status moe_grouped_ffn_noalloc(const moe_layer *layer, const uint16_t *x, in
                                    float *rows, moe_stream_t stream) {
     if (layer == nullptr) return moe::set_error(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_noalloc: layer is NULL");
     if (T < 0 || k < 1) return moe::set_error(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_noalloc: T=%d k=%d", T, k);
-    const size_t need = moe_grouped_ffn_workspace(layer, T, k);
+    // the GEMV kernels' scratch: the bf16 intermediate, T*k*I*2 bytes
+    const size_t need = moe::ffn_gemv_workspace(T, k, layer->I);
     if (need > kNoAllocScratchBytes)
         return moe::set_error(MOE_ERR_INVALID_ARG,
                               "moe_grouped_ffn_noalloc: T*k=%lld routes at I=%d need %zu bytes of scratch; the fixed "
@@ -72,8 +77,8 @@ moe_status moe_grouped_ffn_noalloc(const moe_layer *layer, const uint16_t *x, in
     void *scratch = nullptr;
     moe_status st = scratch_for_current_device(&scratch);
     if (st != MOE_OK) return st;
-    return moe_grouped_ffn(layer, x, T, k, counts, offsets, sorted_route, rows, scratch, kNoAllocScratchBytes,
-                           stream);
+    return moe_grouped_ffn_path(layer, x, T, k, counts, offsets, sorted_route, rows, scratch, kNoAllocScratchBytes,
+                                MOE_FFN_GEMV, stream);
 }
 
 }  // extern "C"

@@ -1,15 +1,688 @@
-// ffn_tc.cu -- grouped gated FFN on the tcgen05 tensor cores (prefill-sized
-// batches).  Placeholder until the tensor-core kernels land: the path reports
-// itself unsupported, so MOE_FFN_AUTO keeps every call on the GEMV kernels.
+// ffn_tc.cu -- grouped gated FFN on the 5th-generation tensor cores
+// (tcgen05.mma, accumulators in TMEM, operands staged in shared memory by TMA).
+//
+// The same two steps as the GEMV path (gated GELU-tanh FFN, w13 gate rows
+// [0,I) and up rows [I,2I), then w2), as ragged grouped GEMMs with the weight
+// rows as the M = 128 operand ("swap AB") and each expert's routes as N:
+//   phase 1:  D[128 x N] = [W13 gate rows i0..i0+63 ; up rows i0..i0+63] . Xs^T
+//             epilogue h[s][i] = bf16(gelu_tanh(D[i]) * D[64 + i])
+//   phase 2:  D[128 x N] = W2[m0..m0+127] . h^T,   epilogue rows[s][m] = D[m]
+// Xs is x gathered into sorted-route order (k_gather_rows), so every B tile is
+// a plain 2-D TMA box.  For bf16 weights TMA writes the A tile straight into
+// the 128-byte-swizzled K-major layout the MMA reads; int8/int4 tiles land raw
+// and eight dequant warps expand them into that layout (int8 codes exactly,
+// with the per-row scale applied in the epilogue; int4 as bf16(q * s) with
+// the group scale, one rounding), so dequantisation is fused into the
+// shared-memory stage.
+//
+// One persistent CTA per SM; warp roles:
+//   warp 0      TMA producer (A weights or raw codes, B activations)
+//   warp 1      TMEM allocation and the single-thread MMA issuer
+//   warps 2..5  epilogue (TMEM -> registers -> global); warp w reads TMEM
+//               lanes 32*(w%4) .. +31
+//   warps 6..13 dequantisation (int8 / int4 only)
+// Pipelines: a ring of kStages shared-memory stages (full / dequantised /
+// empty mbarriers) and two TMEM accumulators (full / empty) so the epilogue of
+// one item overlaps the main loop of the next.  Every mbarrier wait is bounded;
+// on timeout the kernel records an error word and every role drains out.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
+namespace {
 
-size_t ffn_tc_workspace(int, int, int, int, int) { return 0; }
-bool ffn_tc_supports(int, int, int) { return false; }
-cudaError_t launch_ffn_tc(const LayerView &, const uint16_t *, int, int, const int32_t *, const int32_t *,
-                          const int32_t *, float *, void *, cudaStream_t) {
-    return cudaErrorNotSupported;
+constexpr int kBlockM = 128;          // weight rows per tile (TMEM lanes)
+constexpr int kBlockK = 64;           // bf16 elements per stage = one 128-byte swizzle row
+constexpr int kNMax = 128;            // routes per accumulator (TMEM columns)
+constexpr int kAccBufs = 2;
+constexpr int kTmemCols = kNMax * kAccBufs;
+constexpr int kEpiWarps = 4;
+constexpr int kDeqWarps = 8;   // two threads per tile row, half a row each
+constexpr uint32_t kATileBytes = kBlockM * kBlockK * 2;   // 16 KB
+constexpr uint32_t kBTileBytes = kNMax * kBlockK * 2;     // 16 KB
+constexpr long long kWaitCycles = 4000000000ll;           // ~2 s at 2 GHz
+constexpr int kXPitch = 17;                               // exchange row pitch (floats): no bank conflicts
+
+template <int FMT> struct TcFmt;
+template <> struct TcFmt<MOE_W_BF16> { static constexpr int kRawRowBytes = 0;  static constexpr int kStages = 6; };
+template <> struct TcFmt<MOE_W_INT8> { static constexpr int kRawRowBytes = 64; static constexpr int kStages = 5; };
+template <> struct TcFmt<MOE_W_INT4> { static constexpr int kRawRowBytes = 32; static constexpr int kStages = 5; };
+
+__device__ unsigned int g_tc_error;  // non-zero once a bounded wait gave up
+
+struct TcParams {
+    LayerView L;
+    const int32_t *counts, *offsets;
+    int K;                 // reduction length: H (phase 1) or I (phase 2)
+    int n_units;           // output rows of the weight: 2I (phase 1) or H (phase 2)
+    int64_t rows_per_blob; // expert_bytes / row_bytes
+    int64_t q_row_off;     // offset of the code matrix in the blob / row_bytes
+    uint16_t *h;           // [R][I] bf16: phase-1 output
+    float *rows;           // [R][H] fp32: phase-2 output
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: false (and the abort flag set) if the phase did not complete in
+// time or another role already gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            atomicExch(&g_tc_error, 1u);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), leading offset unused (1), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float gelu_tanh(float v) {
+    const float c = 0.7978845608028654f;  // sqrt(2/pi)
+    const float u = c * (v + 0.044715f * v * v * v);
+    return 0.5f * v * (1.0f + tanhf(u));
+}
+
+
+// ------------------------------------------------------------- work items
+// Item = (active expert a, block of <= kNMax of its routes, M tile); M tiles
+// fastest so the CTAs working on one expert share its activation tiles in L2.
+struct Items {
+    int n_act, total, m_tiles;
+};
+
+__device__ void build_items(const TcParams &p, int m_tiles, int *s_act, int *s_base, Items *it) {
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x < 32) {
+        int n_act = 0, run = 0;
+        for (int e0 = 0; e0 < p.L.E; e0 += 32) {
+            const int e = e0 + lane;
+            const int n = (e < p.L.E) ? __ldg(p.counts + e) : 0;
+            const bool act = n > 0;
+            const unsigned m = __ballot_sync(0xffffffffu, act);
+            const int items = act ? m_tiles * ((n + kNMax - 1) / kNMax) : 0;
+            int inc = items;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, off);
+                if (lane >= off) inc += v;
+            }
+            if (act) {
+                const int pos = n_act + __popc(m & ((1u << lane) - 1u));
+                s_act[pos] = e;
+                s_base[pos] = run + inc - items;
+            }
+            run += __shfl_sync(0xffffffffu, inc, 31);
+            n_act += __popc(m);
+        }
+        if (lane == 0) {
+            s_base[n_act] = run;
+            it->n_act = n_act;
+            it->total = run;
+            it->m_tiles = m_tiles;
+        }
+    }
+}
+
+struct ItemInfo {
+    int e, row0, n, n_mma, m0;
+};
+
+__device__ __forceinline__ ItemInfo decode_item(const TcParams &p, const int *s_act, const int *s_base, int n_act,
+                                                int m_tiles, int item) {
+    int lo = 0, hi = n_act - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_base[mid] <= item) lo = mid; else hi = mid - 1;
+    }
+    const int rem = item - s_base[lo];
+    const int nb = rem / m_tiles, mt = rem - nb * m_tiles;
+    ItemInfo r;
+    r.e = s_act[lo];
+    const int n_e = __ldg(p.counts + r.e);
+    r.row0 = __ldg(p.offsets + r.e) + nb * kNMax;
+    r.n = min(kNMax, n_e - nb * kNMax);
+    r.n_mma = (r.n + 15) & ~15;
+    r.m0 = mt;  // tile index; callers scale it
+    return r;
+}
+
+// Row coordinate of weight row `row` of expert e in the home / pool tensor maps.
+__device__ __forceinline__ int a_row_coord(const TcParams &p, int e, int row, bool *in_pool) {
+    const int s = p.L.slot_table ? __ldg(p.L.slot_table + e) : -1;
+    *in_pool = s >= 0;
+    const int64_t blob = s >= 0 ? s : e;
+    return (int)(blob * p.rows_per_blob + p.q_row_off + row);
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int FMT, int PHASE>
+__global__ void __launch_bounds__(32 * (6 + (FMT == MOE_W_BF16 ? 0 : kDeqWarps)), 1)
+k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ CUtensorMap map_pool,
+         const __grid_constant__ CUtensorMap map_b, const TcParams p) {
+    constexpr int S = TcFmt<FMT>::kStages;
+    constexpr int RAW = TcFmt<FMT>::kRawRowBytes * kBlockM;  // raw code bytes per stage
+    constexpr bool kDeq = FMT != MOE_W_BF16;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned carve-up: A tiles | B tiles | raw tiles | exchange | barriers
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = sA + S * kATileBytes;
+    uint8_t *sRaw = sB + S * kBTileBytes;
+    float *sX = reinterpret_cast<float *>(sRaw + S * RAW);        // [2][64][kXPitch] gate/up exchange
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sX + 2 * 64 * kXPitch);
+    uint64_t *full = bars;              // TMA bytes landed (A or raw, and B)
+    uint64_t *deq = bars + S;           // A tile ready in bf16 (int formats)
+    uint64_t *empty = bars + 2 * S;     // MMAs done reading the stage
+    uint64_t *tfull = bars + 3 * S;     // accumulator ready
+    uint64_t *tempty = bars + 3 * S + kAccBufs;  // accumulator drained
+    uint64_t *xfull = bars + 3 * S + 2 * kAccBufs;   // up values written to the exchange
+    uint64_t *xempty = xfull + 2;                    // exchange read by the gate warps
+
+    __shared__ int s_act[kMaxE];
+    __shared__ int s_base[kMaxE + 1];
+    __shared__ Items s_items;
+    __shared__ uint32_t s_tmem;
+    __shared__ volatile int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m_tiles = PHASE == 1 ? p.L.I / 64 : (p.L.H + kBlockM - 1) / kBlockM;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&deq[s], kDeqWarps);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < kAccBufs; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&xfull[b], 2);
+            mbar_init(&xempty[b], 2);
+        }
+        s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    build_items(p, m_tiles, s_act, s_base, &s_items);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const int n_act = s_items.n_act, total = s_items.total;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
+                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+                bool pool;
+                int ya0, ya1;  // A row coordinates of the two 64-row halves
+                if (PHASE == 1) {
+                    ya0 = a_row_coord(p, it.e, it.m0 * 64, &pool);
+                    ya1 = a_row_coord(p, it.e, p.L.I + it.m0 * 64, &pool);
+                } else {
+                    ya0 = a_row_coord(p, it.e, it.m0 * kBlockM, &pool);
+                    ya1 = ya0 + 64;
+                }
+                const CUtensorMap *ma = pool ? &map_pool : &map_home;
+                const uint32_t a_bytes = kDeq ? (uint32_t)RAW : kATileBytes;
+                const uint32_t bytes = a_bytes + (uint32_t)it.n_mma * kBlockK * 2;
+                for (int kk = 0; kk < p.K / kBlockK; ++kk) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, &s_abort)) break;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    if (kDeq) {
+                        uint8_t *dst = sRaw + stage * RAW;
+                        const int xb = kk * TcFmt<FMT>::kRawRowBytes;
+                        tma_load_2d(dst, ma, &full[stage], xb, ya0);
+                        tma_load_2d(dst + 64 * TcFmt<FMT>::kRawRowBytes, ma, &full[stage], xb, ya1);
+                    } else {
+                        uint8_t *dst = sA + stage * kATileBytes;
+                        tma_load_2d(dst, ma, &full[stage], kk * kBlockK, ya0);
+                        tma_load_2d(dst + kATileBytes / 2, ma, &full[stage], kk * kBlockK, ya1);
+                    }
+                    uint8_t *db = sB + stage * kBTileBytes;
+                    for (int j = 0; j < it.n_mma; j += 16)
+                        tma_load_2d(db + j * 128, &map_b, &full[stage], kk * kBlockK, it.row0 + j);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
+                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, &s_abort)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(acc * kNMax);
+                const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(it.n_mma >> 3) << 17) |
+                                       ((uint32_t)(kBlockM >> 4) << 24);
+                bool ok = true;
+                for (int kk = 0; kk < p.K / kBlockK; ++kk) {
+                    if (!mbar_wait(kDeq ? &deq[stage] : &full[stage], phase, &s_abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * kATileBytes);
+                    const uint32_t b0 = smem_u32(sB + stage * kBTileBytes);
+#pragma unroll
+                    for (int j = 0; j < kBlockK / 16; ++j)
+                        tc_mma_bf16(d, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc, (kk | j) != 0);
+                    tc_commit(&empty[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&tfull[acc]);
+                if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1; }
+            }
+        }
+    } else if (warp < 2 + kEpiWarps) {
+        // --------------------------------------------------------- epilogue
+        const int q = warp & 3;                 // TMEM lane quadrant of this warp
+        const int lrow = q * 32 + lane;         // tile row held by this thread
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        uint32_t xcount = 0;  // exchange chunks used so far (buffer = xcount & 1)
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok && !s_abort; item += gridDim.x) {
+            const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+            if (!mbar_wait(&tfull[acc], acc_phase, &s_abort)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kNMax);
+            const uint8_t *blob = expert_blob(p.L, it.e);
+            float scale = 1.0f;
+            if (FMT == MOE_W_INT8) {
+                const int wrow = PHASE == 1 ? (lrow < 64 ? it.m0 * 64 + lrow : p.L.I + it.m0 * 64 + lrow - 64)
+                                            : min(it.m0 * kBlockM + lrow, p.n_units - 1);
+                scale = __ldg(reinterpret_cast<const float *>(blob + (PHASE == 1 ? p.L.off.s13 : p.L.off.s2)) + wrow);
+            }
+            for (int c0 = 0; c0 < it.n_mma; c0 += 16) {
+                float v[16];
+                tmem_ld16(taddr + (uint32_t)c0, v);
+                if (PHASE == 1) {
+                    // tile rows 64..127 hold the up projection, rows 0..63 the gate of
+                    // the same intermediate columns: the up warps pass their values
+                    // through shared memory to the gate warps
+                    const uint32_t xb = xcount & 1, xpar = (xcount >> 1) & 1;
+                    float *xrow = sX + (size_t)xb * 64 * kXPitch + (size_t)(lrow & 63) * kXPitch;
+                    if (lrow >= 64) {
+                        if (!mbar_wait(&xempty[xb], xpar ^ 1, &s_abort)) { ok = false; break; }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) xrow[i] = v[i] * scale;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&xfull[xb]);
+                    } else {
+                        if (!mbar_wait(&xfull[xb], xpar, &s_abort)) { ok = false; break; }
+                        const int icol = it.m0 * 64 + lrow;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int j = c0 + i;
+                            if (j < it.n) {
+                                const float g = v[i] * scale, up = xrow[i];
+                                p.h[(size_t)(it.row0 + j) * p.L.I + icol] = f32_to_bf16_rne(gelu_tanh(g) * up);
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&xempty[xb]);
+                    }
+                    ++xcount;
+                } else {
+                    const int m = it.m0 * kBlockM + lrow;
+                    if (m < p.L.H) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int j = c0 + i;
+                            if (j < it.n) p.rows[(size_t)(it.row0 + j) * p.L.H + m] = v[i] * scale;
+                        }
+                    }
+                }
+            }
+            if (!ok) break;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1; }
+        }
+    } else if (kDeq) {
+        // ---------------------------------------------------- dequantisation
+        // two threads per tile row (half a row, 32 weights = 4 chunks, each):
+        // raw codes -> bf16 in the 128-byte-swizzled K-major layout (8-row groups
+        // of 1024 bytes, 16-byte chunk c of row r stored at chunk c ^ (r % 8)).
+        const int t = (warp - 2 - kEpiWarps) * 32 + lane;
+        const int r = t & (kBlockM - 1), hf = t >> 7;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
+            const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+            const uint8_t *blob = expert_blob(p.L, it.e);
+            const int wrow = PHASE == 1 ? (r < 64 ? it.m0 * 64 + r : p.L.I + it.m0 * 64 + r - 64)
+                                        : min(it.m0 * kBlockM + r, p.n_units - 1);
+            const uint16_t *srow = reinterpret_cast<const uint16_t *>(blob + (PHASE == 1 ? p.L.off.s13 : p.L.off.s2)) +
+                                   (size_t)wrow * (p.K / 64);
+            bool ok = true;
+            for (int kk = 0; kk < p.K / kBlockK; ++kk) {
+                __nv_bfloat162 s2 = __floats2bfloat162_rn(0.0f, 0.0f);
+                if (FMT == MOE_W_INT4) s2 = __bfloat162bfloat162(__ushort_as_bfloat16(__ldg(srow + kk)));
+                if (!mbar_wait(&full[stage], phase, &s_abort)) { ok = false; break; }
+                const uint8_t *src = sRaw + stage * RAW + r * TcFmt<FMT>::kRawRowBytes;
+                uint8_t *dst = sA + stage * kATileBytes + (r >> 3) * 1024 + (r & 7) * 128;
+                if (FMT == MOE_W_INT4) {
+                    // 16 raw bytes = weights 32hf .. 32hf+31 = chunks 4hf .. 4hf+3
+                    const uint4 u = *reinterpret_cast<const uint4 *>(src + 16 * hf);
+                    const uint32_t words[4] = {u.x, u.y, u.z, u.w};
+                    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        // byte j of the word = weight 2j (low nibble), 2j+1 (high):
+                        // pair -> bf16x2 {128 + n_lo, 128 + n_hi} -> minus 136 -> times s
+                        const uint32_t w = words[i], w4 = w >> 4;
+                        uint32_t o[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t dup = __byte_perm(w, w4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
+                            uint32_t v = (dup & 0x000F000Fu) | 0x43004300u;
+                            __nv_bfloat162 q = *reinterpret_cast<__nv_bfloat162 *>(&v);
+                            q = __hmul2(__hsub2(q, bias), s2);
+                            o[j] = *reinterpret_cast<uint32_t *>(&q);
+                        }
+                        const int c = 4 * hf + i;
+                        *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {  // 8 int8 codes -> 16-byte chunk c (codes exact in bf16)
+                        const int c = 4 * hf + i;
+                        const uint2 u = *reinterpret_cast<const uint2 *>(src + 8 * c);
+                        const uint32_t a = u.x ^ 0x80808080u, b = u.y ^ 0x80808080u;
+                        uint32_t o[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t src_w = j < 2 ? a : b;
+                            const uint32_t sel0 = 0x7540u | (uint32_t)(2 * (j & 1)), sel1 = sel0 + 1;
+                            const float f0 = __uint_as_float(__byte_perm(src_w, 0x4B000000u, sel0)) - 8388736.0f;
+                            const float f1 = __uint_as_float(__byte_perm(src_w, 0x4B000000u, sel1)) - 8388736.0f;
+                            __nv_bfloat162 q = __floats2bfloat162_rn(f0, f1);
+                            o[j] = *reinterpret_cast<uint32_t *>(&q);
+                        }
+                        *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&deq[stage]);
+                if (++stage == S) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// x rows gathered into sorted-route order: xs[s] = x[sorted_route[s] / k] for
+// s < offsets[E] (16 bytes per thread).
+__global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ sorted_route,
+                              const int32_t *__restrict__ offsets, int E, int k, int H, int R,
+                              uint16_t *__restrict__ xs) {
+    const int per = H / 8;
+    const int n_valid = __ldg(offsets + E);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)R * per;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int s = (int)(i / per), c = (int)(i % per);
+        if (s >= n_valid) continue;
+        const int tok = __ldg(sorted_route + s) / k;
+        reinterpret_cast<uint4 *>(xs + (size_t)s * H)[c] =
+            __ldg(reinterpret_cast<const uint4 *>(x + (size_t)tok * H) + c);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+cudaError_t get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// 2-D map over `rows` rows of `row_bytes` bytes; box = box_inner elements x box_rows.
+bool encode_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t row_elems,
+               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+    cuuint64_t dims[2] = {row_elems, rows};
+    cuuint64_t strides[1] = {row_elems * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t smem_bytes(int fmt) {
+    const int S = fmt == MOE_W_BF16 ? TcFmt<MOE_W_BF16>::kStages
+                                    : (fmt == MOE_W_INT8 ? TcFmt<MOE_W_INT8>::kStages : TcFmt<MOE_W_INT4>::kStages);
+    const int raw = fmt == MOE_W_BF16 ? 0 : (fmt == MOE_W_INT8 ? 64 : 32) * kBlockM;
+    return 1024 + (size_t)S * (kATileBytes + kBTileBytes + raw) + 2 * 64 * kXPitch * 4 + (3 * S + 2 * kAccBufs + 4) * 8;
+}
+
+template <int FMT, int PHASE>
+cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUtensorMap &mb, const TcParams &p,
+                       int n_sm, cudaStream_t s) {
+    auto kern = k_ffn_tc<FMT, PHASE>;
+    const size_t smem = smem_bytes(FMT);
+    static bool attr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!attr[dev]) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        attr[dev] = true;
+    }
+    const int threads = 32 * (6 + (FMT == MOE_W_BF16 ? 0 : kDeqWarps));
+    kern<<<n_sm, threads, smem, s>>>(mh, mp, mb, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t ffn_tc_workspace(int T, int k, int E, int H, int I) {
+    (void)E;
+    const size_t R = (size_t)T * k;
+    const size_t xs = (R * H * 2 + 255) & ~(size_t)255;
+    return xs + R * I * 2;
+}
+
+bool ffn_tc_supports(int fmt, int H, int I, uint64_t stride) {
+    if (H % 64 || I % 64) return false;
+    // every weight row of every expert must start on a whole row of the tensor
+    // map that spans the blob buffer
+    const BlobOffsets o = blob_offsets(fmt, H, I);
+    const uint64_t rb1 = fmt == MOE_W_BF16 ? (uint64_t)H * 2 : (fmt == MOE_W_INT8 ? (uint64_t)H : (uint64_t)H / 2);
+    const uint64_t rb2 = fmt == MOE_W_BF16 ? (uint64_t)I * 2 : (fmt == MOE_W_INT8 ? (uint64_t)I : (uint64_t)I / 2);
+    return stride % rb1 == 0 && stride % rb2 == 0 && o.q2 % rb2 == 0 && get_encoder() == cudaSuccess;
+}
+
+cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, const int32_t *counts,
+                          const int32_t *offsets, const int32_t *sorted_route, float *rows, void *ws,
+                          cudaStream_t s) {
+    cudaError_t err = get_encoder();
+    if (err != cudaSuccess) return err;
+    if (!ffn_tc_supports(L.fmt, L.H, L.I, L.stride)) return cudaErrorNotSupported;
+    int n_sm = 0;
+    if ((err = sm_count(&n_sm)) != cudaSuccess) return err;
+    const int R = T * k;
+    const int H = L.H, I = L.I, fmt = L.fmt;
+    uint16_t *xs = static_cast<uint16_t *>(ws);
+    uint16_t *h = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + (((size_t)R * H * 2 + 255) & ~(size_t)255));
+
+    // 1. activations into sorted-route order
+    {
+        const int64_t n = (int64_t)R * (H / 8);
+        const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)n_sm * 8);
+        k_gather_rows<<<blocks, 256, 0, s>>>(x, sorted_route, offsets, L.E, k, H, R, xs);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    // 2. tensor maps: weights (home and pool, as rows of one matrix), activations
+    const bool bf = fmt == MOE_W_BF16;
+    const CUtensorMapDataType dt = bf ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const int eb = bf ? 2 : 1;
+    const CUtensorMapSwizzle swa = bf ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const uint32_t raw_inner = fmt == MOE_W_INT8 ? 64 : 32;
+    CUtensorMap mh1, mp1, mh2, mp2, mb1, mb2;
+    for (int ph = 1; ph <= 2; ++ph) {
+        const int K = ph == 1 ? H : I;
+        const uint64_t row_elems = bf ? (uint64_t)K : (fmt == MOE_W_INT8 ? (uint64_t)K : (uint64_t)K / 2);
+        const uint64_t row_bytes = row_elems * eb;
+        const uint32_t box_inner = bf ? kBlockK : raw_inner;
+        CUtensorMap *mh = ph == 1 ? &mh1 : &mh2, *mp = ph == 1 ? &mp1 : &mp2;
+        const uint64_t home_rows = (uint64_t)L.E * L.stride / row_bytes;
+        if (!encode_2d(mh, L.home, dt, eb, row_elems, home_rows, box_inner, 64, swa)) return cudaErrorInvalidValue;
+        // the pool's extent is unknown here: map it with the home's row count
+        // (only rows of slots in use are ever addressed)
+        if (!encode_2d(mp, L.pool ? L.pool : L.home, dt, eb, row_elems, home_rows, box_inner, 64, swa))
+            return cudaErrorInvalidValue;
+        CUtensorMap *mb = ph == 1 ? &mb1 : &mb2;
+        if (!encode_2d(mb, ph == 1 ? (const void *)xs : (const void *)h, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                       (uint64_t)K, (uint64_t)R, kBlockK, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    TcParams p{};
+    p.L = L;
+    p.counts = counts;
+    p.offsets = offsets;
+    p.h = h;
+    p.rows = rows;
+    // phase 1
+    {
+        const uint64_t rb = bf ? (uint64_t)H * 2 : (fmt == MOE_W_INT8 ? (uint64_t)H : (uint64_t)H / 2);
+        p.K = H;
+        p.n_units = 2 * I;
+        p.rows_per_blob = (int64_t)(L.stride / rb);
+        p.q_row_off = (int64_t)(L.off.q13 / rb);
+        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 1>(mh1, mp1, mb1, p, n_sm, s);
+        else if (fmt == MOE_W_INT8) err = launch_one<MOE_W_INT8, 1>(mh1, mp1, mb1, p, n_sm, s);
+        else err = launch_one<MOE_W_INT4, 1>(mh1, mp1, mb1, p, n_sm, s);
+        if (err != cudaSuccess) return err;
+    }
+    // phase 2
+    {
+        const uint64_t rb = bf ? (uint64_t)I * 2 : (fmt == MOE_W_INT8 ? (uint64_t)I : (uint64_t)I / 2);
+        p.K = I;
+        p.n_units = H;
+        p.rows_per_blob = (int64_t)(L.stride / rb);
+        p.q_row_off = (int64_t)(L.off.q2 / rb);
+        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 2>(mh2, mp2, mb2, p, n_sm, s);
+        else if (fmt == MOE_W_INT8) err = launch_one<MOE_W_INT8, 2>(mh2, mp2, mb2, p, n_sm, s);
+        else err = launch_one<MOE_W_INT4, 2>(mh2, mp2, mb2, p, n_sm, s);
+    }
+    return err;
+}
+
+cudaError_t tc_take_error(unsigned *out) {
+    unsigned zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_tc_error, sizeof(unsigned));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(unsigned));
 }
 
 }  // namespace moe

@@ -331,3 +331,78 @@ def test_gemma_layer_prefill_sampled():
     full_rows[routes] = orows
     oy = oracle.combine(full_rows, oi, ow, E)[toks]
     assert rel_err(bf16_dev_to_f64(y)[toks], oy) <= FFN_TOL
+
+
+# ------------------------------------------------------ tensor-core FFN path
+
+def _tc_or_skip(L, lg, x, k):
+    try:
+        return _run_layer(L, lg, x, k, path=moe.MOE_FFN_TC)
+    except moe.MoeError as e:
+        assert e.status == moe.MOE_ERR_UNSUPPORTED, str(e)
+        pytest.skip(f"tensor-core path unsupported here: {e}")
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("E,H,I,k,T", [(8, 256, 128, 2, 16), (8, 512, 192, 3, 37), (6, 1024, 320, 2, 61),
+                                       (4, 384, 64, 4, 300), (3, 256, 128, 3, 200)])
+def test_tc_layer_small_every_element(fmt, E, H, I, k, T):
+    """tcgen05 path forced: every row and output against the oracle; shapes with
+    several M tiles, a partial last tile (H % 128 != 0), ragged route blocks and
+    experts with more than 128 routes (several N blocks)."""
+    w13, w2 = syn.expert_weights(E, H, I, seed=E + H + 1)
+    x = syn.activations(T, H, seed=8)
+    lg = syn.router_logits(T, E, "normal", seed=12)
+    L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    ids, w, counts, offsets, sr, rp, rows, y = _tc_or_skip(L, torch.from_numpy(lg).to(DEV), xd, k)
+    oi, ow, orows, oy = oracle.moe_layer(oracle_layer_for(fmt, w13, w2), lg, x, k)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    g_rows = rows.cpu().numpy()[rp.cpu().numpy()]
+    assert rel_err(g_rows, orows) <= FFN_TOL
+    assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
+
+
+@pytest.mark.parametrize("fmt,kind", [(0, "normal"), (1, "biased"), (2, "normal")])
+@pytest.mark.parametrize("T", [8, 64])
+def test_tc_gemma_layer_decode_sampled(fmt, kind, T):
+    E, H, I, k = 128, 2816, 704, 8
+    w13, w2, L = _full_layer(fmt)
+    x = syn.activations(T, H, seed=300 + T)
+    lg = syn.router_logits(T, E, kind, seed=400 + T)
+    ids, w, counts, offsets, sr, rp, rows, y = _tc_or_skip(
+        L, torch.from_numpy(lg).to(DEV), torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16), k)
+    oi, ow = oracle.route_topk(lg, k)
+    toks = np.unique(np.r_[0, T - 1, np.random.default_rng(T).integers(0, T, size=2)])
+    routes = np.concatenate([np.arange(t * k, (t + 1) * k) for t in toks]).astype(np.int32)
+    experts = sorted(set(oi.ravel()[routes].tolist()))
+    OL = _sparse_oracle_layer(fmt, E, H, I, {e: host_bits(w13[e]) for e in experts},
+                              {e: host_bits(w2[e]) for e in experts})
+    orows = oracle.ffn_some_routes(OL, x, oi, routes)
+    assert rel_err(rows.cpu().numpy()[rp.cpu().numpy()[routes]], orows) <= FFN_TOL
+    full_rows = np.zeros((T * k, H))
+    full_rows[routes] = orows
+    oy = oracle.combine(full_rows, oi, ow, E)[toks]
+    assert rel_err(bf16_dev_to_f64(y)[toks], oy) <= FFN_TOL
+
+
+def test_tc_and_gemv_agree_on_the_slot_table():
+    """Both kernel paths read experts through the slot table the same way."""
+    E, H, I, k, T = 16, 512, 128, 4, 90
+    w13, w2 = syn.expert_weights(E, H, I, seed=21)
+    L = moe.make_layer(0, *device_weights_from_host(w13, w2))
+    eb = L.expert_bytes
+    slot_of = np.full(E, -1, np.int32)
+    slot_of[[2, 11, 5]] = [1, 0, 2]
+    pool = torch.zeros(3 * eb, dtype=torch.uint8, device=DEV)
+    moe.moe_copy_to_slots(L.home, pool, eb, np.nonzero(slot_of >= 0)[0], slot_of[slot_of >= 0])
+    home2 = L.home.clone()
+    for e in np.nonzero(slot_of >= 0)[0]:
+        home2[e * eb:(e + 1) * eb] = 0
+    L2 = moe.MoeLayer(0, E, H, I, home2, pool=pool, slot_table=torch.from_numpy(slot_of).to(DEV))
+    x = torch.from_numpy(syn.activations(T, H, seed=2).view(np.int16)).to(DEV).view(torch.bfloat16)
+    lg = torch.from_numpy(syn.router_logits(T, E, "zipf", seed=2)).to(DEV)
+    a = _run_layer(L, lg, x, k, path=moe.MOE_FFN_GEMV)[-2]
+    b = _tc_or_skip(L2, lg, x, k)[-2]
+    n = a.shape[0]
+    assert rel_err(b.cpu().numpy()[:n], a.cpu().numpy()) <= FFN_TOL

@@ -57,6 +57,8 @@ CONFIGS = {
     "int4-decode": ("int4", "normal", 64, []),
     "int4-prefill": ("int4", "normal", 1024, []),
     "tiny": ("bf16", "normal", 16, []),
+    # 30-layer stack, slot table, Zipf(1.1) routing, refresh every 8 steps
+    "stack30": ("int4", "zipf", 64, [1, 8]),
 }
 
 
@@ -367,6 +369,8 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args, fmt_name, kind, T, E, H, I, k, world, rank)
+    if args.config == "stack30":
+        return stack_main(args, T, E, H, I, k, world, rank, local)
 
     import torch
 
@@ -506,6 +510,193 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# ----------------------------------------------------------- the layer stack
+
+class Stack:
+    """A stack of MoE layers whose experts are read through per-layer cache slots.
+
+    Every layer has its E home blobs and a pool of `slots` blobs; slot_of[l] (host)
+    mirrors the device slot table.  Initial residents are experts 0..slots-1
+    (expert_pool.rs, ExpertPool::new)."""
+
+    def __init__(self, moe, torch, fmt_name, E, H, I, L, slots, dev, seed=0):
+        self.moe, self.torch = moe, torch
+        self.homes = build_layers(moe, torch, fmt_name, E, H, I, L, dev, seed=seed)
+        self.fmt = moe.FMT[fmt_name]
+        self.E, self.H, self.I, self.L, self.slots = E, H, I, L, slots
+        self.eb = self.homes[0].expert_bytes
+        self.slot_of = []
+        self.layers = []
+        self.pools = []
+        for l in range(L):
+            so = np.full(E, -1, np.int32)
+            so[:slots] = np.arange(slots)
+            pool = torch.empty(slots * self.eb, dtype=torch.uint8, device=dev)
+            moe.moe_copy_to_slots(self.homes[l].home, pool, self.eb, np.arange(slots), np.arange(slots))
+            table = torch.from_numpy(so).to(dev)
+            self.layers.append(moe.MoeLayer(self.fmt, E, H, I, self.homes[l].home, pool=pool, slot_table=table,
+                                            expert_bytes=self.eb))
+            self.slot_of.append(so)
+            self.pools.append(pool)
+        self.stats = {"refreshes": 0, "promotions": 0, "demotions": 0, "resident_route_share": []}
+        torch.cuda.synchronize(dev)
+
+    def refresh(self, hits_host):
+        """Placement refresh of every layer from one step's hit histogram
+        (expert_pool.rs: target_gpu_from_counts, then apply_target_placement),
+        promotion copies into the freed slots, slot tables uploaded."""
+        moe = self.moe
+        for l in range(self.L):
+            h = hits_host[l]
+            tot = int(h.sum())
+            if tot:
+                self.stats["resident_route_share"].append(float(h[self.slot_of[l] >= 0].sum()) / tot)
+            target = moe.moe_refresh_target(h, self.slots)
+            so, promote, demote = moe.moe_apply_placement(self.slot_of[l], self.slots, target)
+            if len(promote):
+                moe.moe_copy_to_slots(self.layers[l].home, self.pools[l], self.eb, promote, so[promote])
+                self.layers[l].slot_table.copy_(self.torch.from_numpy(so), non_blocking=False)
+            self.slot_of[l] = so
+            self.stats["promotions"] += len(promote)
+            self.stats["demotions"] += len(demote)
+        self.stats["refreshes"] += 1
+
+
+def stack_steps(torch, moe, stack, T, k, steps, warmup, seed, refresh_every=8, path=0):
+    """`steps` decode steps through the whole stack; a placement refresh from the
+    hits of every step that is a multiple of `refresh_every`.  Returns total ms."""
+    import synthetic as syn
+
+    dev = stack.layers[0].home.device
+    E, H, L = stack.E, stack.H, stack.L
+    W = refresh_every
+    n = steps + warmup
+    # inputs of every step, resident in HBM: Zipf(1.1) logits per (step, layer), x per step
+    lg_all = torch.empty((n, L, T, E), dtype=torch.float32, device=dev)
+    x_all = torch.empty((n, T, H), dtype=torch.bfloat16, device=dev)
+    for st in range(n):
+        lg_all[st] = torch.from_numpy(np.stack([syn.router_logits(T, E, "zipf", seed=seed, layer=l, step=st)
+                                                for l in range(L)])).to(dev)
+        x_all[st] = torch.from_numpy(syn.activations(T, H, seed=seed, layer=st).view(np.int16)).to(dev).view(torch.bfloat16)
+    lg_stage = torch.empty((W, L, T, E), dtype=torch.float32, device=dev)
+    x_stage = torch.empty((W, T, H), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(moe.moe_grouped_ffn_workspace(stack.layers[0], T, k), dtype=torch.uint8, device=dev)
+    R = T * k
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    perm = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
+            torch.empty(R, dtype=torch.int32, device=dev), torch.empty(R, dtype=torch.int32, device=dev))
+    rows = torch.empty((R, H), dtype=torch.float32, device=dev)
+    ybuf = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    hits = torch.zeros((L, E), dtype=torch.int32, device=dev)
+
+    def one_step(j, with_hits):
+        x = x_stage[j]
+        for l in range(L):
+            lay = stack.layers[l]
+            moe.moe_route_topk(lg_stage[j, l], k, ids, w)
+            moe.moe_permute(ids, E, hits=hits[l] if with_hits else None, out=perm)
+            moe.moe_grouped_ffn(lay, x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
+            y = ybuf[l & 1]
+            moe.moe_combine(rows, perm[3], w, y)
+            x = y
+
+    def window_inputs(first):
+        m = min(W, n - first)
+        lg_stage[:m].copy_(lg_all[first:first + m])
+        x_stage[:m].copy_(x_all[first:first + m])
+
+    # prime one-time set-up, then capture: graph A = the refresh step (with hits),
+    # graph B = the W-1 steps after it
+    window_inputs(0)
+    one_step(0, True)
+    torch.cuda.synchronize()
+    hits.zero_()
+    ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ga):
+        one_step(0, True)
+    with torch.cuda.graph(gb):
+        for j in range(1, W):
+            one_step(j, False)
+    torch.cuda.synchronize()
+
+    def run(first, count):
+        st = first
+        while st < first + count:
+            window_inputs(st)
+            hits.zero_()
+            ga.replay()                                # step st (a multiple of W): counts hits
+            stack.refresh(hits.cpu().numpy().view(np.uint32))  # syncs on the hit histogram
+            rest = min(W - 1, first + count - st - 1)
+            if rest == W - 1:
+                gb.replay()
+            else:
+                for j in range(1, 1 + rest):
+                    one_step(j, False)
+            st += 1 + rest
+
+    run(0, warmup)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    run(warmup, steps)
+    t1.record()
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1)
+
+
+def stack_main(args, T, E, H, I, k, world, rank, local):
+    """30-layer stacks (int4 and bf16, both resident), 18 cache slots per layer,
+    Zipf(1.1) routing, placement refresh every 8 steps; tokens/s through the stack."""
+    import torch
+
+    import moe_router_softmax_b200 as moe
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    L, slots = (args.layers if args.layers != 30 else 30), 18
+    steps = args.steps if args.steps != 3000 else 256
+    warmup = max(args.warmup if args.warmup != 30 else 8, 3)
+    path = {"auto": moe.MOE_FFN_AUTO, "gemv": moe.MOE_FFN_GEMV, "tc": moe.MOE_FFN_TC}[args.path]
+    s4 = Stack(moe, torch, "int4", E, H, I, L, slots, dev, seed=1)
+    s16 = Stack(moe, torch, "bf16", E, H, I, L, slots, dev, seed=2)
+    resident_gb = (sum(h.home.numel() for h in s4.homes) + sum(h.home.numel() for h in s16.homes) +
+                   sum(p.numel() for p in s4.pools) + sum(p.numel() for p in s16.pools)) / 1e9
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = stack_steps(torch, moe, s4, T, k, steps, warmup, seed=11, path=path)
+    clk = clocks.stop()
+    value = world * T * steps / (ms / 1e3)
+    sweep = {}
+    for name, st, Ts in [("bf16", s16, T)] + ([] if args.quick else [("int4", s4, t) for t in (1, 8) if t != T]):
+        ms2 = stack_steps(torch, moe, st, Ts, k, steps, warmup, seed=12 + Ts, path=path)
+        sweep[f"{name}_T{Ts}"] = {"tokens_per_s": round(world * Ts * steps / (ms2 / 1e3), 1),
+                                  "ms_per_step": round(ms2 / steps, 4)}
+    share = s4.stats["resident_route_share"]
+    hbm_peak = measured_peaks()[0]
+    line = {
+        "metric": "MoE layer tokens/s and expert-weight HBM GB/s (% of roofline) at decode/prefill",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": round(ms / steps, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4", "data": "synthetic (seeded; Zipf(1.1) routing; random weights)",
+        "config": {"workload": f"moe-stack{L}-int4-decode-T{T}", "layers": L, "experts": E, "hidden": H,
+                   "intermediate": I, "top_k": k, "tokens": T, "slots_per_layer": slots, "refresh_every": 8,
+                   "logits": "zipf(1.1)", "resident_gb": round(resident_gb, 1), "ffn_path": args.path,
+                   "l2": "inputs larger than L2: each step reads 30 layers' routed experts"},
+        "placement": {"refreshes": s4.stats["refreshes"], "promotions": s4.stats["promotions"],
+                      "demotions": s4.stats["demotions"],
+                      "routes_on_resident_slots": round(sum(share) / len(share), 4) if share else None},
+        "sweep": sweep,
+        "hbm_peak_gbs": hbm_peak,
+        "gpu_launches": steps * L * (4 + (3 if (path == moe.MOE_FFN_TC or
+                                                 (path == moe.MOE_FFN_AUTO and T * k >= 65)) else 2)),
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def reference_arm(args, fmt_name, kind, T, E, H, I, k, world, rank):

@@ -239,6 +239,13 @@ MOE_API moe_status moe_pack_expert(int32_t fmt, const void *w13, const void *s13
 MOE_API moe_status moe_copy_to_slots(const void *home, void *pool, uint64_t expert_bytes, const int32_t *experts,
                              const int32_t *slots, int32_t n, moe_stream_t stream);
 
+/* Diagnostics: synchronise the device, then read and clear the first problem
+ * the tensor-core kernels recorded since the last call.  *code = 0 and MOE_OK
+ * if none; MOE_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the
+ * kernel then drained out without finishing its work); MOE_ERR_CUDA if an
+ * index check failed (the access was skipped; *info holds the value). */
+MOE_API moe_status moe_take_device_errors(uint32_t *code, uint32_t *info);
+
 /* ---------------------------------------------------------------------------
  * Expert residency pool, host only (rlx_runtime expert_pool.rs).
  * ------------------------------------------------------------------------- */

@@ -35,7 +35,7 @@ EXPORTS = [
     "moe_expert_hits", "moe_grouped_ffn_workspace", "moe_grouped_ffn", "moe_grouped_ffn_path", "moe_combine",
     "moe_layer_forward_workspace", "moe_layer_forward", "moe_quantize_int8", "moe_quantize_int4",
     "moe_pack_expert", "moe_copy_to_slots", "moe_refresh_target", "moe_apply_placement",
-    "moe_should_refresh", "moe_budget_from_vram", "moe_grouped_ffn_noalloc",
+    "moe_should_refresh", "moe_budget_from_vram", "moe_grouped_ffn_noalloc", "moe_take_device_errors",
 ]
 
 
@@ -78,6 +78,7 @@ _SIG = {
     "moe_should_refresh": (i32, [i32, i32, i64, i32, i64]),
     "moe_budget_from_vram": (i64, [i64, i64, i64, i64, i64, i64]),
     "moe_grouped_ffn_noalloc": (i32, [LP, P, i32, i32, P, P, P, P, P]),
+    "moe_take_device_errors": (i32, [P, P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -277,6 +278,16 @@ def moe_copy_to_slots(home: torch.Tensor, pool: torch.Tensor, expert_bytes: int,
     assert ex.size == sl.size
     _check(_lib.moe_copy_to_slots(_dev(home, torch.uint8, "home"), _dev(pool, torch.uint8, "pool"), int(expert_bytes),
                                   pe, ps, ex.size, _stream(stream)))
+
+
+def moe_take_device_errors():
+    """Synchronise, then return (code, info) of the first problem a tensor-core
+    kernel recorded since the last call ((0, 0) if none)."""
+    c, i = ctypes.c_uint32(0), ctypes.c_uint32(0)
+    st = _lib.moe_take_device_errors(ctypes.byref(c), ctypes.byref(i))
+    if st not in (MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_CUDA):
+        _check(st)
+    return int(c.value), int(i.value)
 
 
 def moe_refresh_target(hits: np.ndarray, budget: int) -> np.ndarray:

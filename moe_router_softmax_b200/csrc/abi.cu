@@ -22,6 +22,7 @@ size_t ffn_tc_workspace(int T, int k, int E, int H, int I);
 bool ffn_tc_supports(int fmt, int H, int I, uint64_t stride);
 cudaError_t launch_ffn_tc(const LayerView &, const uint16_t *, int, int, const int32_t *, const int32_t *,
                           const int32_t *, float *, void *, cudaStream_t);
+cudaError_t tc_take_error(unsigned *code, unsigned *info);
 
 static thread_local char g_err[512];
 
@@ -288,6 +289,21 @@ moe_status moe_pack_expert(int32_t fmt, const void *w13, const void *s13, const 
     if (e == cudaSuccess) e = cudaMemcpyAsync(b + o.q2, w2, o.s2 - o.q2, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess && fmt != MOE_W_BF16) e = cudaMemcpyAsync(b + o.s2, s2, o.total - o.s2, cudaMemcpyDeviceToDevice, s);
     return cuda_status(e, "moe_pack_expert copy");
+}
+
+moe_status moe_take_device_errors(uint32_t *code, uint32_t *info) {
+    CHECK_ARG(code && info, "moe_take_device_errors: NULL pointer");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e, "moe_take_device_errors: device synchronise");
+    unsigned c = 0, i = 0;
+    e = tc_take_error(&c, &i);
+    if (e != cudaSuccess) return cuda_status(e, "moe_take_device_errors: read");
+    *code = c;
+    *info = i;
+    if (c >= 0x1000u && c < 0x2000u)
+        return set_error(MOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (warp %u)", c & 0xFFFu);
+    if (c) return set_error(MOE_ERR_CUDA, "a tensor-core kernel failed an index check (site %u, value %u)", c & 0xFFFu, i);
+    return MOE_OK;
 }
 
 moe_status moe_copy_to_slots(const void *home, void *pool, uint64_t expert_bytes, const int32_t *experts,

@@ -16,15 +16,21 @@
 // shared-memory stage.
 //
 // One persistent CTA per SM; warp roles:
-//   warp 0      TMA producer (A weights or raw codes, B activations)
+//   warp 0      TMA producer of A: the weight tiles (bf16) or the raw codes
+//               (int8 / int4)
 //   warp 1      TMEM allocation and the single-thread MMA issuer
 //   warps 2..5  epilogue (TMEM -> registers -> global); warp w reads TMEM
 //               lanes 32*(w%4) .. +31
-//   warps 6..13 dequantisation (int8 / int4 only)
-// Pipelines: a ring of kStages shared-memory stages (full / dequantised /
-// empty mbarriers) and two TMEM accumulators (full / empty) so the epilogue of
-// one item overlaps the main loop of the next.  Every mbarrier wait is bounded;
-// on timeout the kernel records an error word and every role drains out.
+//   warp 6      TMA producer of B: the routes' activation tiles
+//   warps 7..22 dequantisation (int8 / int4 only): two groups of eight warps
+//               taking alternate stages
+// Pipelines: separate rings for A, B and (int formats) raw codes, each with
+// full / empty mbarriers, so a slow operand never holds the other's slots; B
+// slots are sized by the launch's route block, so small decode blocks get many
+// stages in flight; two TMEM accumulators (full / empty) let the epilogue of
+// one item overlap the main loop of the next.  Every mbarrier wait is bounded
+// (and suspends in hardware while it waits); on timeout the kernel records an
+// error word and every role drains out.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -38,27 +44,53 @@ namespace moe {
 namespace {
 
 constexpr int kBlockM = 128;          // weight rows per tile (TMEM lanes)
-constexpr int kBlockK = 64;           // bf16 elements per stage = one 128-byte swizzle row
-constexpr int kNMax = 128;            // routes per accumulator (TMEM columns)
+constexpr int kBlockK = 64;           // bf16 elements per MMA stage = one 128-byte swizzle row
+constexpr int kNMax = 128;            // max routes per block (TMEM columns per accumulator)
 constexpr int kAccBufs = 2;
 constexpr int kTmemCols = kNMax * kAccBufs;
 constexpr int kEpiWarps = 4;
-constexpr int kDeqWarps = 8;   // two threads per tile row, half a row each
+constexpr int kDeqWarps = 8;          // per group: two threads per tile row, half a row each
+constexpr int kDeqGroups = 2;         // groups take alternate stages, so two stages expand at once
 constexpr uint32_t kATileBytes = kBlockM * kBlockK * 2;   // 16 KB
-constexpr uint32_t kBTileBytes = kNMax * kBlockK * 2;     // 16 KB
+constexpr int kMaxBSlots = 32;
+constexpr int kRawRowBytes = 128;     // per raw stage row
 constexpr long long kWaitCycles = 4000000000ll;           // ~2 s at 2 GHz
 constexpr int kXPitch = 17;                               // exchange row pitch (floats): no bank conflicts
 
+// Three rings of shared-memory stages, each with its own full / empty
+// mbarriers, so no operand's load latency holds another's slots:
+//  A:   kAStages weight tiles of 128 rows x 64 bf16 (TMA for bf16 weights, the
+//       dequant warps for int8/int4);
+//  B:   up to kMaxBSlots activation tiles of n_block rows x 64 bf16 (TMA), as
+//       many as fit in kBRegion bytes for this launch's block size;
+//  raw: kRawStages stages of 128 code bytes per row (int formats: 256 int4 or
+//       128 int8 weights, kSub MMA stages each), whole 128-byte runs of a row.
 template <int FMT> struct TcFmt;
-template <> struct TcFmt<MOE_W_BF16> { static constexpr int kRawRowBytes = 0;  static constexpr int kStages = 6; };
-template <> struct TcFmt<MOE_W_INT8> { static constexpr int kRawRowBytes = 64; static constexpr int kStages = 5; };
-template <> struct TcFmt<MOE_W_INT4> { static constexpr int kRawRowBytes = 32; static constexpr int kStages = 5; };
+template <> struct TcFmt<MOE_W_BF16> {
+    static constexpr int kSub = 1, kSubBytes = 0, kAStages = 8, kRawStages = 0, kBRegion = 64 * 1024;
+};
+template <> struct TcFmt<MOE_W_INT8> {
+    static constexpr int kSub = 2, kSubBytes = 64, kAStages = 4, kRawStages = 5, kBRegion = 48 * 1024;
+};
+template <> struct TcFmt<MOE_W_INT4> {
+    static constexpr int kSub = 4, kSubBytes = 32, kAStages = 4, kRawStages = 5, kBRegion = 48 * 1024;
+};
 
-__device__ unsigned int g_tc_error;  // non-zero once a bounded wait gave up
+// First problem a tensor-core kernel recorded (0 = none): 0x1000 | role for
+// a bounded wait that gave up; 0x2000 | site for an index check that failed
+// (the access is skipped).  Read and cleared by moe_take_device_errors().
+__device__ unsigned int g_tc_error;
+__device__ unsigned int g_tc_error_info;
+__device__ __forceinline__ void record_error(unsigned code, unsigned info) {
+    if (atomicCAS(&g_tc_error, 0u, code) == 0u) g_tc_error_info = info;
+}
 
 struct TcParams {
     LayerView L;
+    int R;                 // rows of xs / h / rows (T * k)
     const int32_t *counts, *offsets;
+    int n_block;           // routes per block (multiple of 16, <= kNMax)
+    int b_slots;           // B ring slots of n_block * 128 bytes
     int K;                 // reduction length: H (phase 1) or I (phase 2)
     int n_units;           // output rows of the weight: 2I (phase 1) or H (phase 2)
     int64_t rows_per_blob; // expert_bytes / row_bytes
@@ -81,14 +113,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// try_wait suspends the thread in hardware until the phase completes or the
+// hint (ns) expires, so waiting roles do not spin on the issue slots.
+constexpr uint32_t kSuspendNs = 100000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -102,7 +137,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitCycles) {
             *abort_flag = 1;
-            atomicExch(&g_tc_error, 1u);
+            record_error(0x1000u | (threadIdx.x >> 5), (unsigned)((smem_u32(bar) << 1) | (parity & 1)));
             return false;
         }
     }
@@ -176,7 +211,7 @@ __device__ void build_items(const TcParams &p, int m_tiles, int *s_act, int *s_b
             const int n = (e < p.L.E) ? __ldg(p.counts + e) : 0;
             const bool act = n > 0;
             const unsigned m = __ballot_sync(0xffffffffu, act);
-            const int items = act ? m_tiles * ((n + kNMax - 1) / kNMax) : 0;
+            const int items = act ? m_tiles * ((n + p.n_block - 1) / p.n_block) : 0;
             int inc = items;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -216,9 +251,15 @@ __device__ __forceinline__ ItemInfo decode_item(const TcParams &p, const int *s_
     ItemInfo r;
     r.e = s_act[lo];
     const int n_e = __ldg(p.counts + r.e);
-    r.row0 = __ldg(p.offsets + r.e) + nb * kNMax;
-    r.n = min(kNMax, n_e - nb * kNMax);
+    r.row0 = __ldg(p.offsets + r.e) + nb * p.n_block;
+    r.n = min(p.n_block, n_e - nb * p.n_block);
     r.n_mma = (r.n + 15) & ~15;
+    if (r.n <= 0 || r.n_mma > p.n_block || r.row0 < 0 || r.row0 + r.n > p.R) {
+        record_error(0x2003u, (unsigned)item);
+        r.n = 0;       // nothing is written for an item that fails the check,
+        r.n_mma = 16;  // and its tiles stay inside their slots
+        r.row0 = 0;
+    }
     r.m0 = mt;  // tile index; callers scale it
     return r;
 }
@@ -232,29 +273,44 @@ __device__ __forceinline__ int a_row_coord(const TcParams &p, int e, int row, bo
 }
 
 // ---------------------------------------------------------------- the kernel
+template <int FMT>
+__host__ __device__ constexpr int kRawBytes() { return FMT == MOE_W_BF16 ? 0 : kRawRowBytes * kBlockM; }
+
+// warps: 0 A/raw producer, 1 MMA, 2..5 epilogue, 6 B producer, 7.. dequant
+constexpr int kWarpB = 2 + kEpiWarps;
+constexpr int kWarpDeq0 = kWarpB + 1;
+
+template <int FMT>
+__host__ __device__ constexpr int tc_threads() { return 32 * (kWarpDeq0 + (FMT == MOE_W_BF16 ? 0 : kDeqGroups * kDeqWarps)); }
+
 template <int FMT, int PHASE>
-__global__ void __launch_bounds__(32 * (6 + (FMT == MOE_W_BF16 ? 0 : kDeqWarps)), 1)
+__global__ void __launch_bounds__(tc_threads<FMT>(), 1)
 k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ CUtensorMap map_pool,
          const __grid_constant__ CUtensorMap map_b, const TcParams p) {
-    constexpr int S = TcFmt<FMT>::kStages;
-    constexpr int RAW = TcFmt<FMT>::kRawRowBytes * kBlockM;  // raw code bytes per stage
+    constexpr int SA = TcFmt<FMT>::kAStages;
+    constexpr int SR = TcFmt<FMT>::kRawStages;
+    constexpr int RAW = kRawBytes<FMT>();
+    constexpr int SUB = TcFmt<FMT>::kSub;
     constexpr bool kDeq = FMT != MOE_W_BF16;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte aligned carve-up: A tiles | B tiles | raw tiles | exchange | barriers
+    // 1024-byte aligned carve-up: A ring | B region | raw ring | exchange | barriers
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
-    uint8_t *sB = sA + S * kATileBytes;
-    uint8_t *sRaw = sB + S * kBTileBytes;
-    float *sX = reinterpret_cast<float *>(sRaw + S * RAW);        // [2][64][kXPitch] gate/up exchange
+    uint8_t *sB = sA + SA * kATileBytes;
+    uint8_t *sRaw = sB + TcFmt<FMT>::kBRegion;
+    float *sX = reinterpret_cast<float *>(sRaw + SR * RAW);       // [2][64][kXPitch] gate/up exchange
     uint64_t *bars = reinterpret_cast<uint64_t *>(sX + 2 * 64 * kXPitch);
-    uint64_t *full = bars;              // TMA bytes landed (A or raw, and B)
-    uint64_t *deq = bars + S;           // A tile ready in bf16 (int formats)
-    uint64_t *empty = bars + 2 * S;     // MMAs done reading the stage
-    uint64_t *tfull = bars + 3 * S;     // accumulator ready
-    uint64_t *tempty = bars + 3 * S + kAccBufs;  // accumulator drained
-    uint64_t *xfull = bars + 3 * S + 2 * kAccBufs;   // up values written to the exchange
-    uint64_t *xempty = xfull + 2;                    // exchange read by the gate warps
+    uint64_t *a_full = bars;                       // A tile ready (TMA bytes, or the dequant warps)
+    uint64_t *a_empty = a_full + SA;               // MMAs done reading the A tile
+    uint64_t *b_full = a_empty + SA;               // B tile landed
+    uint64_t *b_empty = b_full + kMaxBSlots;       // MMAs done reading the B tile
+    uint64_t *tfull = b_empty + kMaxBSlots;        // accumulator ready
+    uint64_t *tempty = tfull + kAccBufs;           // accumulator drained
+    uint64_t *xfull = tempty + kAccBufs;           // up values written to the exchange
+    uint64_t *xempty = xfull + 2;                  // exchange read by the gate warps
+    uint64_t *r_full = xempty + 2;                 // raw codes landed (int formats)
+    uint64_t *r_empty = r_full + SR;               // raw codes consumed by the dequant warps
 
     __shared__ int s_act[kMaxE];
     __shared__ int s_base[kMaxE + 1];
@@ -264,12 +320,17 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = PHASE == 1 ? p.L.I / 64 : (p.L.H + kBlockM - 1) / kBlockM;
+    const int nk = p.K / kBlockK;
+    const uint32_t b_slot_bytes = (uint32_t)p.n_block * 128;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&deq[s], kDeqWarps);
-            mbar_init(&empty[s], 1);
+        for (int i = 0; i < SA; ++i) {
+            mbar_init(&a_full[i], kDeq ? kDeqWarps : 1);
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < kMaxBSlots; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
         }
         for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(&tfull[b], 1);
@@ -278,6 +339,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         for (int b = 0; b < 2; ++b) {
             mbar_init(&xfull[b], 2);
             mbar_init(&xempty[b], 2);
+        }
+        for (int r = 0; r < SR; ++r) {
+            mbar_init(&r_full[r], 1);
+            mbar_init(&r_empty[r], kDeqGroups * kDeqWarps);
         }
         s_abort = 0;
         fence_barrier_init();
@@ -296,14 +361,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     const int n_act = s_items.n_act, total = s_items.total;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+        // ------------------------------------- A producer: weights or raw codes
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
                 const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
                 bool pool;
-                int ya0, ya1;  // A row coordinates of the two 64-row halves
+                int ya0, ya1;  // row coordinates of the two 64-row halves of the tile
                 if (PHASE == 1) {
                     ya0 = a_row_coord(p, it.e, it.m0 * 64, &pool);
                     ya1 = a_row_coord(p, it.e, p.L.I + it.m0 * 64, &pool);
@@ -312,33 +377,53 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     ya1 = ya0 + 64;
                 }
                 const CUtensorMap *ma = pool ? &map_pool : &map_home;
-                const uint32_t a_bytes = kDeq ? (uint32_t)RAW : kATileBytes;
-                const uint32_t bytes = a_bytes + (uint32_t)it.n_mma * kBlockK * 2;
-                for (int kk = 0; kk < p.K / kBlockK; ++kk) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, &s_abort)) break;
-                    mbar_arrive_expect_tx(&full[stage], bytes);
-                    if (kDeq) {
+                bool ok = true;
+                if (kDeq) {
+                    for (int rs = 0; rs < (nk + SUB - 1) / SUB; ++rs) {
+                        if (!mbar_wait(&r_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&r_full[stage], (uint32_t)RAW);
                         uint8_t *dst = sRaw + stage * RAW;
-                        const int xb = kk * TcFmt<FMT>::kRawRowBytes;
-                        tma_load_2d(dst, ma, &full[stage], xb, ya0);
-                        tma_load_2d(dst + 64 * TcFmt<FMT>::kRawRowBytes, ma, &full[stage], xb, ya1);
-                    } else {
-                        uint8_t *dst = sA + stage * kATileBytes;
-                        tma_load_2d(dst, ma, &full[stage], kk * kBlockK, ya0);
-                        tma_load_2d(dst + kATileBytes / 2, ma, &full[stage], kk * kBlockK, ya1);
+                        tma_load_2d(dst, ma, &r_full[stage], rs * kRawRowBytes, ya0);
+                        tma_load_2d(dst + 64 * kRawRowBytes, ma, &r_full[stage], rs * kRawRowBytes, ya1);
+                        if (++stage == SR) { stage = 0; phase ^= 1; }
                     }
-                    uint8_t *db = sB + stage * kBTileBytes;
-                    for (int j = 0; j < it.n_mma; j += 16)
-                        tma_load_2d(db + j * 128, &map_b, &full[stage], kk * kBlockK, it.row0 + j);
-                    if (++stage == S) { stage = 0; phase ^= 1; }
+                } else {
+                    for (int kk = 0; kk < nk; ++kk) {
+                        if (!mbar_wait(&a_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&a_full[stage], kATileBytes);
+                        uint8_t *dst = sA + stage * kATileBytes;
+                        tma_load_2d(dst, ma, &a_full[stage], kk * kBlockK, ya0);
+                        tma_load_2d(dst + kATileBytes / 2, ma, &a_full[stage], kk * kBlockK, ya1);
+                        if (++stage == SA) { stage = 0; phase ^= 1; }
+                    }
                 }
+                if (!ok) break;
+            }
+        }
+    } else if (warp == kWarpB) {
+        // ------------------------------------------------ B producer: routes
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
+                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+                bool ok = true;
+                for (int kk = 0; kk < nk; ++kk) {
+                    if (!mbar_wait(&b_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&b_full[stage], (uint32_t)it.n_mma * 128);
+                    uint8_t *db = sB + stage * b_slot_bytes;
+                    for (int j = 0; j < it.n_mma; j += 16)
+                        tma_load_2d(db + j * 128, &map_b, &b_full[stage], kk * kBlockK, it.row0 + j);
+                    if (++stage == p.b_slots) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
+            int sa = 0, sb = 0;
+            uint32_t pa = 0, pb = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
@@ -349,16 +434,19 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                 const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(it.n_mma >> 3) << 17) |
                                        ((uint32_t)(kBlockM >> 4) << 24);
                 bool ok = true;
-                for (int kk = 0; kk < p.K / kBlockK; ++kk) {
-                    if (!mbar_wait(kDeq ? &deq[stage] : &full[stage], phase, &s_abort)) { ok = false; break; }
+                for (int kk = 0; kk < nk; ++kk) {
+                    if (!mbar_wait(&a_full[sa], pa, &s_abort)) { ok = false; break; }
+                    if (!mbar_wait(&b_full[sb], pb, &s_abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * kATileBytes);
-                    const uint32_t b0 = smem_u32(sB + stage * kBTileBytes);
+                    const uint32_t a0 = smem_u32(sA + sa * kATileBytes);
+                    const uint32_t b0 = smem_u32(sB + sb * b_slot_bytes);
 #pragma unroll
                     for (int j = 0; j < kBlockK / 16; ++j)
                         tc_mma_bf16(d, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc, (kk | j) != 0);
-                    tc_commit(&empty[stage]);
-                    if (++stage == S) { stage = 0; phase ^= 1; }
+                    tc_commit(&a_empty[sa]);
+                    tc_commit(&b_empty[sb]);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (++sb == p.b_slots) { sb = 0; pb ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit(&tfull[acc]);
@@ -407,6 +495,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                         for (int i = 0; i < 16; ++i) {
                             const int j = c0 + i;
                             if (j < it.n) {
+                                if (it.row0 + j >= p.R || icol >= p.L.I || it.row0 + j < 0) {
+                                    record_error(0x2001u, (unsigned)(it.row0 + j));
+                                    continue;
+                                }
                                 const float g = v[i] * scale, up = xrow[i];
                                 p.h[(size_t)(it.row0 + j) * p.L.I + icol] = f32_to_bf16_rne(gelu_tanh(g) * up);
                             }
@@ -421,7 +513,13 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int j = c0 + i;
-                            if (j < it.n) p.rows[(size_t)(it.row0 + j) * p.L.H + m] = v[i] * scale;
+                            if (j < it.n) {
+                                if (it.row0 + j >= p.R || it.row0 + j < 0) {
+                                    record_error(0x2002u, (unsigned)(it.row0 + j));
+                                    continue;
+                                }
+                                p.rows[(size_t)(it.row0 + j) * p.L.H + m] = v[i] * scale;
+                            }
                         }
                     }
                 }
@@ -437,10 +535,13 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         // two threads per tile row (half a row, 32 weights = 4 chunks, each):
         // raw codes -> bf16 in the 128-byte-swizzled K-major layout (8-row groups
         // of 1024 bytes, 16-byte chunk c of row r stored at chunk c ^ (r % 8)).
-        const int t = (warp - 2 - kEpiWarps) * 32 + lane;
+        const int dw = warp - kWarpDeq0;              // 0 .. kDeqGroups*kDeqWarps-1
+        const int group = dw / kDeqWarps;
+        const int t = (dw % kDeqWarps) * 32 + lane;
         const int r = t & (kBlockM - 1), hf = t >> 7;
-        int stage = 0;
-        uint32_t phase = 0;
+        int stage = 0, rstage = 0;
+        uint32_t phase = 0, rphase = 0;
+        uint32_t step = 0;                              // k-steps seen, across items
         for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
             const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
             const uint8_t *blob = expert_blob(p.L, it.e);
@@ -449,25 +550,40 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             const uint16_t *srow = reinterpret_cast<const uint16_t *>(blob + (PHASE == 1 ? p.L.off.s13 : p.L.off.s2)) +
                                    (size_t)wrow * (p.K / 64);
             bool ok = true;
-            for (int kk = 0; kk < p.K / kBlockK; ++kk) {
+            for (int kk = 0; kk < nk; ++kk, ++step) {
+                const int sub = kk % SUB;
+                const bool raw_last = sub == SUB - 1 || kk == nk - 1;  // last MMA stage of this raw stage
+                if ((int)(step % kDeqGroups) != group) {   // the other group's stage
+                    if (++stage == SA) { stage = 0; phase ^= 1; }
+                    if (raw_last) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&r_empty[rstage]);
+                        if (++rstage == SR) { rstage = 0; rphase ^= 1; }
+                    }
+                    continue;
+                }
                 __nv_bfloat162 s2 = __floats2bfloat162_rn(0.0f, 0.0f);
                 if (FMT == MOE_W_INT4) s2 = __bfloat162bfloat162(__ushort_as_bfloat16(__ldg(srow + kk)));
-                if (!mbar_wait(&full[stage], phase, &s_abort)) { ok = false; break; }
-                const uint8_t *src = sRaw + stage * RAW + r * TcFmt<FMT>::kRawRowBytes;
+                // the codes have landed, and the MMAs are done with this A slot
+                if (!mbar_wait(&r_full[rstage], rphase, &s_abort)) { ok = false; break; }
+                if (!mbar_wait(&a_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
+                const uint8_t *src = sRaw + rstage * RAW + r * kRawRowBytes + sub * TcFmt<FMT>::kSubBytes;
                 uint8_t *dst = sA + stage * kATileBytes + (r >> 3) * 1024 + (r & 7) * 128;
                 if (FMT == MOE_W_INT4) {
                     // 16 raw bytes = weights 32hf .. 32hf+31 = chunks 4hf .. 4hf+3
                     const uint4 u = *reinterpret_cast<const uint4 *>(src + 16 * hf);
                     const uint32_t words[4] = {u.x, u.y, u.z, u.w};
+                    // bf16 128 + n (n in the low mantissa bits of 128.0 = 0x4300),
+                    // minus 136 -> n - 8 exactly, times s -> one rounding
                     const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        // byte j of the word = weight 2j (low nibble), 2j+1 (high):
-                        // pair -> bf16x2 {128 + n_lo, 128 + n_hi} -> minus 136 -> times s
+                        // byte j of the word = weight 2j (low nibble), 2j+1 (high)
                         const uint32_t w = words[i], w4 = w >> 4;
                         uint32_t o[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
+                            // {w.byte j, -, (w >> 4).byte j, -}: n_lo and n_hi in the low bits of each half
                             const uint32_t dup = __byte_perm(w, w4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
                             uint32_t v = (dup & 0x000F000Fu) | 0x43004300u;
                             __nv_bfloat162 q = *reinterpret_cast<__nv_bfloat162 *>(&v);
@@ -498,8 +614,12 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&deq[stage]);
-                if (++stage == S) { stage = 0; phase ^= 1; }
+                if (lane == 0) {
+                    mbar_arrive(&a_full[stage]);
+                    if (raw_last) mbar_arrive(&r_empty[rstage]);
+                }
+                if (++stage == SA) { stage = 0; phase ^= 1; }
+                if (raw_last && ++rstage == SR) { rstage = 0; rphase ^= 1; }
             }
             if (!ok) break;
         }
@@ -524,7 +644,12 @@ __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__r
          i += (int64_t)gridDim.x * blockDim.x) {
         const int s = (int)(i / per), c = (int)(i % per);
         if (s >= n_valid) continue;
-        const int tok = __ldg(sorted_route + s) / k;
+        const int route = __ldg(sorted_route + s);
+        const int tok = route / k;
+        if (route < 0 || route >= R) {
+            record_error(0x2004u, (unsigned)s);
+            continue;
+        }
         reinterpret_cast<uint4 *>(xs + (size_t)s * H)[c] =
             __ldg(reinterpret_cast<const uint4 *>(x + (size_t)tok * H) + c);
     }
@@ -556,18 +681,23 @@ bool encode_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int ele
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t smem_bytes(int fmt) {
-    const int S = fmt == MOE_W_BF16 ? TcFmt<MOE_W_BF16>::kStages
-                                    : (fmt == MOE_W_INT8 ? TcFmt<MOE_W_INT8>::kStages : TcFmt<MOE_W_INT4>::kStages);
-    const int raw = fmt == MOE_W_BF16 ? 0 : (fmt == MOE_W_INT8 ? 64 : 32) * kBlockM;
-    return 1024 + (size_t)S * (kATileBytes + kBTileBytes + raw) + 2 * 64 * kXPitch * 4 + (3 * S + 2 * kAccBufs + 4) * 8;
+template <int FMT>
+constexpr size_t smem_bytes() {
+    return 1024 + (size_t)TcFmt<FMT>::kAStages * kATileBytes + TcFmt<FMT>::kBRegion +
+           (size_t)TcFmt<FMT>::kRawStages * kRawBytes<FMT>() + 2 * 64 * kXPitch * 4 +
+           (size_t)(2 * TcFmt<FMT>::kAStages + 2 * kMaxBSlots + 2 * kAccBufs + 4 + 2 * TcFmt<FMT>::kRawStages) * 8;
 }
+// dynamic + static shared memory (s_act, s_base, ...: 9216 bytes) within the
+// 232448-byte per-block limit
+static_assert(smem_bytes<MOE_W_BF16>() + 9216 <= 232448, "bf16 tensor-core kernel exceeds shared memory");
+static_assert(smem_bytes<MOE_W_INT8>() + 9216 <= 232448, "int8 tensor-core kernel exceeds shared memory");
+static_assert(smem_bytes<MOE_W_INT4>() + 9216 <= 232448, "int4 tensor-core kernel exceeds shared memory");
 
 template <int FMT, int PHASE>
 cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUtensorMap &mb, const TcParams &p,
                        int n_sm, cudaStream_t s) {
     auto kern = k_ffn_tc<FMT, PHASE>;
-    const size_t smem = smem_bytes(FMT);
+    const size_t smem = smem_bytes<FMT>();
     static bool attr[kMaxDevices] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -578,8 +708,7 @@ cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUten
         if (err != cudaSuccess) return err;
         attr[dev] = true;
     }
-    const int threads = 32 * (6 + (FMT == MOE_W_BF16 ? 0 : kDeqWarps));
-    kern<<<n_sm, threads, smem, s>>>(mh, mp, mb, p);
+    kern<<<n_sm, tc_threads<FMT>(), smem, s>>>(mh, mp, mb, p);
     return cudaGetLastError();
 }
 
@@ -627,7 +756,7 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     const CUtensorMapDataType dt = bf ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     const int eb = bf ? 2 : 1;
     const CUtensorMapSwizzle swa = bf ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
-    const uint32_t raw_inner = fmt == MOE_W_INT8 ? 64 : 32;
+    const uint32_t raw_inner = kRawRowBytes;
     CUtensorMap mh1, mp1, mh2, mp2, mb1, mb2;
     for (int ph = 1; ph <= 2; ++ph) {
         const int K = ph == 1 ? H : I;
@@ -648,10 +777,20 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     }
     TcParams p{};
     p.L = L;
+    p.R = R;
     p.counts = counts;
     p.offsets = offsets;
+    // route block: an expert never gets a token twice, so min(T, 128) rows hold
+    // all of an expert's routes in one block (measured best: smaller blocks
+    // re-stream the weights of busier experts)
+    p.n_block = std::min(kNMax, (std::max(T, 1) + 15) / 16 * 16);
+    p.b_slots = std::min(kMaxBSlots, (fmt == MOE_W_BF16 ? TcFmt<MOE_W_BF16>::kBRegion : TcFmt<MOE_W_INT4>::kBRegion) /
+                                         (p.n_block * 128));
     p.h = h;
     p.rows = rows;
+    // every pointer the kernels write through must be set (host-side guard)
+    if (p.h == nullptr || p.rows == nullptr || p.counts == nullptr || p.offsets == nullptr || xs == nullptr)
+        return cudaErrorInvalidValue;
     // phase 1
     {
         const uint64_t rb = bf ? (uint64_t)H * 2 : (fmt == MOE_W_INT8 ? (uint64_t)H : (uint64_t)H / 2);
@@ -678,11 +817,12 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     return err;
 }
 
-cudaError_t tc_take_error(unsigned *out) {
+cudaError_t tc_take_error(unsigned *code, unsigned *info) {
     unsigned zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(out, g_tc_error, sizeof(unsigned));
-    if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(unsigned));
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_tc_error, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(info, g_tc_error_info, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(unsigned));
+    return e;
 }
 
 }  // namespace moe

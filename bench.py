@@ -48,6 +48,9 @@ import numpy as np  # noqa: E402
 NCU_TRAFFIC_BYTES = {
     # profiles/ffn_gemv_bf16_T64.md: phase 1 1.0059 GB + 4.04 MB, phase 2 0.5027 GB + 5.28 MB
     ("decode-bf16", 64, "gemv"): 1.5180e9,
+    # profiles/ffn_tc_bf16_decode_T64.md: phase 1 1.0027 GB + 5.00 MB, phase 2 0.5004 GB + 8.40 MB
+    ("decode-bf16", 64, "auto"): 1.5165e9,
+    ("decode-bf16", 64, "tc"): 1.5165e9,
 }
 
 CONFIGS = {
@@ -346,15 +349,16 @@ def cpu_baseline(moe, torch, cfg_fmt, layers, batches, T, k, seconds, first_toke
     threads = oracle.get_threads()
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.moe_layer(OL, lg[n:n + 1], x[n:n + 1], k)
+        t = n % T  # cycle through the batch's tokens until the time budget is spent
+        oracle.moe_layer(OL, lg[t:t + 1], x[t:t + 1], k)
         n += 1
         el = time.perf_counter() - t0
-        if el >= seconds or n >= T or first_token_only:
+        if el >= seconds or first_token_only:
             break
     del home_host
     return {"value": n / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} of the {T} tokens of one batch ({n * k} routes), whole layer "
-                      f"(route, per-route fp64 FFN, combine), {el:.1f} s"}
+            "sample": f"{n} token evaluations cycling through the {T} tokens of one batch ({n * k} routes), "
+                      f"whole layer (route, per-route fp64 FFN, combine), {el:.1f} s"}
 
 
 def main():

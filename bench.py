@@ -82,6 +82,25 @@ def parse():
     return ap.parse_args()
 
 
+# --------------------------------------------------------------- multi-rank
+
+def max_over_ranks(dist, value: float, device=None) -> float:
+    """The slowest rank's time: every rank passes its own elapsed ms and gets the
+    maximum (replicas run the same workload; the job is as fast as its slowest)."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -403,12 +422,9 @@ def main():
     ms, ffn_ms = time_steps(torch, runner, args.steps, args.warmup, dist)
     clk = clocks.stop()
 
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(dist, ms, dev)
     ms_step = ms / args.steps
-    value = world * T * args.steps / (ms / 1e3)
+    value = whole_job_rate(T * args.steps, world, ms)
 
     # roofline of the dominant kernel (the grouped FFN: two launches per step)
     eb = moe.moe_expert_bytes(moe.FMT[fmt_name], H, I)
@@ -429,10 +445,7 @@ def main():
         r2 = Runner(moe, torch, layers, b2, Ts, k, dev, path)
         d2 = r2.distinct_experts()
         ms2, ffn2 = time_steps(torch, r2, args.steps, args.warmup, dist)
-        if dist is not None:
-            t = torch.tensor([ms2], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms2 = float(t.item())
+        ms2 = max_over_ranks(dist, ms2, dev)
         dd = sum(d2) / len(d2)
         f2 = sum(ffn2) / len(ffn2)
         sweep_out[f"T{Ts}"] = {
@@ -446,10 +459,7 @@ def main():
 
     e2e_ms, h2d, d2h = (float("nan"), 0, 0) if args.quick else time_e2e(torch, moe, layers, batches, T, k,
                                                                          args.steps, args.warmup, dev)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(dist, e2e_ms, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:

@@ -67,6 +67,7 @@ def _L():
         c.oracle_bf16_rne.argtypes = [ctypes.c_float]
         c.oracle_route_topk.argtypes = [P, i32, i32, i32, P, P]
         c.oracle_permute.argtypes = [P, i32, i32, i32, P, P, P, P]
+        c.oracle_route_min_weight.argtypes = [P, P, P, i32, i32, i32, ctypes.c_float]
         c.oracle_hits.argtypes = [P, i64, i32, P]
         c.oracle_quantize_int8.argtypes = [P, i32, i32, P, P]
         c.oracle_quantize_int4.argtypes = [P, i32, i32, P, P]
@@ -141,6 +142,16 @@ def route_topk(logits: np.ndarray, k: int):
     ids = np.zeros((T, k), np.int32)
     w = np.zeros((T, k), np.float32)
     _L().oracle_route_topk(_p(logits), T, E, k, _p(ids), _p(w))
+    return ids, w
+
+
+def route_min_weight(ids: np.ndarray, w: np.ndarray, slot_table, E: int, min_weight: float):
+    """Returns new (ids, w) after [miss] min_weight partial routing."""
+    ids = _c(ids, np.int32).copy()
+    w = _c(w, np.float32).copy()
+    T, k = ids.shape
+    st = None if slot_table is None else _c(slot_table, np.int32)
+    _L().oracle_route_min_weight(_p(ids), _p(w), None if st is None else _p(st), T, k, E, float(min_weight))
     return ids, w
 
 

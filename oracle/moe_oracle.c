@@ -243,6 +243,49 @@ void oracle_route_topk(const float *logits, int T, int E, int k, int32_t *ids, f
     free(e);
 }
 
+/*
+ * [miss] min_weight (prain README.md, "Trading quality for speed"): a
+ * per-token threshold on the fraction of the router weight whose experts are
+ * actually evaluated.  With the threshold below 1, light routes to experts held
+ * outside VRAM may be left out once enough weight is covered, and the weights
+ * that remain are enlarged so they again add up to the token's total.  Reading,
+ * per token, in fp32:
+ *   walk the routes in rank order (heaviest first) keeping a running sum `kept`
+ *   of the weights kept so far; a route whose expert has no cache slot
+ *   (slot_table[e] < 0, or no table) is dropped when kept >= min_weight,
+ *   otherwise kept (kept = kept + w_j).  min_weight >= 1 changes nothing.
+ *   Then total = sum of all k weights (in order) and every kept weight becomes
+ *   w_j * (total / kept); a dropped route gets id -1 and weight 0.  If nothing is
+ *   kept (min_weight <= 0 and no resident expert) every route is dropped.
+ */
+void oracle_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, int T, int k, int E,
+                             float min_weight)
+{
+    if (!(min_weight < 1.0f)) return;
+    for (int t = 0; t < T; ++t) {
+        int32_t *id = ids + (size_t)t * k;
+        float *wt = w + (size_t)t * k;
+        float kept = 0.0f, total = 0.0f;
+        char drop[64];
+        for (int j = 0; j < k; ++j) {
+            int e = id[j];
+            int resident = slot_table != NULL && e >= 0 && e < E && slot_table[e] >= 0;
+            drop[j] = (!resident && kept >= min_weight);
+            if (!drop[j]) kept = kept + wt[j];
+        }
+        for (int j = 0; j < k; ++j) total = total + wt[j];
+        float r = kept > 0.0f ? total / kept : 0.0f;
+        for (int j = 0; j < k; ++j) {
+            if (drop[j] || kept <= 0.0f) {
+                id[j] = -1;
+                wt[j] = 0.0f;
+            } else {
+                wt[j] = wt[j] * r;
+            }
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ permute */
 /*
  * Group the R = T*k routes by expert (Winery-Strata remote_experts.cpp,

@@ -60,6 +60,11 @@ uint16_t oracle_bf16_rne(float f);
 /* routing: ids [T,k] (descending logit, ties to the lower id), w [T,k] */
 void oracle_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w);
 
+/* [miss] min_weight partial routing: drop a token's lightest non-resident routes
+ * once the kept share reaches min_weight; rescale the kept weights (in place) */
+void oracle_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, int T, int k, int E,
+                             float min_weight);
+
 /* stable counting sort of the T*k routes by expert id */
 void oracle_permute(const int32_t *ids, int T, int k, int E, int32_t *counts, int32_t *offsets,
                     int32_t *sorted_route, int32_t *route_pos);

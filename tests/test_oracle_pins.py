@@ -524,3 +524,70 @@ def test_placement_invariants_under_random_refreshes():
         assert all(before[e] < 0 for e in pr) and all(before[e] >= 0 for e in de)
         for p, d in zip(pr, de):
             assert so[p] == before[d]                     # promoted takes the demoted slot
+
+
+# ------------------------------------------------------------ [miss] min_weight
+
+def _mw_case(seed, T=200, E=32, k=8, resident_frac=0.4):
+    rng = np.random.default_rng(seed)
+    lg = syn.router_logits(T, E, "zipf", seed=seed)
+    ids, w = oracle.route_topk(lg, k)
+    slot = np.where(rng.random(E) < resident_frac, np.arange(E), -1).astype(np.int32)
+    return ids, w, slot
+
+
+def test_min_weight_one_or_all_resident_changes_nothing():
+    ids, w, slot = _mw_case(1)
+    for mw in (1.0, 1.5):
+        i2, w2 = oracle.route_min_weight(ids, w, slot, 32, mw)
+        assert np.array_equal(i2, ids) and np.array_equal(w2, w)
+    i3, w3 = oracle.route_min_weight(ids, w, np.arange(32, dtype=np.int32), 32, 0.3)
+    assert np.array_equal(i3, ids) and np.array_equal(w3, w)
+
+
+def test_min_weight_keeps_the_share_and_the_full_weight():
+    """Kept share before rescaling >= min_weight (or every route kept); dropped
+    routes are non-resident and lighter than every kept non-resident route; kept
+    weights sum back to the token's full weight."""
+    ids, w, slot = _mw_case(2)
+    for mw in (0.2, 0.5, 0.8, 0.95):
+        i2, w2 = oracle.route_min_weight(ids, w, slot, 32, mw)
+        for t in range(ids.shape[0]):
+            kept = i2[t] >= 0
+            dropped = ~kept
+            if dropped.any():
+                assert w[t][kept].astype(np.float64).sum() >= mw - 1e-6
+                assert all(slot[e] < 0 for e in ids[t][dropped])
+                nonres_kept = [j for j in np.nonzero(kept)[0] if slot[ids[t][j]] < 0]
+                if nonres_kept:
+                    assert w[t][dropped].max() <= w[t][nonres_kept].min()
+            assert abs(w2[t].astype(np.float64).sum() - w[t].astype(np.float64).sum()) < 1e-5
+            assert np.all(w2[t][dropped] == 0)
+
+
+def test_min_weight_is_monotone_and_zero_keeps_only_resident():
+    ids, w, slot = _mw_case(3)
+    prev = None
+    for mw in (0.95, 0.7, 0.4, 0.1):
+        i2, _ = oracle.route_min_weight(ids, w, slot, 32, mw)
+        drops = i2 < 0
+        if prev is not None:
+            assert np.all(drops[prev])   # lowering min_weight never brings a route back
+        prev = drops
+    i0, w0 = oracle.route_min_weight(ids, w, slot, 32, 0.0)
+    res = slot[ids] >= 0
+    assert np.array_equal(i0 >= 0, res)
+    none = ~res.any(axis=1)
+    assert np.all(w0[none] == 0)
+
+
+def test_min_weight_hand_example():
+    ids = np.array([[3, 0, 2, 1]], np.int32)
+    w = np.array([[0.5, 0.25, 0.125, 0.125]], np.float32)
+    slot = np.array([-1, 0, -1, -1], np.int32)   # only expert 1 is resident
+    i2, w2 = oracle.route_min_weight(ids, w, slot, 4, 0.6)
+    # 0.5 kept (share 0.5 < 0.6), 0.25 kept (share 0.75), expert 2 dropped (non-resident,
+    # share reached), expert 1 kept (resident); scale 1 / 0.875
+    assert i2.tolist() == [[3, 0, -1, 1]]
+    np.testing.assert_array_equal(w2, np.float32([[0.5 * np.float32(1 / 0.875), 0.25 * np.float32(1 / 0.875), 0,
+                                                   0.125 * np.float32(1 / 0.875)]]))

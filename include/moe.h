@@ -124,6 +124,21 @@ MOE_API moe_status moe_route_topk(const float *logits, int32_t T, int32_t E, int
                           moe_stream_t stream);
 
 /*
+ * [miss] min_weight partial routing (prain README.md, "Trading quality for
+ * speed"), applied in place to the output of moe_route_topk.  Per token, routes
+ * are taken heaviest first with a running sum `kept` of the weights kept so far
+ * (fp32, in order); a route whose expert has no cache slot (slot_table[e] < 0,
+ * or slot_table NULL) is dropped once kept >= min_weight.  Dropped routes get
+ * id -1 (moe_permute then leaves them out) and weight 0; every kept weight is
+ * multiplied by total / kept (fp32, IEEE), so the kept weights again sum to the
+ * token's total.  min_weight >= 1 is a no-op; a token with nothing kept (only
+ * possible for min_weight <= 0) has all its routes dropped and contributes 0.
+ * ids int32 [T][k], w fp32 [T][k], slot_table int32 [E] (device, nullable).
+ */
+MOE_API moe_status moe_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, int32_t T, int32_t k,
+                                        int32_t E, float min_weight, moe_stream_t stream);
+
+/*
  * Stable counting sort of the R = T*k routes by expert (remote_experts.cpp,
  * RemoteExperts::begin: a route r belongs to token r / k; inside an expert's
  * group the routes keep ascending r).  Groups are laid out by ascending

@@ -36,6 +36,7 @@ EXPORTS = [
     "moe_layer_forward_workspace", "moe_layer_forward", "moe_quantize_int8", "moe_quantize_int4",
     "moe_pack_expert", "moe_copy_to_slots", "moe_refresh_target", "moe_apply_placement",
     "moe_should_refresh", "moe_budget_from_vram", "moe_grouped_ffn_noalloc", "moe_take_device_errors",
+    "moe_route_min_weight",
 ]
 
 
@@ -79,6 +80,7 @@ _SIG = {
     "moe_budget_from_vram": (i64, [i64, i64, i64, i64, i64, i64]),
     "moe_grouped_ffn_noalloc": (i32, [LP, P, i32, i32, P, P, P, P, P]),
     "moe_take_device_errors": (i32, [P, P]),
+    "moe_route_min_weight": (i32, [P, P, P, i32, i32, i32, ctypes.c_float, P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -171,6 +173,16 @@ def moe_route_topk(logits: torch.Tensor, k: int, ids: torch.Tensor | None = None
     w = torch.empty((T, k), dtype=torch.float32, device=logits.device) if w is None else w
     _check(_lib.moe_route_topk(_dev(logits, torch.float32, "logits"), T, E, k, _dev(ids, torch.int32, "ids"),
                                _dev(w, torch.float32, "w"), _stream(stream)))
+    return ids, w
+
+
+def moe_route_min_weight(ids: torch.Tensor, w: torch.Tensor, E: int, min_weight: float,
+                         slot_table: torch.Tensor | None = None, stream=None):
+    """In place: [miss] min_weight partial routing of moe_route_topk's output."""
+    T, k = ids.shape
+    _check(_lib.moe_route_min_weight(_dev(ids, torch.int32, "ids"), _dev(w, torch.float32, "w"),
+                                     None if slot_table is None else _dev(slot_table, torch.int32, "slot_table"),
+                                     T, k, E, float(min_weight), _stream(stream)))
     return ids, w
 
 

@@ -9,6 +9,7 @@
 namespace moe {
 
 cudaError_t launch_route_topk(const float *, int, int, int, int32_t *, float *, cudaStream_t);
+cudaError_t launch_route_min_weight(int32_t *, float *, const int32_t *, int, int, int, float, cudaStream_t);
 cudaError_t launch_permute(const int32_t *, int, int, int32_t *, int32_t *, int32_t *, int32_t *, uint32_t *,
                            cudaStream_t);
 cudaError_t launch_expert_hits(const int32_t *, int64_t, int, uint32_t *, cudaStream_t);
@@ -121,6 +122,18 @@ moe_status moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k, 
     if (T == 0) return MOE_OK;
     CHECK_ARG(logits && ids && w, "moe_route_topk: NULL pointer");
     return cuda_status(launch_route_topk(logits, T, E, k, ids, w, (cudaStream_t)stream), "moe_route_topk launch");
+}
+
+moe_status moe_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, int32_t T, int32_t k, int32_t E,
+                                float min_weight, moe_stream_t stream) {
+    moe_status st = check_shape(E, k, 64, 64);
+    if (st != MOE_OK) return st;
+    if ((st = check_tk(T, k)) != MOE_OK) return st;
+    CHECK_ARG(min_weight == min_weight, "min_weight is NaN");
+    if (T == 0 || !(min_weight < 1.0f)) return MOE_OK;
+    CHECK_ARG(ids && w, "moe_route_min_weight: NULL pointer");
+    return cuda_status(launch_route_min_weight(ids, w, slot_table, T, k, E, min_weight, (cudaStream_t)stream),
+                       "moe_route_min_weight launch");
 }
 
 moe_status moe_permute(const int32_t *ids, int32_t T, int32_t k, int32_t E, int32_t *counts, int32_t *offsets,

@@ -116,7 +116,44 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
     }
 }
 
+// [miss] min_weight partial routing, one thread per token: heaviest route
+// first, a route whose expert has no cache slot is dropped once the kept weight
+// has reached min_weight; the kept weights are scaled by total / kept.
+__global__ void __launch_bounds__(256) k_route_min_weight(int32_t *__restrict__ ids, float *__restrict__ w,
+                                                          const int32_t *__restrict__ slot_table, int T, int k,
+                                                          int E, float min_weight) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    int32_t *id = ids + (size_t)t * k;
+    float *wt = w + (size_t)t * k;
+    uint32_t dropped = 0;
+    float kept = 0.0f, total = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const int e = id[j];
+        const bool resident = slot_table != nullptr && e >= 0 && e < E && __ldg(slot_table + e) >= 0;
+        if (!resident && kept >= min_weight) dropped |= 1u << j;
+        else kept = __fadd_rn(kept, wt[j]);
+    }
+    for (int j = 0; j < k; ++j) total = __fadd_rn(total, wt[j]);
+    const float scale = kept > 0.0f ? __fdiv_rn(total, kept) : 0.0f;
+    for (int j = 0; j < k; ++j) {
+        if (((dropped >> j) & 1u) || !(kept > 0.0f)) {
+            id[j] = -1;
+            wt[j] = 0.0f;
+        } else {
+            wt[j] = __fmul_rn(wt[j], scale);
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, int T, int k, int E,
+                                    float min_weight, cudaStream_t s) {
+    if (T == 0 || !(min_weight < 1.0f)) return cudaSuccess;
+    k_route_min_weight<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(ids, w, slot_table, T, k, E, min_weight);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w,
                               cudaStream_t s) {

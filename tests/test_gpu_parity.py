@@ -406,3 +406,42 @@ def test_tc_and_gemv_agree_on_the_slot_table():
     b = _tc_or_skip(L2, lg, x, k)[-2]
     n = a.shape[0]
     assert rel_err(b.cpu().numpy()[:n], a.cpu().numpy()) <= FFN_TOL
+
+
+# ------------------------------------------------------- [miss] min_weight
+
+@pytest.mark.parametrize("mw", [0.0, 0.3, 0.6, 0.95, 1.0])
+def test_route_min_weight_bit_exact(mw):
+    T, E, k = 300, 128, 8
+    lg = syn.router_logits(T, E, "zipf", seed=31)
+    oi, ow = oracle.route_topk(lg, k)
+    slot = np.where(np.random.default_rng(4).random(E) < 0.15, np.arange(E), -1).astype(np.int32)
+    ids = torch.from_numpy(oi).to(DEV)
+    w = torch.from_numpy(ow).to(DEV)
+    moe.moe_route_min_weight(ids, w, E, mw, slot_table=torch.from_numpy(slot).to(DEV))
+    ri, rw = oracle.route_min_weight(oi, ow, slot, E, mw)
+    assert np.array_equal(ids.cpu().numpy(), ri)
+    assert bits_equal(w.cpu().numpy(), rw)
+
+
+def test_layer_with_min_weight_matches_oracle():
+    """The whole layer with partial routing: dropped routes join no group and add
+    nothing; the kept ones carry the rescaled weights."""
+    E, H, I, k, T = 16, 512, 128, 4, 40
+    w13, w2 = syn.expert_weights(E, H, I, seed=9)
+    L = moe.make_layer(0, *device_weights_from_host(w13, w2))
+    x = syn.activations(T, H, seed=9)
+    lg = syn.router_logits(T, E, "zipf", seed=9)
+    slot = np.where(np.arange(E) % 3 == 0, np.arange(E), -1).astype(np.int32)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    ids, w = moe.moe_route_topk(torch.from_numpy(lg).to(DEV), k)
+    moe.moe_route_min_weight(ids, w, E, 0.5, slot_table=torch.from_numpy(slot).to(DEV))
+    counts, offsets, sr, rp = moe.moe_permute(ids, E)
+    rows = moe.moe_grouped_ffn(L, xd, k, counts, offsets, sr)
+    y = moe.moe_combine(rows, rp, w)
+    oi, ow = oracle.route_topk(lg, k)
+    oi, ow = oracle.route_min_weight(oi, ow, slot, E, 0.5)
+    OL = oracle_layer_for(0, w13, w2)
+    oy = oracle.combine(oracle.ffn_routes(OL, x, oi), oi, ow, E)
+    assert (oi < 0).any()
+    assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL

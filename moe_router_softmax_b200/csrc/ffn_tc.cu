@@ -89,8 +89,7 @@ struct TcParams {
     LayerView L;
     int R;                 // rows of xs / h / rows (T * k)
     const int32_t *counts, *offsets;
-    int n_block;           // routes per block (multiple of 16, <= kNMax)
-    int b_slots;           // B ring slots of n_block * 128 bytes
+    int n_block;           // cap on the route block (multiple of 16, <= kNMax)
     int K;                 // reduction length: H (phase 1) or I (phase 2)
     int n_units;           // output rows of the weight: 2I (phase 1) or H (phase 2)
     int64_t rows_per_blob; // expert_bytes / row_bytes
@@ -198,20 +197,29 @@ __device__ __forceinline__ float gelu_tanh(float v) {
 // ------------------------------------------------------------- work items
 // Item = (active expert a, block of <= kNMax of its routes, M tile); M tiles
 // fastest so the CTAs working on one expert share its activation tiles in L2.
+// The route block n_block (rows of one B tile, columns of one accumulator) is
+// the busiest expert's route count rounded up to 16, capped by p.n_block: every
+// expert then fits one block, and a decode batch whose experts hold a handful of
+// routes gets small B slots, so many B stages are in flight.
 struct Items {
-    int n_act, total, m_tiles;
+    int n_act, total, m_tiles, n_block, b_slots;
 };
 
-__device__ void build_items(const TcParams &p, int m_tiles, int *s_act, int *s_base, Items *it) {
+__device__ void build_items(const TcParams &p, int m_tiles, int b_region, int *s_act, int *s_base, Items *it) {
     const int lane = threadIdx.x & 31;
     if (threadIdx.x < 32) {
+        int n_max = 1;
+        for (int e = lane; e < p.L.E; e += 32) n_max = max(n_max, __ldg(p.counts + e));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) n_max = max(n_max, __shfl_xor_sync(0xffffffffu, n_max, off));
+        const int n_block = min(p.n_block, (n_max + 15) & ~15);
         int n_act = 0, run = 0;
         for (int e0 = 0; e0 < p.L.E; e0 += 32) {
             const int e = e0 + lane;
             const int n = (e < p.L.E) ? __ldg(p.counts + e) : 0;
             const bool act = n > 0;
             const unsigned m = __ballot_sync(0xffffffffu, act);
-            const int items = act ? m_tiles * ((n + p.n_block - 1) / p.n_block) : 0;
+            const int items = act ? m_tiles * ((n + n_block - 1) / n_block) : 0;
             int inc = items;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -231,6 +239,8 @@ __device__ void build_items(const TcParams &p, int m_tiles, int *s_act, int *s_b
             it->n_act = n_act;
             it->total = run;
             it->m_tiles = m_tiles;
+            it->n_block = n_block;
+            it->b_slots = min(kMaxBSlots, b_region / (n_block * 128));
         }
     }
 }
@@ -240,7 +250,7 @@ struct ItemInfo {
 };
 
 __device__ __forceinline__ ItemInfo decode_item(const TcParams &p, const int *s_act, const int *s_base, int n_act,
-                                                int m_tiles, int item) {
+                                                int m_tiles, int n_block, int item) {
     int lo = 0, hi = n_act - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -251,10 +261,10 @@ __device__ __forceinline__ ItemInfo decode_item(const TcParams &p, const int *s_
     ItemInfo r;
     r.e = s_act[lo];
     const int n_e = __ldg(p.counts + r.e);
-    r.row0 = __ldg(p.offsets + r.e) + nb * p.n_block;
-    r.n = min(p.n_block, n_e - nb * p.n_block);
+    r.row0 = __ldg(p.offsets + r.e) + nb * n_block;
+    r.n = min(n_block, n_e - nb * n_block);
     r.n_mma = (r.n + 15) & ~15;
-    if (r.n <= 0 || r.n_mma > p.n_block || r.row0 < 0 || r.row0 + r.n > p.R) {
+    if (r.n <= 0 || r.n_mma > n_block || r.row0 < 0 || r.row0 + r.n > p.R) {
         record_error(0x2003u, (unsigned)item);
         r.n = 0;       // nothing is written for an item that fails the check,
         r.n_mma = 16;  // and its tiles stay inside their slots
@@ -321,7 +331,6 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = PHASE == 1 ? p.L.I / 64 : (p.L.H + kBlockM - 1) / kBlockM;
     const int nk = p.K / kBlockK;
-    const uint32_t b_slot_bytes = (uint32_t)p.n_block * 128;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SA; ++i) {
@@ -353,12 +362,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    build_items(p, m_tiles, s_act, s_base, &s_items);
+    build_items(p, m_tiles, TcFmt<FMT>::kBRegion, s_act, s_base, &s_items);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     const int n_act = s_items.n_act, total = s_items.total;
+    const int n_block = s_items.n_block, b_slots = s_items.b_slots;
+    const uint32_t b_slot_bytes = (uint32_t)n_block * 128;
 
     if (warp == 0) {
         // ------------------------------------- A producer: weights or raw codes
@@ -366,7 +377,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             int stage = 0;
             uint32_t phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
-                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 bool pool;
                 int ya0, ya1;  // row coordinates of the two 64-row halves of the tile
                 if (PHASE == 1) {
@@ -406,7 +417,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             int stage = 0;
             uint32_t phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
-                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 bool ok = true;
                 for (int kk = 0; kk < nk; ++kk) {
                     if (!mbar_wait(&b_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
@@ -414,7 +425,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     uint8_t *db = sB + stage * b_slot_bytes;
                     for (int j = 0; j < it.n_mma; j += 16)
                         tma_load_2d(db + j * 128, &map_b, &b_full[stage], kk * kBlockK, it.row0 + j);
-                    if (++stage == p.b_slots) { stage = 0; phase ^= 1; }
+                    if (++stage == b_slots) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
             }
@@ -427,7 +438,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             int acc = 0;
             uint32_t acc_phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
-                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, &s_abort)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * kNMax);
@@ -446,7 +457,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     tc_commit(&a_empty[sa]);
                     tc_commit(&b_empty[sb]);
                     if (++sa == SA) { sa = 0; pa ^= 1; }
-                    if (++sb == p.b_slots) { sb = 0; pb ^= 1; }
+                    if (++sb == b_slots) { sb = 0; pb ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit(&tfull[acc]);
@@ -462,7 +473,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         uint32_t xcount = 0;  // exchange chunks used so far (buffer = xcount & 1)
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok && !s_abort; item += gridDim.x) {
-            const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+            const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
             if (!mbar_wait(&tfull[acc], acc_phase, &s_abort)) break;
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kNMax);
@@ -543,7 +554,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         uint32_t phase = 0, rphase = 0;
         uint32_t step = 0;                              // k-steps seen, across items
         for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
-            const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, item);
+            const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
             const uint8_t *blob = expert_blob(p.L, it.e);
             const int wrow = PHASE == 1 ? (r < 64 ? it.m0 * 64 + r : p.L.I + it.m0 * 64 + r - 64)
                                         : min(it.m0 * kBlockM + r, p.n_units - 1);
@@ -780,12 +791,11 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     p.R = R;
     p.counts = counts;
     p.offsets = offsets;
-    // route block: an expert never gets a token twice, so min(T, 128) rows hold
-    // all of an expert's routes in one block (measured best: smaller blocks
-    // re-stream the weights of busier experts)
+    // cap on the route block: an expert never gets a token twice, so min(T, 128)
+    // rows hold all of an expert's routes in one block (smaller blocks would
+    // re-stream the weights of busier experts); the kernels shrink it to the
+    // busiest expert's count
     p.n_block = std::min(kNMax, (std::max(T, 1) + 15) / 16 * 16);
-    p.b_slots = std::min(kMaxBSlots, (fmt == MOE_W_BF16 ? TcFmt<MOE_W_BF16>::kBRegion : TcFmt<MOE_W_INT4>::kBRegion) /
-                                         (p.n_block * 128));
     p.h = h;
     p.rows = rows;
     // every pointer the kernels write through must be set (host-side guard)

@@ -69,6 +69,8 @@ def _L():
         c.oracle_permute.argtypes = [P, i32, i32, i32, P, P, P, P]
         c.oracle_route_min_weight.argtypes = [P, P, P, i32, i32, i32, ctypes.c_float]
         c.oracle_hits.argtypes = [P, i64, i32, P]
+        c.oracle_hits_window.argtypes = [P, i32, i32, P]
+        c.oracle_router_logits.argtypes = [P, P, i32, i32, i32, P]
         c.oracle_quantize_int8.argtypes = [P, i32, i32, P, P]
         c.oracle_quantize_int4.argtypes = [P, i32, i32, P, P]
         c.oracle_int4_candidates.argtypes = [P, P, P]
@@ -174,6 +176,27 @@ def hits(ids: np.ndarray, E: int, hits_in: np.ndarray | None = None) -> np.ndarr
     h = np.zeros(E, np.uint32) if hits_in is None else _c(hits_in, np.uint32).copy()
     _L().oracle_hits(_p(ids), ids.size, E, _p(h))
     return h
+
+
+def hits_window(ring: np.ndarray) -> np.ndarray:
+    """Window sum of per-step hit histograms ring[W, E] -> uint32[E]."""
+    ring = _c(ring, np.uint32)
+    W, E = ring.shape
+    out = np.zeros(E, np.uint32)
+    _L().oracle_hits_window(_p(ring), W, E, _p(out))
+    return out
+
+
+def router_logits(x_bits: np.ndarray, w_router: np.ndarray) -> np.ndarray:
+    """fp64 logits[T, E] of the router projection x[T, H] (bf16 bits) . w_router[E, H]^T (fp32)."""
+    x_bits = _c(x_bits, np.uint16)
+    w_router = _c(w_router, np.float32)
+    T, H = x_bits.shape
+    E = w_router.shape[0]
+    assert w_router.shape[1] == H
+    out = np.zeros((T, E), np.float64)
+    _L().oracle_router_logits(_p(x_bits), _p(w_router), T, H, E, _p(out))
+    return out
 
 
 def quantize_int8(w_bits: np.ndarray):

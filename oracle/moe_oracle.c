@@ -286,6 +286,28 @@ void oracle_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, 
     }
 }
 
+/*
+ * The step before the path: the router projection (prain README.md,
+ * "Experiments": the router is an fp32 GEMV over the hidden state).  Reading:
+ * a plain linear map with no bias, logits[t][e] = sum_h x[t][h] * w_router[e][h],
+ * x the layer's bf16 input row, w_router fp32 [E][H]; here every product and
+ * the sum over h (in h order) are taken in fp64.  Top-k routing then runs on
+ * the logits as oracle_route_topk states.
+ */
+void oracle_router_logits(const uint16_t *x, const float *w_router, int T, int H, int E, double *logits)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *xr = x + (size_t)t * H;
+        for (int e = 0; e < E; ++e) {
+            const float *wr = w_router + (size_t)e * H;
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h) acc += (double)bf16_value(xr[h]) * (double)wr[h];
+            logits[(size_t)t * E + e] = acc;
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ permute */
 /*
  * Group the R = T*k routes by expert (Winery-Strata remote_experts.cpp,
@@ -327,6 +349,21 @@ void oracle_hits(const int32_t *ids, long n, int E, uint32_t *hits)
 {
     for (long i = 0; i < n; ++i)
         if (ids[i] >= 0 && ids[i] < E) hits[ids[i]] += 1u;
+}
+
+/*
+ * Windowed hit counts, a variant of the refresh window (rlx_runtime
+ * expert_pool.rs counts only the refreshing step's routes): the hits of the
+ * last W steps, kept as W per-step histograms ring[W][E]; the window's count of
+ * expert e is the sum of its W entries.
+ */
+void oracle_hits_window(const uint32_t *ring, int W, int E, uint32_t *sum)
+{
+    for (int e = 0; e < E; ++e) {
+        uint32_t acc = 0;
+        for (int s = 0; s < W; ++s) acc += ring[(size_t)s * E + e];
+        sum[e] = acc;
+    }
 }
 
 /* --------------------------------------------------------------- quantisers */

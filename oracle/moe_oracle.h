@@ -65,12 +65,17 @@ void oracle_route_topk(const float *logits, int T, int E, int k, int32_t *ids, f
 void oracle_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, int T, int k, int E,
                              float min_weight);
 
+/* the step before the path: logits[t][e] = sum_h x[t][h] * w_router[e][h] in fp64 (x bf16 bits) */
+void oracle_router_logits(const uint16_t *x, const float *w_router, int T, int H, int E, double *logits);
+
 /* stable counting sort of the T*k routes by expert id */
 void oracle_permute(const int32_t *ids, int T, int k, int E, int32_t *counts, int32_t *offsets,
                     int32_t *sorted_route, int32_t *route_pos);
 
 /* hits[e] += number of ids equal to e; ids outside [0,E) are ignored */
 void oracle_hits(const int32_t *ids, long n, int E, uint32_t *hits);
+/* sum[e] = sum over the W rows of ring[W][E] (hits of the last W steps) */
+void oracle_hits_window(const uint32_t *ring, int W, int E, uint32_t *sum);
 
 /* quantisers: w bf16 bits [rows,K] */
 void oracle_quantize_int8(const uint16_t *w, int rows, int K, int8_t *q, float *scale);

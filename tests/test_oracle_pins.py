@@ -591,3 +591,68 @@ def test_min_weight_hand_example():
     assert i2.tolist() == [[3, 0, -1, 1]]
     np.testing.assert_array_equal(w2, np.float32([[0.5 * np.float32(1 / 0.875), 0.25 * np.float32(1 / 0.875), 0,
                                                    0.125 * np.float32(1 / 0.875)]]))
+
+
+# ------------------------------------------------------ router projection (f3)
+
+def _bf16_bits(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_router_logits_equal_a_library_matmul():
+    """The projection is a plain matrix product: numpy's fp64 matmul of the same
+    bf16 x and fp32 router weights agrees to fp64 rounding of the sums."""
+    rng = np.random.default_rng(3)
+    T, Hh, E = 9, 2816, 128
+    x = syn.activations(T, Hh, seed=4)
+    wr = (rng.standard_normal((E, Hh)) * 0.02).astype(np.float32)
+    got = oracle.router_logits(x, wr)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float().numpy().astype(np.float64)
+    want = xf @ wr.astype(np.float64).T
+    scale = np.abs(xf) @ np.abs(wr.astype(np.float64)).T
+    assert np.all(np.abs(got - want) <= 1e-12 * scale)
+
+
+def test_router_logits_one_hot_rows_pick_weight_columns():
+    """x = c * e_h (c a power of two) gives logits = c * w_router[:, h] exactly;
+    a transposed operand or a wrong row index fails this."""
+    rng = np.random.default_rng(5)
+    Hh, E = 96, 24
+    wr = rng.standard_normal((E, Hh)).astype(np.float32)
+    xs = np.zeros((Hh, Hh), np.float32)
+    for h in range(Hh):
+        xs[h, h] = 2.0 ** (h % 5 - 2)
+    got = oracle.router_logits(_bf16_bits(xs), wr)
+    for h in range(Hh):
+        assert np.array_equal(got[h], (2.0 ** (h % 5 - 2)) * wr[:, h].astype(np.float64))
+
+
+def test_router_then_topk_with_identity_weights_is_topk_of_x():
+    """With w_router = [I_E | 0] the logits are x's first E values, so routing
+    them reduces to top-k of those values (exact: each logit is one product)."""
+    T, Hh, E, k = 7, 64, 16, 4
+    x = syn.activations(T, Hh, seed=8)
+    wr = np.zeros((E, Hh), np.float32)
+    wr[:, :E] = np.eye(E, dtype=np.float32)
+    lg = oracle.router_logits(x, wr)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert np.array_equal(lg, xf[:, :E].astype(np.float64))
+    ids, _ = oracle.route_topk(lg.astype(np.float32), k)
+    want = np.argsort(-xf[:, :E], axis=1, kind="stable")[:, :k]
+    assert np.array_equal(ids, want)
+
+
+# ------------------------------------------------- windowed hit counts (f3)
+
+def test_hits_window_equals_bincount_over_the_window():
+    """The sum of W per-step histograms is the bincount of all W steps' ids
+    (numpy's bincount over the concatenation)."""
+    rng = np.random.default_rng(11)
+    E, W = 128, 8
+    steps = [rng.integers(0, E, size=(rng.integers(1, 200),), dtype=np.int32) for _ in range(W)]
+    ring = np.stack([oracle.hits(s, E) for s in steps])
+    got = oracle.hits_window(ring)
+    want = np.bincount(np.concatenate(steps), minlength=E).astype(np.uint32)
+    assert np.array_equal(got, want)
+    assert np.array_equal(oracle.hits_window(ring[:1]), ring[0])
+    assert not oracle.hits_window(np.zeros((W, E), np.uint32)).any()

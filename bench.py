@@ -340,6 +340,41 @@ def time_e2e(torch, moe, layers, batches, T, k, steps, warmup, dev):
     return ms, T * E * 4 + T * H * 2, T * H * 2
 
 
+def time_router(torch, moe, T, E, H, k, dev, n=200):
+    """The router projection fused with top-k (the step before the layer), one
+    launch per call on a different copy of the fp32 router weights (enough copies
+    to span twice the L2), n calls replayed from one CUDA graph."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(8, -(-2 * l2 // (E * H * 4)))
+    g = torch.Generator(device=dev)
+    g.manual_seed(17)
+    wr = torch.randn((copies, E, H), generator=g, device=dev, dtype=torch.float32) * 0.02
+    x = (torch.randn((T, H), generator=g, device=dev, dtype=torch.float32)).to(torch.bfloat16)
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        moe.moe_router_topk(x, wr[0], k, ids=ids, w=w)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(n):
+                moe.moe_router_topk(x, wr[i % copies], k, ids=ids, w=w)
+        graph.replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        stream.synchronize()
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        b.synchronize()
+    us = a.elapsed_time(b) * 1e3 / n
+    alg = E * H * 4 + T * H * 2 + T * k * 8
+    del graph, wr
+    return {"us": round(us, 2), "tokens_per_s": round(T / (us / 1e6), 1), "alg_bytes": alg,
+            "hbm_gbs": round(alg / (us / 1e6) / 1e9, 1), "router_copies": copies}
+
+
 def cpu_baseline(moe, torch, cfg_fmt, layers, batches, T, k, seconds, first_token_only=False):
     """The oracle (as it stands) on a bounded sample: whole tokens of batch 0 of
     layer 0, one at a time, until `seconds` have passed."""
@@ -457,6 +492,13 @@ def main():
             "ffn_frac_of_hbm": round((dd * eb + Ts * H * 2) / (f2 / 1e3) / 1e9 / hbm_peak, 4),
         }
 
+    router = {}
+    if args.config != "tiny":
+        for Tr in ([T] if args.quick else sorted({1, T, 1024})):
+            r = time_router(torch, moe, Tr, E, H, k, dev)
+            r["frac_of_hbm"] = round(r["hbm_gbs"] / hbm_peak, 4)
+            router[f"T{Tr}"] = r
+
     e2e_ms, h2d, d2h = (float("nan"), 0, 0) if args.quick else time_e2e(torch, moe, layers, batches, T, k,
                                                                          args.steps, args.warmup, dev)
     e2e_ms = max_over_ranks(dist, e2e_ms, dev)
@@ -513,6 +555,7 @@ def main():
             "avg_launch_us": round(ffn_avg_ms * 1e3, 2),
         }),
         "sweep": sweep_out,
+        "router_topk": router,
         "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": runner.launches_per_step() * args.steps,

@@ -124,6 +124,24 @@ MOE_API moe_status moe_route_topk(const float *logits, int32_t T, int32_t E, int
                           moe_stream_t stream);
 
 /*
+ * The step before the path, fused with it: the fp32 router projection (prain
+ * README.md, "Experiments": the router is an fp32 GEMV) followed by
+ * moe_route_topk's recipe, in one launch.
+ *   logits[t][e] = sum_h x[t][h] * w_router[e][h]   (fp32 fused multiply-adds)
+ * x bf16 [T][H] row-major (8-byte aligned, H a multiple of 4); w_router fp32
+ * [E][H] row-major (16-byte aligned); logits fp32 [T][E] (output, nullable: pass
+ * it to see the values the routing decided on); ids int32 [T][k] and w fp32
+ * [T][k] exactly as moe_route_topk produces from those logits.  The logits are
+ * fp32 sums (lane-strided partial sums over h, then a butterfly), so they match
+ * an exact projection to rounding; ids and w are bit-exact functions of them.
+ * One cluster of 8 CTAs per group of up to 16 tokens; each CTA stages its
+ * group's rows in shared memory (MOE_ERR_UNSUPPORTED when even one row, 2*H
+ * bytes plus the logits, exceeds 200 KiB).
+ */
+MOE_API moe_status moe_router_topk(const uint16_t *x, const float *w_router, int32_t T, int32_t H, int32_t E,
+                                   int32_t k, float *logits, int32_t *ids, float *w, moe_stream_t stream);
+
+/*
  * [miss] min_weight partial routing (prain README.md, "Trading quality for
  * speed"), applied in place to the output of moe_route_topk.  Per token, routes
  * are taken heaviest first with a running sum `kept` of the weights kept so far
@@ -283,6 +301,14 @@ MOE_API moe_status moe_refresh_target(const uint32_t *hits, int32_t E, int32_t b
 MOE_API moe_status moe_apply_placement(int32_t *slot_of, int32_t E, int32_t n_slots, const int32_t *target,
                                int32_t n_target, int32_t *promote, int32_t *demote, int32_t *n_promote,
                                int32_t *n_demote);
+
+/*
+ * Windowed hit counts (host, pure CPU): sum[e] = sum over s < W of
+ * ring[s][e], the hits of the last W steps kept as one histogram per step (a
+ * variant of expert_pool.rs, which counts only the refreshing step's routes).
+ * ring uint32 [W][E] and sum uint32 [E] are host memory.
+ */
+MOE_API moe_status moe_hits_window(const uint32_t *ring, int32_t W, int32_t E, uint32_t *sum);
 
 /* should_refresh: 0 without offload; 1 in refresh mode or on a prefill block;
  * else 1 when step is a multiple of interval (interval < 1 counts as 1). */

@@ -36,7 +36,7 @@ EXPORTS = [
     "moe_layer_forward_workspace", "moe_layer_forward", "moe_quantize_int8", "moe_quantize_int4",
     "moe_pack_expert", "moe_copy_to_slots", "moe_refresh_target", "moe_apply_placement",
     "moe_should_refresh", "moe_budget_from_vram", "moe_grouped_ffn_noalloc", "moe_take_device_errors",
-    "moe_route_min_weight",
+    "moe_route_min_weight", "moe_router_topk", "moe_hits_window",
 ]
 
 
@@ -81,6 +81,8 @@ _SIG = {
     "moe_grouped_ffn_noalloc": (i32, [LP, P, i32, i32, P, P, P, P, P]),
     "moe_take_device_errors": (i32, [P, P]),
     "moe_route_min_weight": (i32, [P, P, P, i32, i32, i32, ctypes.c_float, P]),
+    "moe_router_topk": (i32, [P, P, i32, i32, i32, i32, P, P, P, P]),
+    "moe_hits_window": (i32, [P, i32, i32, P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -174,6 +176,27 @@ def moe_route_topk(logits: torch.Tensor, k: int, ids: torch.Tensor | None = None
     _check(_lib.moe_route_topk(_dev(logits, torch.float32, "logits"), T, E, k, _dev(ids, torch.int32, "ids"),
                                _dev(w, torch.float32, "w"), _stream(stream)))
     return ids, w
+
+
+def moe_router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int, logits: torch.Tensor | bool | None = None,
+                    ids: torch.Tensor | None = None, w: torch.Tensor | None = None, stream=None):
+    """Router projection x[T,H] (bf16) . w_router[E,H]^T (fp32) fused with top-k.
+    Returns (ids, w) or, with logits=True or a [T,E] fp32 tensor, (ids, w, logits)."""
+    T, H = x.shape
+    E = w_router.shape[0]
+    if w_router.shape[1] != H:
+        raise ValueError("w_router must be [E, H]")
+    want_logits = logits is not None and logits is not False
+    if logits is True:
+        logits = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    elif logits is False:
+        logits = None
+    ids = torch.empty((T, k), dtype=torch.int32, device=x.device) if ids is None else ids
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device) if w is None else w
+    _check(_lib.moe_router_topk(_dev(x, BF16, "x"), _dev(w_router, torch.float32, "w_router"), T, H, E, k,
+                                _dev(logits, torch.float32, "logits"), _dev(ids, torch.int32, "ids"),
+                                _dev(w, torch.float32, "w"), _stream(stream)))
+    return (ids, w, logits) if want_logits else (ids, w)
 
 
 def moe_route_min_weight(ids: torch.Tensor, w: torch.Tensor, E: int, min_weight: float,
@@ -322,6 +345,15 @@ def moe_apply_placement(slot_of: np.ndarray, n_slots: int, target: np.ndarray):
                                     pr.ctypes.data_as(ctypes.c_void_p), de.ctypes.data_as(ctypes.c_void_p),
                                     ctypes.byref(npr), ctypes.byref(nde)))
     return so, pr[: npr.value].copy(), de[: nde.value].copy()
+
+
+def moe_hits_window(ring: np.ndarray) -> np.ndarray:
+    """Host: window sum of per-step hit histograms ring[W, E] -> uint32[E]."""
+    r, pr = _host(ring, np.uint32)
+    W, E = r.shape
+    out = np.zeros(E, np.uint32)
+    _check(_lib.moe_hits_window(pr, W, E, out.ctypes.data_as(ctypes.c_void_p)))
+    return out
 
 
 def moe_should_refresh(offload_enabled: bool, mode_refresh: bool, step: int, is_prefill_block: bool,

@@ -9,6 +9,11 @@
 namespace moe {
 
 cudaError_t launch_route_topk(const float *, int, int, int, int32_t *, float *, cudaStream_t);
+cudaError_t launch_router_topk(const uint16_t *, const float *, int, int, int, int, float *, int32_t *, float *,
+                               cudaStream_t);
+int router_tok(int T, int H, int E);
+size_t router_smem(int tok, int H, int E);
+extern const size_t kRouterMaxSmemBytes;
 cudaError_t launch_route_min_weight(int32_t *, float *, const int32_t *, int, int, int, float, cudaStream_t);
 cudaError_t launch_permute(const int32_t *, int, int, int32_t *, int32_t *, int32_t *, int32_t *, uint32_t *,
                            cudaStream_t);
@@ -122,6 +127,26 @@ moe_status moe_route_topk(const float *logits, int32_t T, int32_t E, int32_t k, 
     if (T == 0) return MOE_OK;
     CHECK_ARG(logits && ids && w, "moe_route_topk: NULL pointer");
     return cuda_status(launch_route_topk(logits, T, E, k, ids, w, (cudaStream_t)stream), "moe_route_topk launch");
+}
+
+moe_status moe_router_topk(const uint16_t *x, const float *w_router, int32_t T, int32_t H, int32_t E, int32_t k,
+                           float *logits, int32_t *ids, float *w, moe_stream_t stream) {
+    moe_status st = check_shape(E, k, 64, 64);
+    if (st != MOE_OK) return st;
+    if ((st = check_tk(T, k)) != MOE_OK) return st;
+    CHECK_ARG(H >= 4 && H % 4 == 0, "H=%d must be a positive multiple of 4", H);
+    CHECK_ARG(T <= 0 || (T + router_tok(T, H, E) - 1) / router_tok(T, H, E) <= 65535,
+              "T=%d: more than 65535 token groups", T);
+    CHECK_ARG((int64_t)T * E <= INT32_MAX, "T*E=%lld does not fit int32", (long long)T * E);
+    if (T == 0) return MOE_OK;
+    CHECK_ARG(x && w_router && ids && w, "moe_router_topk: NULL pointer");
+    CHECK_ARG(((uintptr_t)x & 7u) == 0 && aligned16(w_router), "x must be 8-byte and w_router 16-byte aligned");
+    const size_t smem = router_smem(router_tok(T, H, E), H, E);
+    if (smem > kRouterMaxSmemBytes)
+        return set_error(MOE_ERR_UNSUPPORTED, "moe_router_topk: H=%d needs %zu bytes of shared memory per CTA (max %zu)",
+                         H, smem, kRouterMaxSmemBytes);
+    return cuda_status(launch_router_topk(x, w_router, T, H, E, k, logits, ids, w, (cudaStream_t)stream),
+                       "moe_router_topk launch");
 }
 
 moe_status moe_route_min_weight(int32_t *ids, float *w, const int32_t *slot_table, int32_t T, int32_t k, int32_t E,

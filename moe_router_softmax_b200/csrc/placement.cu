@@ -70,6 +70,17 @@ moe_status moe_apply_placement(int32_t *slot_of, int32_t E, int32_t n_slots, con
     return MOE_OK;
 }
 
+moe_status moe_hits_window(const uint32_t *ring, int32_t W, int32_t E, uint32_t *sum) {
+    if (!ring || !sum) return set_error(MOE_ERR_INVALID_ARG, "moe_hits_window: NULL pointer");
+    if (E < 1 || E > kMaxE || W < 1) return set_error(MOE_ERR_INVALID_ARG, "moe_hits_window: E=%d W=%d", E, W);
+    for (int32_t e = 0; e < E; ++e) {
+        uint32_t acc = 0;
+        for (int32_t s = 0; s < W; ++s) acc += ring[(size_t)s * E + e];
+        sum[e] = acc;
+    }
+    return MOE_OK;
+}
+
 int32_t moe_should_refresh(int32_t offload_enabled, int32_t mode_refresh, int64_t step, int32_t is_prefill_block,
                            int64_t interval) {
     if (!offload_enabled) return 0;

@@ -6,9 +6,29 @@
 // the kept logits (the full denominator cancels).  All fp32 steps are written
 // with explicit round-to-nearest intrinsics so that no multiply-add is fused
 // behind our back: the result is bit-for-bit the recipe of moe_route_topk.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace moe {
+
+// dynamic shared memory of one router CTA: TOK x EB fp32 logits and TOK x H
+// bf16 activation rows; TOK = tokens per cluster: the batch itself up to 4,
+// 8 for decode batches, 16 past 64 tokens (fewer re-reads of the router
+// weights), halved while the rows do not fit
+constexpr size_t kRouterMaxSmem = 200 * 1024;
+extern const size_t kRouterMaxSmemBytes = kRouterMaxSmem;
+size_t router_smem(int tok, int H, int E) {
+    return (((size_t)tok * ((E + 7) / 8) * 4 + 15) & ~(size_t)15) + (size_t)tok * H * 2;
+}
+int router_tok(int T, int H, int E) {
+    int tok = T <= 1 ? 1 : (T == 2 ? 2 : (T <= 4 ? 4 : (T <= 64 ? 8 : 16)));
+    while (tok > 1 && router_smem(tok, H, E) > kRouterMaxSmem) tok >>= 1;
+    return tok;
+}
+
 namespace {
 
 // exp_p -- the library's fp32 exponential, from the mathematics:
@@ -52,13 +72,12 @@ __device__ __forceinline__ bool ranks_before(float va, int ea, float vb, int eb)
     return ea < eb;
 }
 
-template <int VPL>
-__global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ logits, int T, int E, int k,
-                                                    int32_t *__restrict__ ids, float *__restrict__ w) {
+// Top-k and weights of one token, by one warp.  load(e) returns logit e for
+// e < E; lane l holds experts l, l+32, ...; the k winners are taken one at a
+// time by a warp arg-best, then the softmax over them (max logit first).
+template <int VPL, class Load>
+__device__ __forceinline__ void route_token_warp(Load load, int E, int k, int32_t *ids_row, float *w_row) {
     const int lane = threadIdx.x & 31;
-    const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-    if (t >= T) return;
-    const float *l = logits + (size_t)t * E;
     float v[VPL];
     uint32_t avail = 0;
 #pragma unroll
@@ -66,7 +85,7 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
         int e = lane + 32 * i;
         v[i] = 0.0f;
         if (e < E) {
-            v[i] = __ldg(l + e);
+            v[i] = load(e);
             avail |= 1u << i;
         }
     }
@@ -111,9 +130,186 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
     float S = 0.0f;
     for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, ej, j));
     if (lane < k) {
-        ids[(size_t)t * k + lane] = my_e;
-        w[(size_t)t * k + lane] = __fdiv_rn(ej, S);
+        ids_row[lane] = my_e;
+        w_row[lane] = __fdiv_rn(ej, S);
     }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ logits, int T, int E, int k,
+                                                    int32_t *__restrict__ ids, float *__restrict__ w) {
+    const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    if (t >= T) return;
+    const float *l = logits + (size_t)t * E;
+    route_token_warp<VPL>([l](int e) { return __ldg(l + e); }, E, k, ids + (size_t)t * k, w + (size_t)t * k);
+}
+
+// ------------------------------------------------ router projection + top-k
+// The step before the routing: logits[t][e] = sum_h x[t][h] * w_router[e][h]
+// (x bf16, router weights fp32, fp32 fused multiply-adds), then the top-k
+// recipe above on those logits, in one launch.
+//
+// A cluster of kRouterCluster CTAs takes TOK tokens; CTA r of the cluster
+// projects experts [r*EB, (r+1)*EB) (EB = ceil(E / kRouterCluster)) for all TOK
+// tokens into its shared memory, so the router weights are read once per
+// cluster and every SM of the cluster streams a different slice of them (the
+// group's activation rows are staged in its shared memory).  After
+// a cluster barrier, CTA r routes token r of the group: its warp 0 reads the E
+// logits from the eight CTAs' shared memory (distributed shared memory) and
+// runs route_token_warp.  A second cluster barrier keeps every slice alive
+// until all reads are done.
+//
+// Summation order of one logit: lane l of the warp owning expert e sums the
+// products of h = 4l .. 4l+3 (mod 128) in increasing h, then the 32 lane sums
+// are added by a butterfly (xor 16, 8, 4, 2, 1).
+constexpr int kRouterCluster = 8;
+constexpr int kRouterThreads = 256;
+constexpr int kRouterWarps = kRouterThreads / 32;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+template <int TOK, int VPL>
+__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouterThreads)
+    k_router_topk(const uint16_t *__restrict__ x, const float *__restrict__ wr, int T, int H, int E, int k,
+                  float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ w) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int EB = (E + kRouterCluster - 1) / kRouterCluster;
+    const int t0 = blockIdx.y * TOK;
+    const int nt = min(TOK, T - t0);
+    float *s_logit = reinterpret_cast<float *>(smem);                                  // [TOK][EB]
+    uint16_t *s_x = reinterpret_cast<uint16_t *>(smem + ((TOK * EB * 4 + 15) & ~15));  // [TOK][H]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // this CTA's slice of the router weights (rows e_lo .. e_hi-1, contiguous)
+    // is requested into L2 first, so its DRAM latency overlaps the staging below
+    const int e_lo = rank * EB, e_hi = min(E, e_lo + EB);
+    if (e_hi > e_lo) {
+        const char *slice = reinterpret_cast<const char *>(wr + (size_t)e_lo * H);
+        const size_t bytes = (size_t)(e_hi - e_lo) * H * 4;
+        for (size_t off = (size_t)threadIdx.x * 128; off < bytes; off += (size_t)kRouterThreads * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(slice + off));
+    }
+
+    // the group's activation rows (zero past the last token)
+    const int h4 = H / 4;
+    for (int i = threadIdx.x; i < TOK * h4; i += kRouterThreads) {
+        const int t = i / h4, c = i - t * h4;
+        uint2 v = make_uint2(0u, 0u);
+        if (t < nt) v = __ldg(reinterpret_cast<const uint2 *>(x + (size_t)(t0 + t) * H) + c);
+        reinterpret_cast<uint2 *>(s_x + (size_t)t * H)[c] = v;
+    }
+    __syncthreads();
+
+    // projection: warp w takes experts e_lo + 2w, +1, then + 2*kRouterWarps, ...
+    // U chunks of 128 h per lane are loaded before they are used, so U loads of
+    // each operand are in flight (the sums still run in increasing h)
+    constexpr int U = TOK <= 8 ? 8 : 4;
+    for (int e0 = e_lo + 2 * warp; e0 < e_hi; e0 += 2 * kRouterWarps) {
+        const bool two = e0 + 1 < e_hi;
+        const float *w0 = wr + (size_t)e0 * H;
+        const float *w1 = wr + (size_t)(two ? e0 + 1 : e0) * H;
+        float a0[TOK], a1[TOK];
+#pragma unroll
+        for (int t = 0; t < TOK; ++t) a0[t] = a1[t] = 0.0f;
+        for (int hb = lane * 4; hb < H; hb += 128 * U) {
+            float4 p[U], q[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int h = hb + 128 * u;
+                p[u] = q[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (h < H) {
+                    p[u] = __ldg(reinterpret_cast<const float4 *>(w0 + h));
+                    q[u] = __ldg(reinterpret_cast<const float4 *>(w1 + h));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int h = hb + 128 * u;
+                if (h < H) {
+#pragma unroll
+                    for (int t = 0; t < TOK; ++t) {
+                        const uint2 xv = *reinterpret_cast<const uint2 *>(s_x + (size_t)t * H + h);
+                        const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+                        const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
+                        a0[t] = __fmaf_rn(x0, p[u].x, a0[t]);
+                        a0[t] = __fmaf_rn(x1, p[u].y, a0[t]);
+                        a0[t] = __fmaf_rn(x2, p[u].z, a0[t]);
+                        a0[t] = __fmaf_rn(x3, p[u].w, a0[t]);
+                        a1[t] = __fmaf_rn(x0, q[u].x, a1[t]);
+                        a1[t] = __fmaf_rn(x1, q[u].y, a1[t]);
+                        a1[t] = __fmaf_rn(x2, q[u].z, a1[t]);
+                        a1[t] = __fmaf_rn(x3, q[u].w, a1[t]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < TOK; ++t) {
+            a0[t] = warp_sum(a0[t]);
+            a1[t] = warp_sum(a1[t]);
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int t = 0; t < TOK; ++t) {
+                s_logit[t * EB + (e0 - e_lo)] = a0[t];
+                if (two) s_logit[t * EB + (e0 + 1 - e_lo)] = a1[t];
+                if (logits != nullptr && t < nt) {
+                    logits[(size_t)(t0 + t) * E + e0] = a0[t];
+                    if (two) logits[(size_t)(t0 + t) * E + e0 + 1] = a1[t];
+                }
+            }
+        }
+    }
+
+    cluster.sync();
+    // CTA r routes tokens r, r + 8, ... of the group, one warp each
+    const int t = rank + kRouterCluster * warp;
+    if (warp < (TOK + kRouterCluster - 1) / kRouterCluster && t < nt) {
+        route_token_warp<VPL>(
+            [&](int e) {
+                const float *slice = cluster.map_shared_rank(s_logit, e / EB);
+                return slice[t * EB + e % EB];
+            },
+            E, k, ids + (size_t)(t0 + t) * k, w + (size_t)(t0 + t) * k);
+    }
+    cluster.sync();
+}
+
+template <int TOK, int VPL>
+cudaError_t launch_router(const uint16_t *x, const float *wr, int T, int H, int E, int k, float *logits,
+                          int32_t *ids, float *w, cudaStream_t s) {
+    auto kern = k_router_topk<TOK, VPL>;
+    static bool attr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!attr[dev]) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRouterMaxSmem);
+        if (err != cudaSuccess) return err;
+        attr[dev] = true;
+    }
+    dim3 grid(kRouterCluster, (unsigned)((T + TOK - 1) / TOK));
+    kern<<<grid, kRouterThreads, router_smem(TOK, H, E), s>>>(x, wr, T, H, E, k, logits, ids, w);
+    return cudaGetLastError();
+}
+
+template <int VPL>
+cudaError_t launch_router_vpl(const uint16_t *x, const float *wr, int T, int H, int E, int k, float *logits,
+                              int32_t *ids, float *w, cudaStream_t s) {
+    const int tok = router_tok(T, H, E);
+    if (router_smem(tok, H, E) > kRouterMaxSmem) return cudaErrorInvalidValue;
+    if (tok == 16) return launch_router<16, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
+    if (tok == 1) return launch_router<1, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
+    if (tok == 2) return launch_router<2, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
+    if (tok == 4) return launch_router<4, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
+    return launch_router<8, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
 }
 
 // [miss] min_weight partial routing, one thread per token: heaviest route
@@ -153,6 +349,13 @@ cudaError_t launch_route_min_weight(int32_t *ids, float *w, const int32_t *slot_
     if (T == 0 || !(min_weight < 1.0f)) return cudaSuccess;
     k_route_min_weight<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(ids, w, slot_table, T, k, E, min_weight);
     return cudaGetLastError();
+}
+
+cudaError_t launch_router_topk(const uint16_t *x, const float *w_router, int T, int H, int E, int k, float *logits,
+                               int32_t *ids, float *w, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    if (E <= 128) return launch_router_vpl<4>(x, w_router, T, H, E, k, logits, ids, w, s);
+    return launch_router_vpl<32>(x, w_router, T, H, E, k, logits, ids, w, s);
 }
 
 cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w,

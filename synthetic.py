@@ -10,6 +10,8 @@ experts, hidden 2816, expert intermediate 704, top-8); the weights, routing
 traces and prompts of that model are not available, so these draws stand in:
 
 * expert weights ~ N(0, 0.02), activations ~ N(0, 1), both rounded to bf16 (RNE);
+* router weights (the fp32 projection before the routing) ~ N(0, 0.02) in fp32,
+  so that at hidden 2816 the projected logits are close to N(0, 1);
 * router logits ~ N(0, 1) fp32 (uniform expert popularity);
 * "biased": N(0, 1) plus a per-expert bias drawn once per layer from N(0, 1.5)
   (standard deviation 1.5), to skew popularity;
@@ -28,7 +30,7 @@ from __future__ import annotations
 import numpy as np
 
 # stream ids, so that each tensor has its own sub-seed
-S_W13, S_W2, S_X, S_LOGITS, S_BIAS, S_PERM, S_GUMBEL = 1, 2, 3, 4, 5, 6, 7
+S_W13, S_W2, S_X, S_LOGITS, S_BIAS, S_PERM, S_GUMBEL, S_ROUTER = 1, 2, 3, 4, 5, 6, 7, 8
 
 WEIGHT_STD = 0.02
 
@@ -66,6 +68,11 @@ def expert_weights(E: int, H: int, I: int, seed: int = 0, layer: int = 0):
     w13 = normal_bf16((E, 2 * I, H), WEIGHT_STD, seed, S_W13, layer)
     w2 = normal_bf16((E, H, I), WEIGHT_STD, seed, S_W2, layer)
     return w13, w2
+
+
+def router_weights(E: int, H: int, seed: int = 0, layer: int = 0) -> np.ndarray:
+    """Router projection weights [E, H] fp32, N(0, 0.02)."""
+    return _rng(seed, S_ROUTER, layer).standard_normal((E, H), dtype=np.float32) * np.float32(WEIGHT_STD)
 
 
 def router_logits(T: int, E: int, kind: str = "normal", seed: int = 0, layer: int = 0,

@@ -143,3 +143,32 @@ def test_placement_rejects_bad_input():
     so[[0, 1]] = 0
     with pytest.raises(moe.MoeError):
         moe.moe_apply_placement(so, 4, np.array([2]))  # slot held twice
+
+
+def test_router_topk_rejects_bad_arguments_before_launch():
+    L = moe._lib
+    ok = dict(x=256, wr=256, T=4, H=2816, E=128, k=8, lg=None, ids=256, w=256)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return L.moe_router_topk(a["x"], a["wr"], a["T"], a["H"], a["E"], a["k"], a["lg"], a["ids"], a["w"], None)
+
+    assert call(k=129) == moe.MOE_ERR_INVALID_ARG           # k > E
+    assert call(E=0) == moe.MOE_ERR_INVALID_ARG
+    assert call(H=2818) == moe.MOE_ERR_INVALID_ARG          # H % 4
+    assert call(x=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(wr=264) == moe.MOE_ERR_INVALID_ARG          # router weights not 16-byte aligned
+    assert call(x=260) == moe.MOE_ERR_INVALID_ARG           # x not 8-byte aligned
+    assert call(T=-1) == moe.MOE_ERR_INVALID_ARG
+    assert call(T=70000 * 16) == moe.MOE_ERR_INVALID_ARG    # more than 65535 token groups
+    st = call(T=1, H=120000)                                 # one row of 120000 bf16 exceeds 200 KiB
+    assert st == moe.MOE_ERR_UNSUPPORTED and "shared memory" in moe.moe_last_error()
+    assert call(T=0) == moe.MOE_OK                           # nothing to do
+
+
+def test_hits_window_matches_oracle():
+    rng = np.random.default_rng(2)
+    ring = rng.integers(0, 50, size=(8, 128), dtype=np.uint32)
+    assert np.array_equal(moe.moe_hits_window(ring), oracle.hits_window(ring))
+    with pytest.raises(moe.MoeError):
+        moe.moe_hits_window(np.zeros((0, 128), np.uint32))

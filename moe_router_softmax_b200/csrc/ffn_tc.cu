@@ -9,11 +9,14 @@
 //   phase 2:  D[128 x N] = W2[m0..m0+127] . h^T,   epilogue rows[s][m] = D[m]
 // Xs is x gathered into sorted-route order (k_gather_rows), so every B tile is
 // a plain 2-D TMA box.  For bf16 weights TMA writes the A tile straight into
-// the 128-byte-swizzled K-major layout the MMA reads; int8/int4 tiles land raw
-// and eight dequant warps expand them into that layout (int8 codes exactly,
-// with the per-row scale applied in the epilogue; int4 as bf16(q * s) with
-// the group scale, one rounding), so dequantisation is fused into the
-// shared-memory stage.
+// the 128-byte-swizzled K-major layout the MMA reads from shared memory.
+// int8/int4 codes land raw (128-byte swizzled, so the dequant warps read them
+// without bank conflicts) and eight dequant warps expand each stage into bf16
+// (int8 codes exactly, with the per-row scale applied in the epilogue; int4 as
+// bf16(q * s) with the group scale, one rounding) and store it in tensor
+// memory, where the MMA takes its A operand: the expanded weights never touch
+// shared memory, whose bandwidth the MMAs' operand reads would otherwise share
+// with the expansion.
 //
 // One persistent CTA per SM; warp roles:
 //   warp 0      TMA producer of A: the weight tiles (bf16) or the raw codes
@@ -47,7 +50,7 @@ constexpr int kBlockM = 128;          // weight rows per tile (TMEM lanes)
 constexpr int kBlockK = 64;           // bf16 elements per MMA stage = one 128-byte swizzle row
 constexpr int kNMax = 128;            // max routes per block (TMEM columns per accumulator)
 constexpr int kAccBufs = 2;
-constexpr int kTmemCols = kNMax * kAccBufs;
+constexpr int kAccCols = kNMax * kAccBufs;   // TMEM columns of the accumulators
 constexpr int kEpiWarps = 4;
 constexpr int kDeqWarps = 8;          // per group: two threads per tile row, half a row each
 constexpr int kDeqGroups = 2;         // groups take alternate stages, so two stages expand at once
@@ -59,21 +62,33 @@ constexpr int kXPitch = 17;                               // exchange row pitch 
 
 // Three rings of shared-memory stages, each with its own full / empty
 // mbarriers, so no operand's load latency holds another's slots:
-//  A:   kAStages weight tiles of 128 rows x 64 bf16 (TMA for bf16 weights, the
-//       dequant warps for int8/int4);
+//  A:   kAStages weight tiles of 128 rows x 64 bf16 (bf16 weights: TMA into
+//       shared memory; int8/int4: the dequant warps, into tensor memory);
 //  B:   up to kMaxBSlots activation tiles of n_block rows x 64 bf16 (TMA), as
 //       many as fit in kBRegion bytes for this launch's block size;
 //  raw: kRawStages stages of 128 code bytes per row (int formats: 256 int4 or
 //       128 int8 weights, kSub MMA stages each), whole 128-byte runs of a row.
+// For int8 / int4 the A ring lives in tensor memory instead (kASmem = 0): the
+// dequant warps store the bf16 tiles with tcgen05.st and the MMAs read A from
+// TMEM, so the expanded weights never pass through shared memory.
+// A stage covers kKS of K (kKS / 64 swizzle atoms): one 64-wide atom for bf16;
+// two for the int formats, so that the single MMA-issuing thread pays one
+// barrier wait and one pair of commits per 8 MMAs instead of per 4 (each
+// tcgen05 instruction and each barrier wait costs that thread tens of
+// nanoseconds, which bounds a decode batch's small MMAs).
+// kSub stages share one raw stage of kRawRowBytes per row (kSubBytes each).
 template <int FMT> struct TcFmt;
 template <> struct TcFmt<MOE_W_BF16> {
-    static constexpr int kSub = 1, kSubBytes = 0, kAStages = 8, kRawStages = 0, kBRegion = 64 * 1024;
+    static constexpr int kKS = 64, kSub = 1, kSubBytes = 0, kAStages = 8, kASmem = 1, kRawStages = 0;
+    static constexpr int kBRegion = 64 * 1024, kTmemCols = kAccCols;
 };
 template <> struct TcFmt<MOE_W_INT8> {
-    static constexpr int kSub = 2, kSubBytes = 64, kAStages = 4, kRawStages = 5, kBRegion = 48 * 1024;
+    static constexpr int kKS = 128, kSub = 1, kSubBytes = 128, kAStages = 4, kASmem = 0, kRawStages = 6;
+    static constexpr int kBRegion = 96 * 1024, kTmemCols = 512;  // accumulators, then 4 A stages of 64 columns
 };
 template <> struct TcFmt<MOE_W_INT4> {
-    static constexpr int kSub = 4, kSubBytes = 32, kAStages = 4, kRawStages = 5, kBRegion = 48 * 1024;
+    static constexpr int kKS = 128, kSub = 2, kSubBytes = 64, kAStages = 4, kASmem = 0, kRawStages = 6;
+    static constexpr int kBRegion = 96 * 1024, kTmemCols = 512;
 };
 
 // First problem a tensor-core kernel recorded (0 = none): 0x1000 | role for
@@ -144,9 +159,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
@@ -174,6 +186,27 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, ui
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// A from tensor memory (columns a_tmem.. of lanes 0..127, bf16 pairs), B from
+// shared memory.
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's TMEM lane (asynchronous:
+// tmem_st_wait() orders them before what follows).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // 16 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
     uint32_t r[16];
@@ -205,7 +238,8 @@ struct Items {
     int n_act, total, m_tiles, n_block, b_slots;
 };
 
-__device__ void build_items(const TcParams &p, int m_tiles, int b_region, int *s_act, int *s_base, Items *it) {
+__device__ void build_items(const TcParams &p, int m_tiles, int b_region, int atoms, int *s_act, int *s_base,
+                            Items *it) {
     const int lane = threadIdx.x & 31;
     if (threadIdx.x < 32) {
         int n_max = 1;
@@ -240,7 +274,7 @@ __device__ void build_items(const TcParams &p, int m_tiles, int b_region, int *s
             it->total = run;
             it->m_tiles = m_tiles;
             it->n_block = n_block;
-            it->b_slots = min(kMaxBSlots, b_region / (n_block * 128));
+            it->b_slots = min(kMaxBSlots, b_region / (n_block * 128 * atoms));
         }
     }
 }
@@ -302,12 +336,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     constexpr int RAW = kRawBytes<FMT>();
     constexpr int SUB = TcFmt<FMT>::kSub;
     constexpr bool kDeq = FMT != MOE_W_BF16;
+    constexpr int KS = TcFmt<FMT>::kKS, ATOMS = KS / kBlockK;
+    constexpr int A_COLS = KS / 2;  // TMEM columns of one A stage (int formats: bf16 pairs)
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned carve-up: A ring | B region | raw ring | exchange | barriers
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
-    uint8_t *sB = sA + SA * kATileBytes;
+    uint8_t *sB = sA + (TcFmt<FMT>::kASmem ? SA * kATileBytes : 0);
     uint8_t *sRaw = sB + TcFmt<FMT>::kBRegion;
     float *sX = reinterpret_cast<float *>(sRaw + SR * RAW);       // [2][64][kXPitch] gate/up exchange
     uint64_t *bars = reinterpret_cast<uint64_t *>(sX + 2 * 64 * kXPitch);
@@ -330,7 +366,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = PHASE == 1 ? p.L.I / 64 : (p.L.H + kBlockM - 1) / kBlockM;
-    const int nk = p.K / kBlockK;
+    const int nk = (p.K + KS - 1) / KS;  // stages; the last may hold fewer atoms (p.K is a multiple of 64)
+    auto atoms_at = [&](int kk) { return min(ATOMS, (p.K - kk * KS) / kBlockK); };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SA; ++i) {
@@ -358,18 +395,19 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                     "r"(kTmemCols)
+                     "r"(TcFmt<FMT>::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    build_items(p, m_tiles, TcFmt<FMT>::kBRegion, s_act, s_base, &s_items);
+    build_items(p, m_tiles, TcFmt<FMT>::kBRegion, ATOMS, s_act, s_base, &s_items);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     const int n_act = s_items.n_act, total = s_items.total;
     const int n_block = s_items.n_block, b_slots = s_items.b_slots;
-    const uint32_t b_slot_bytes = (uint32_t)n_block * 128;
+    const uint32_t b_atom_bytes = (uint32_t)n_block * 128;       // one 64-wide atom of a B slot
+    const uint32_t b_slot_bytes = b_atom_bytes * ATOMS;
 
     if (warp == 0) {
         // ------------------------------------- A producer: weights or raw codes
@@ -420,11 +458,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                 const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 bool ok = true;
                 for (int kk = 0; kk < nk; ++kk) {
+                    const int na = atoms_at(kk);
                     if (!mbar_wait(&b_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&b_full[stage], (uint32_t)it.n_mma * 128);
+                    mbar_arrive_expect_tx(&b_full[stage], (uint32_t)(na * it.n_mma * 128));
                     uint8_t *db = sB + stage * b_slot_bytes;
-                    for (int j = 0; j < it.n_mma; j += 16)
-                        tma_load_2d(db + j * 128, &map_b, &b_full[stage], kk * kBlockK, it.row0 + j);
+                    for (int a = 0; a < na; ++a)
+                        for (int j = 0; j < it.n_mma; j += 16)
+                            tma_load_2d(db + a * b_atom_bytes + j * 128, &map_b, &b_full[stage],
+                                        (kk * ATOMS + a) * kBlockK, it.row0 + j);
                     if (++stage == b_slots) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
@@ -447,13 +488,28 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                 bool ok = true;
                 for (int kk = 0; kk < nk; ++kk) {
                     if (!mbar_wait(&a_full[sa], pa, &s_abort)) { ok = false; break; }
-                    if (!mbar_wait(&b_full[sb], pb, &s_abort)) { ok = false; break; }
+                    // int formats: the dequant warps saw this B slot land before
+                    // they completed a_full, so only bf16 waits for it here
+                    if (!kDeq && !mbar_wait(&b_full[sb], pb, &s_abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + sa * kATileBytes);
                     const uint32_t b0 = smem_u32(sB + sb * b_slot_bytes);
+                    if (kDeq) {
+                        // A stage sa: TMEM columns kAccCols + A_COLS sa .., 32 per atom,
+                        // 8 per 16-wide K step
+                        const uint32_t a_t = tmem + (uint32_t)(kAccCols + sa * A_COLS);
+                        const int na = atoms_at(kk);
+                        for (int a = 0; a < na; ++a) {
 #pragma unroll
-                    for (int j = 0; j < kBlockK / 16; ++j)
-                        tc_mma_bf16(d, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc, (kk | j) != 0);
+                            for (int j = 0; j < kBlockK / 16; ++j)
+                                tc_mma_bf16_ts(d, a_t + 32 * a + 8 * j, sw128_desc(b0 + a * b_atom_bytes + 32 * j),
+                                               idesc, (kk | a | j) != 0);
+                        }
+                    } else {
+                        const uint32_t a0 = smem_u32(sA + sa * kATileBytes);
+#pragma unroll
+                        for (int j = 0; j < kBlockK / 16; ++j)
+                            tc_mma_bf16(d, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc, (kk | j) != 0);
+                    }
                     tc_commit(&a_empty[sa]);
                     tc_commit(&b_empty[sb]);
                     if (++sa == SA) { sa = 0; pa ^= 1; }
@@ -543,16 +599,21 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         }
     } else if (kDeq) {
         // ---------------------------------------------------- dequantisation
-        // two threads per tile row (half a row, 32 weights = 4 chunks, each):
-        // raw codes -> bf16 in the 128-byte-swizzled K-major layout (8-row groups
-        // of 1024 bytes, 16-byte chunk c of row r stored at chunk c ^ (r % 8)).
+        // two threads per tile row, each expanding one 64-wide atom of the
+        // stage (64 weights): raw codes -> 32 bf16 pairs -> TMEM lane r,
+        // columns 32 hf .. 32 hf + 31 of the A stage.  A warp may only reach
+        // TMEM lanes 32 (warp % 4) .. +31, so the row is taken from the warp's
+        // lane quadrant; the eight warps of a group cover each quadrant twice
+        // (both atoms of its rows).  The first warp of the group also waits for
+        // the stage's B slot, so a completed a_full means A and B are both ready.
         const int dw = warp - kWarpDeq0;              // 0 .. kDeqGroups*kDeqWarps-1
         const int group = dw / kDeqWarps;
-        const int t = (dw % kDeqWarps) * 32 + lane;
-        const int r = t & (kBlockM - 1), hf = t >> 7;
-        int stage = 0, rstage = 0;
-        uint32_t phase = 0, rphase = 0;
-        uint32_t step = 0;                              // k-steps seen, across items
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane, hf = (dw % kDeqWarps) / 4;
+        const bool b_waiter = (dw % kDeqWarps) == 0;
+        int stage = 0, rstage = 0, bstage = 0;
+        uint32_t phase = 0, rphase = 0, bphase = 0;
+        uint32_t step = 0;                              // stages seen, across items
         for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
             const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
             const uint8_t *blob = expert_blob(p.L, it.e);
@@ -563,9 +624,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             bool ok = true;
             for (int kk = 0; kk < nk; ++kk, ++step) {
                 const int sub = kk % SUB;
-                const bool raw_last = sub == SUB - 1 || kk == nk - 1;  // last MMA stage of this raw stage
+                const bool raw_last = sub == SUB - 1 || kk == nk - 1;  // last stage of this raw stage
                 if ((int)(step % kDeqGroups) != group) {   // the other group's stage
                     if (++stage == SA) { stage = 0; phase ^= 1; }
+                    if (++bstage == b_slots) { bstage = 0; bphase ^= 1; }
                     if (raw_last) {
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&r_empty[rstage]);
@@ -573,63 +635,79 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     }
                     continue;
                 }
+                const bool mine = hf < atoms_at(kk);  // this thread's atom lies inside K
                 __nv_bfloat162 s2 = __floats2bfloat162_rn(0.0f, 0.0f);
-                if (FMT == MOE_W_INT4) s2 = __bfloat162bfloat162(__ushort_as_bfloat16(__ldg(srow + kk)));
+                if (FMT == MOE_W_INT4 && mine)
+                    s2 = __bfloat162bfloat162(__ushort_as_bfloat16(__ldg(srow + kk * ATOMS + hf)));
                 // the codes have landed, and the MMAs are done with this A slot
                 if (!mbar_wait(&r_full[rstage], rphase, &s_abort)) { ok = false; break; }
                 if (!mbar_wait(&a_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
-                const uint8_t *src = sRaw + rstage * RAW + r * kRawRowBytes + sub * TcFmt<FMT>::kSubBytes;
-                uint8_t *dst = sA + stage * kATileBytes + (r >> 3) * 1024 + (r & 7) * 128;
-                if (FMT == MOE_W_INT4) {
-                    // 16 raw bytes = weights 32hf .. 32hf+31 = chunks 4hf .. 4hf+3
-                    const uint4 u = *reinterpret_cast<const uint4 *>(src + 16 * hf);
-                    const uint32_t words[4] = {u.x, u.y, u.z, u.w};
-                    // bf16 128 + n (n in the low mantissa bits of 128.0 = 0x4300),
-                    // minus 136 -> n - 8 exactly, times s -> one rounding
-                    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+                tc_fence_after();
+                if (mine) {
+                    // the raw tile landed 128-byte swizzled (16-byte chunk j of row r
+                    // at chunk j ^ (r % 8)), so the 32 rows a warp reads at once
+                    // spread over all banks
+                    const uint8_t *src = sRaw + rstage * RAW + r * kRawRowBytes;
+                    // first 16-byte chunk of this thread's atom: 64 codes = 32 (int4) / 64 (int8) bytes
+                    const int cj0 = sub * (TcFmt<FMT>::kSubBytes / 16) + hf * (FMT == MOE_W_INT4 ? 2 : 4);
+                    uint32_t o[32];  // bf16 pairs (weights 64 hf + 2j, +1 in the low, high half)
+                    if (FMT == MOE_W_INT4) {
+                        // bf16 128 + n (n in the low mantissa bits of 128.0 = 0x4300),
+                        // minus 136 -> n - 8 exactly, times s -> one rounding
+                        const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        // byte j of the word = weight 2j (low nibble), 2j+1 (high)
-                        const uint32_t w = words[i], w4 = w >> 4;
-                        uint32_t o[4];
+                        for (int c = 0; c < 2; ++c) {
+                            const uint4 u = *reinterpret_cast<const uint4 *>(src + (((cj0 + c) ^ (r & 7)) << 4));
+                            const uint32_t words[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            // {w.byte j, -, (w >> 4).byte j, -}: n_lo and n_hi in the low bits of each half
-                            const uint32_t dup = __byte_perm(w, w4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
-                            uint32_t v = (dup & 0x000F000Fu) | 0x43004300u;
-                            __nv_bfloat162 q = *reinterpret_cast<__nv_bfloat162 *>(&v);
-                            q = __hmul2(__hsub2(q, bias), s2);
-                            o[j] = *reinterpret_cast<uint32_t *>(&q);
+                            for (int i = 0; i < 4; ++i) {
+                                // byte j of the word = weight 2j (low nibble), 2j+1 (high)
+                                const uint32_t w = words[i], w4 = w >> 4;
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    // {w.byte j, -, (w >> 4).byte j, -}: n_lo and n_hi in the low bits of each half
+                                    const uint32_t dup =
+                                        __byte_perm(w, w4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
+                                    uint32_t v = (dup & 0x000F000Fu) | 0x43004300u;
+                                    __nv_bfloat162 q = *reinterpret_cast<__nv_bfloat162 *>(&v);
+                                    q = __hmul2(__hsub2(q, bias), s2);
+                                    o[16 * c + 4 * i + j] = *reinterpret_cast<uint32_t *>(&q);
+                                }
+                            }
                         }
-                        const int c = 4 * hf + i;
-                        *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {  // 8 int8 codes -> 16-byte chunk c (codes exact in bf16)
-                        const int c = 4 * hf + i;
-                        const uint2 u = *reinterpret_cast<const uint2 *>(src + 8 * c);
-                        const uint32_t a = u.x ^ 0x80808080u, b = u.y ^ 0x80808080u;
-                        uint32_t o[4];
+                        for (int c = 0; c < 4; ++c) {  // 16 codes per chunk -> 8 bf16 pairs (codes exact in bf16)
+                            const uint4 u = *reinterpret_cast<const uint4 *>(src + (((cj0 + c) ^ (r & 7)) << 4));
+                            const uint32_t words[4] = {u.x ^ 0x80808080u, u.y ^ 0x80808080u, u.z ^ 0x80808080u,
+                                                       u.w ^ 0x80808080u};
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t src_w = j < 2 ? a : b;
-                            const uint32_t sel0 = 0x7540u | (uint32_t)(2 * (j & 1)), sel1 = sel0 + 1;
-                            const float f0 = __uint_as_float(__byte_perm(src_w, 0x4B000000u, sel0)) - 8388736.0f;
-                            const float f1 = __uint_as_float(__byte_perm(src_w, 0x4B000000u, sel1)) - 8388736.0f;
-                            __nv_bfloat162 q = __floats2bfloat162_rn(f0, f1);
-                            o[j] = *reinterpret_cast<uint32_t *>(&q);
+                            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                                for (int j = 0; j < 2; ++j) {
+                                    const uint32_t sel0 = 0x7540u | (uint32_t)(2 * j), sel1 = sel0 + 1;
+                                    const float f0 = __uint_as_float(__byte_perm(words[i], 0x4B000000u, sel0)) - 8388736.0f;
+                                    const float f1 = __uint_as_float(__byte_perm(words[i], 0x4B000000u, sel1)) - 8388736.0f;
+                                    __nv_bfloat162 q = __floats2bfloat162_rn(f0, f1);
+                                    o[8 * c + 2 * i + j] = *reinterpret_cast<uint32_t *>(&q);
+                                }
+                            }
                         }
-                        *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                     }
+                    const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(kAccCols + stage * A_COLS + 32 * hf);
+                    tmem_st16(ta, o);
+                    tmem_st16(ta + 16, o + 16);
+                    tmem_st_wait();
                 }
-                fence_proxy_async_smem();
+                if (b_waiter && !mbar_wait(&b_full[bstage], bphase, &s_abort)) { ok = false; break; }
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&a_full[stage]);
                     if (raw_last) mbar_arrive(&r_empty[rstage]);
                 }
                 if (++stage == SA) { stage = 0; phase ^= 1; }
+                if (++bstage == b_slots) { bstage = 0; bphase ^= 1; }
                 if (raw_last && ++rstage == SR) { rstage = 0; rphase ^= 1; }
             }
             if (!ok) break;
@@ -640,7 +718,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TcFmt<FMT>::kTmemCols)
+                     : "memory");
     }
 }
 
@@ -694,7 +773,7 @@ bool encode_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int ele
 
 template <int FMT>
 constexpr size_t smem_bytes() {
-    return 1024 + (size_t)TcFmt<FMT>::kAStages * kATileBytes + TcFmt<FMT>::kBRegion +
+    return 1024 + (size_t)(TcFmt<FMT>::kASmem ? TcFmt<FMT>::kAStages : 0) * kATileBytes + TcFmt<FMT>::kBRegion +
            (size_t)TcFmt<FMT>::kRawStages * kRawBytes<FMT>() + 2 * 64 * kXPitch * 4 +
            (size_t)(2 * TcFmt<FMT>::kAStages + 2 * kMaxBSlots + 2 * kAccBufs + 4 + 2 * TcFmt<FMT>::kRawStages) * 8;
 }
@@ -766,7 +845,7 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     const bool bf = fmt == MOE_W_BF16;
     const CUtensorMapDataType dt = bf ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     const int eb = bf ? 2 : 1;
-    const CUtensorMapSwizzle swa = bf ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const CUtensorMapSwizzle swa = CU_TENSOR_MAP_SWIZZLE_128B;  // weight tiles and raw code tiles alike
     const uint32_t raw_inner = kRawRowBytes;
     CUtensorMap mh1, mp1, mh2, mp2, mb1, mb2;
     for (int ph = 1; ph <= 2; ++ph) {

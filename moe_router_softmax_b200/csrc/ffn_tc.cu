@@ -406,6 +406,12 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     const uint32_t tmem = s_tmem;
     const int n_act = s_items.n_act, total = s_items.total;
     const int n_block = s_items.n_block, b_slots = s_items.b_slots;
+    // A small route block leaves each MMA little work, and consecutive MMAs
+    // into one accumulator wait on each other's result; the four 16-wide K
+    // steps of a 64-wide atom then go to nacc separate partial accumulators
+    // (n_block columns apart inside the accumulator's kNMax columns), which the
+    // epilogue adds up.
+    const int nacc = n_block <= kNMax / 4 ? 4 : (n_block <= kNMax / 2 ? 2 : 1);
     const uint32_t b_atom_bytes = (uint32_t)n_block * 128;       // one 64-wide atom of a B slot
     const uint32_t b_slot_bytes = b_atom_bytes * ATOMS;
 
@@ -501,14 +507,16 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                         for (int a = 0; a < na; ++a) {
 #pragma unroll
                             for (int j = 0; j < kBlockK / 16; ++j)
-                                tc_mma_bf16_ts(d, a_t + 32 * a + 8 * j, sw128_desc(b0 + a * b_atom_bytes + 32 * j),
-                                               idesc, (kk | a | j) != 0);
+                                tc_mma_bf16_ts(d + (uint32_t)((j % nacc) * n_block), a_t + 32 * a + 8 * j,
+                                               sw128_desc(b0 + a * b_atom_bytes + 32 * j), idesc,
+                                               (kk | a | (j / nacc)) != 0);
                         }
                     } else {
                         const uint32_t a0 = smem_u32(sA + sa * kATileBytes);
 #pragma unroll
                         for (int j = 0; j < kBlockK / 16; ++j)
-                            tc_mma_bf16(d, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc, (kk | j) != 0);
+                            tc_mma_bf16(d + (uint32_t)((j % nacc) * n_block), sw128_desc(a0 + 32 * j),
+                                        sw128_desc(b0 + 32 * j), idesc, (kk | (j / nacc)) != 0);
                     }
                     tc_commit(&a_empty[sa]);
                     tc_commit(&b_empty[sb]);
@@ -543,6 +551,12 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             for (int c0 = 0; c0 < it.n_mma; c0 += 16) {
                 float v[16];
                 tmem_ld16(taddr + (uint32_t)c0, v);
+                for (int pa = 1; pa < nacc; ++pa) {
+                    float w[16];
+                    tmem_ld16(taddr + (uint32_t)(pa * n_block + c0), w);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] += w[i];
+                }
                 if (PHASE == 1) {
                     // tile rows 64..127 hold the up projection, rows 0..63 the gate of
                     // the same intermediate columns: the up warps pass their values

@@ -77,6 +77,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--quick", action="store_true", help="main batch only: no sweep, no e2e, no CPU baseline")
+    ap.add_argument("--stack-refresh", default="device", choices=["device", "host"],
+                    help="stack30: placement refresh on the device (graph-captured, copies overlapped) or on the host")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"],
                     help="grouped-FFN kernels: AUTO picks by routes per call")
     return ap.parse_args()
@@ -246,7 +248,7 @@ class Runner:
     def launches_per_step(self):
         """route, permute, FFN (2 GEMV launches, or gather + 2 tensor-core launches), combine"""
         R = self.T * self.k
-        auto_tc = R >= (65 if self.layers[0].fmt == self.moe.MOE_W_INT4 else 32)
+        auto_tc = R >= (32 if self.layers[0].fmt == self.moe.MOE_W_BF16 else 96)
         tc = self.path == self.moe.MOE_FFN_TC or (self.path == self.moe.MOE_FFN_AUTO and auto_tc)
         return 4 + (3 if tc else 2)
 
@@ -587,12 +589,14 @@ class Stack:
         self.slot_of = []
         self.layers = []
         self.pools = []
+        self.tables = torch.empty((L, E), dtype=torch.int32, device=dev)  # row l = layer l's slot table
         for l in range(L):
             so = np.full(E, -1, np.int32)
             so[:slots] = np.arange(slots)
             pool = torch.empty(slots * self.eb, dtype=torch.uint8, device=dev)
             moe.moe_copy_to_slots(self.homes[l].home, pool, self.eb, np.arange(slots), np.arange(slots))
-            table = torch.from_numpy(so).to(dev)
+            table = self.tables[l]
+            table.copy_(torch.from_numpy(so))
             self.layers.append(moe.MoeLayer(self.fmt, E, H, I, self.homes[l].home, pool=pool, slot_table=table,
                                             expert_bytes=self.eb))
             self.slot_of.append(so)
@@ -705,6 +709,116 @@ def stack_steps(torch, moe, stack, T, k, steps, warmup, seed, refresh_every=8, p
     return t0.elapsed_time(t1)
 
 
+def stack_steps_device(torch, moe, stack, T, k, steps, warmup, seed, refresh_every=8, path=0):
+    """The same decode steps with the placement refresh done on the device
+    (moe_refresh_device after each layer's forward at the refresh step, its
+    promotion copies on a second stream, joined before that layer's next
+    forward), so that a window of `refresh_every` steps is one CUDA graph with
+    no host round trip and the copies overlap the following layers' compute.
+    `steps` and `warmup` are rounded up to whole windows.  Returns (total ms,
+    steps timed)."""
+    import synthetic as syn
+
+    dev = stack.layers[0].home.device
+    E, H, L, S = stack.E, stack.H, stack.L, stack.slots
+    W = refresh_every
+    steps = -(-steps // W) * W
+    warmup = max(1, -(-warmup // W)) * W
+    n = steps + warmup
+    lg_all = torch.empty((n, L, T, E), dtype=torch.float32, device=dev)
+    x_all = torch.empty((n, T, H), dtype=torch.bfloat16, device=dev)
+    for st in range(n):
+        lg_all[st] = torch.from_numpy(np.stack([syn.router_logits(T, E, "zipf", seed=seed, layer=l, step=st)
+                                                for l in range(L)])).to(dev)
+        x_all[st] = torch.from_numpy(syn.activations(T, H, seed=seed, layer=st).view(np.int16)).to(dev).view(torch.bfloat16)
+    lg_stage = torch.empty((W, L, T, E), dtype=torch.float32, device=dev)
+    x_stage = torch.empty((W, T, H), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(moe.moe_grouped_ffn_workspace(stack.layers[0], T, k), dtype=torch.uint8, device=dev)
+    R = T * k
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    perm = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
+            torch.empty(R, dtype=torch.int32, device=dev), torch.empty(R, dtype=torch.int32, device=dev))
+    rows = torch.empty((R, H), dtype=torch.float32, device=dev)
+    ybuf = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    hits = torch.zeros((L, E), dtype=torch.int32, device=dev)
+    promo = torch.zeros((L, S, 2), dtype=torch.int32, device=dev)
+    status = torch.zeros((L, 3), dtype=torch.int32, device=dev)
+    snap = torch.empty((L, E), dtype=torch.int32, device=dev)
+    acc = torch.zeros(4, dtype=torch.int64, device=dev)  # promotions, demotions, resident routes, routes
+    side = torch.cuda.Stream(dev)
+
+    def layer(j, l, x):
+        moe.moe_route_topk(lg_stage[j, l], k, ids, w)
+        moe.moe_permute(ids, E, hits=hits[l] if j == 0 else None, out=perm)
+        moe.moe_grouped_ffn(stack.layers[l], x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
+        y = ybuf[l & 1]
+        moe.moe_combine(rows, perm[3], w, y)
+        return y
+
+    def window():
+        main = torch.cuda.current_stream()
+        hits.zero_()
+        snap.copy_(stack.tables)
+        done = []
+        x = x_stage[0]
+        for l in range(L):
+            x = layer(0, l, x)
+            moe.moe_refresh_device(hits[l], S, stack.tables[l], S, promo=promo[l], status=status[l])
+            ev = torch.cuda.Event()
+            ev.record(main)
+            side.wait_event(ev)
+            with torch.cuda.stream(side):
+                moe.moe_promote_copies(stack.homes[l].home, stack.pools[l], stack.eb, promo[l], status[l], S)
+                ev2 = torch.cuda.Event()
+                ev2.record(side)
+            done.append(ev2)
+        acc[0] += status[:, 0].sum()
+        acc[1] += status[:, 1].sum()
+        acc[2] += (hits * (snap >= 0)).sum()
+        acc[3] += hits.sum()
+        for j in range(1, W):
+            x = x_stage[j]
+            for l in range(L):
+                if j == 1:
+                    main.wait_event(done[l])  # layer l's promoted blobs and table are in place
+                x = layer(j, l, x)
+        main.wait_stream(side)
+
+    def window_inputs(first):
+        lg_stage.copy_(lg_all[first:first + W])
+        x_stage.copy_(x_all[first:first + W])
+
+    window_inputs(0)
+    window()  # one-time set-up outside the capture (it also performs a refresh)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        window()
+    torch.cuda.synchronize()
+    acc.zero_()
+
+    def run(first, count):
+        for st in range(first, first + count, W):
+            window_inputs(st)
+            g.replay()
+
+    run(0, warmup)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    run(warmup, steps)
+    t1.record()
+    torch.cuda.synchronize()
+    a = acc.cpu().numpy()
+    windows = (warmup + steps) // W
+    stack.stats = {"refreshes": windows, "promotions": int(a[0]), "demotions": int(a[1]),
+                   "resident_route_share": [float(a[2]) / float(a[3])] if a[3] else []}
+    del g
+    return t0.elapsed_time(t1), steps
+
+
 def stack_main(args, T, E, H, I, k, world, rank, local):
     """30-layer stacks (int4 and bf16, both resident), 18 cache slots per layer,
     Zipf(1.1) routing, placement refresh every 8 steps; tokens/s through the stack."""
@@ -720,27 +834,37 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
     path = {"auto": moe.MOE_FFN_AUTO, "gemv": moe.MOE_FFN_GEMV, "tc": moe.MOE_FFN_TC}[args.path]
     s4 = Stack(moe, torch, "int4", E, H, I, L, slots, dev, seed=1)
     s16 = Stack(moe, torch, "bf16", E, H, I, L, slots, dev, seed=2)
+    device_refresh = args.stack_refresh == "device"
+
+    def run_stack(st, Ts, seed):
+        if device_refresh:
+            return stack_steps_device(torch, moe, st, Ts, k, steps, warmup, seed=seed, path=path)
+        return stack_steps(torch, moe, st, Ts, k, steps, warmup, seed=seed, path=path), steps
+
     resident_gb = (sum(h.home.numel() for h in s4.homes) + sum(h.home.numel() for h in s16.homes) +
                    sum(p.numel() for p in s4.pools) + sum(p.numel() for p in s16.pools)) / 1e9
     clocks = ClockSampler(local)
     clocks.start()
-    ms = stack_steps(torch, moe, s4, T, k, steps, warmup, seed=11, path=path)
+    ms, steps_done = run_stack(s4, T, 11)
     clk = clocks.stop()
-    value = world * T * steps / (ms / 1e3)
+    value = world * T * steps_done / (ms / 1e3)
     sweep = {}
     for name, st, Ts in [("bf16", s16, T)] + ([] if args.quick else [("int4", s4, t) for t in (1, 8) if t != T]):
-        ms2 = stack_steps(torch, moe, st, Ts, k, steps, warmup, seed=12 + Ts, path=path)
-        sweep[f"{name}_T{Ts}"] = {"tokens_per_s": round(world * Ts * steps / (ms2 / 1e3), 1),
-                                  "ms_per_step": round(ms2 / steps, 4)}
+        ms2, n2 = run_stack(st, Ts, 12 + Ts)
+        sweep[f"{name}_T{Ts}"] = {"tokens_per_s": round(world * Ts * n2 / (ms2 / 1e3), 1),
+                                  "ms_per_step": round(ms2 / n2, 4)}
     share = s4.stats["resident_route_share"]
     hbm_peak = measured_peaks()[0]
     line = {
         "metric": "MoE layer tokens/s and expert-weight HBM GB/s (% of roofline) at decode/prefill",
-        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warmup,
-        "ms_per_step": round(ms / steps, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": steps_done, "warmup": warmup,
+        "ms_per_step": round(ms / steps_done, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4", "data": "synthetic (seeded; Zipf(1.1) routing; random weights)",
         "config": {"workload": f"moe-stack{L}-int4-decode-T{T}", "layers": L, "experts": E, "hidden": H,
                    "intermediate": I, "top_k": k, "tokens": T, "slots_per_layer": slots, "refresh_every": 8,
+                   "refresh": ("on the device, promotion copies on a second stream overlapping compute; one CUDA "
+                               "graph per 8-step window" if device_refresh else
+                               "on the host (hit histogram read back, placement, copies, table upload)"),
                    "logits": "zipf(1.1)", "resident_gb": round(resident_gb, 1), "ffn_path": args.path,
                    "l2": "inputs larger than L2: each step reads 30 layers' routed experts"},
         "placement": {"refreshes": s4.stats["refreshes"], "promotions": s4.stats["promotions"],
@@ -748,8 +872,9 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
                       "routes_on_resident_slots": round(sum(share) / len(share), 4) if share else None},
         "sweep": sweep,
         "hbm_peak_gbs": hbm_peak,
-        "gpu_launches": steps * L * (4 + (3 if (path == moe.MOE_FFN_TC or
-                                                 (path == moe.MOE_FFN_AUTO and T * k >= 65)) else 2)),
+        "gpu_launches": steps_done * L * (4 + (3 if (path == moe.MOE_FFN_TC or
+                                                      (path == moe.MOE_FFN_AUTO and T * k >= 96)) else 2))
+                        + (steps_done // 8) * L * (2 if device_refresh else 0),
         "clocks": clk,
     }
     if rank == 0:

@@ -266,6 +266,31 @@ MOE_API moe_status moe_quantize_int4(const uint16_t *w, int32_t rows, int32_t K,
 MOE_API moe_status moe_pack_expert(int32_t fmt, const void *w13, const void *s13, const void *w2, const void *s2,
                            int32_t H, int32_t I, void *blob, moe_stream_t stream);
 
+/*
+ * The placement refresh on the device (rlx_runtime expert_pool.rs,
+ * target_gpu_from_counts then apply_target_placement): exactly what
+ * moe_refresh_target followed by moe_apply_placement compute on the host, with
+ * every array in device memory, so that a refresh needs no host round trip and
+ * can be captured in a CUDA graph.  hits uint32 [E]; slot_table int32 [E] (the
+ * layer's table, updated in place: demoted experts get -1, promoted experts
+ * their new slot); promo int32 [2 * n_slots] receives (expert, slot) pairs in
+ * promotion order; status int32 [3] receives {promotions, demotions, 0}, or
+ * {0, 0, 1} when slot_table was inconsistent (a slot >= n_slots or held twice:
+ * nothing is changed).  budget <= n_slots <= 1024, E <= 1024.  One CTA.
+ */
+MOE_API moe_status moe_refresh_device(const uint32_t *hits, int32_t E, int32_t budget, int32_t *slot_table,
+                                      int32_t n_slots, int32_t *promo, int32_t *status, moe_stream_t stream);
+
+/*
+ * The promotion copies of a device refresh: for j < min(status[0], max_promo),
+ * blob promo[2j] of home is copied into slot promo[2j+1] of pool (one kernel
+ * reading the list from device memory; expert_bytes a multiple of 16, home and
+ * pool 16-byte aligned).  Issue it on a second stream to overlap it with
+ * compute; the layer's next forward must be ordered after it (an event).
+ */
+MOE_API moe_status moe_promote_copies(const void *home, void *pool, uint64_t expert_bytes, const int32_t *promo,
+                                      const int32_t *status, int32_t max_promo, moe_stream_t stream);
+
 /* Copy blobs of experts experts[i] from home into pool slot slots[i] (the
  * promotion copies of a placement refresh).  experts and slots are HOST
  * arrays of n entries.  Device-to-device copies on `stream`. */

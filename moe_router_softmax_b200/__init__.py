@@ -36,7 +36,7 @@ EXPORTS = [
     "moe_layer_forward_workspace", "moe_layer_forward", "moe_quantize_int8", "moe_quantize_int4",
     "moe_pack_expert", "moe_copy_to_slots", "moe_refresh_target", "moe_apply_placement",
     "moe_should_refresh", "moe_budget_from_vram", "moe_grouped_ffn_noalloc", "moe_take_device_errors",
-    "moe_route_min_weight", "moe_router_topk", "moe_hits_window",
+    "moe_route_min_weight", "moe_router_topk", "moe_hits_window", "moe_refresh_device", "moe_promote_copies",
 ]
 
 
@@ -83,6 +83,8 @@ _SIG = {
     "moe_route_min_weight": (i32, [P, P, P, i32, i32, i32, ctypes.c_float, P]),
     "moe_router_topk": (i32, [P, P, i32, i32, i32, i32, P, P, P, P]),
     "moe_hits_window": (i32, [P, i32, i32, P]),
+    "moe_refresh_device": (i32, [P, i32, i32, P, i32, P, P, P]),
+    "moe_promote_copies": (i32, [P, P, u64, P, P, i32, P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -354,6 +356,29 @@ def moe_hits_window(ring: np.ndarray) -> np.ndarray:
     out = np.zeros(E, np.uint32)
     _check(_lib.moe_hits_window(pr, W, E, out.ctypes.data_as(ctypes.c_void_p)))
     return out
+
+
+def moe_refresh_device(hits: torch.Tensor, budget: int, slot_table: torch.Tensor, n_slots: int,
+                       promo: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None):
+    """Device placement refresh (slot_table updated in place).  Returns (promo, status):
+    promo int32 [n_slots, 2] (expert, slot) pairs, status int32 [3] (promotions, demotions, error)."""
+    E = slot_table.numel()
+    dev = slot_table.device
+    promo = torch.empty((max(n_slots, 1), 2), dtype=torch.int32, device=dev) if promo is None else promo
+    status = torch.empty(3, dtype=torch.int32, device=dev) if status is None else status
+    _check(_lib.moe_refresh_device(_dev(hits, (torch.int32, torch.uint32), "hits"), E, budget,
+                                   _dev(slot_table, torch.int32, "slot_table"), n_slots,
+                                   _dev(promo, torch.int32, "promo"), _dev(status, torch.int32, "status"),
+                                   _stream(stream)))
+    return promo, status
+
+
+def moe_promote_copies(home: torch.Tensor, pool: torch.Tensor, expert_bytes: int, promo: torch.Tensor,
+                       status: torch.Tensor, max_promo: int, stream=None) -> None:
+    """Copy the promoted blobs listed on the device by moe_refresh_device."""
+    _check(_lib.moe_promote_copies(_dev(home, None, "home"), _dev(pool, None, "pool"), expert_bytes,
+                                   _dev(promo, torch.int32, "promo"), _dev(status, torch.int32, "status"),
+                                   max_promo, _stream(stream)))
 
 
 def moe_should_refresh(offload_enabled: bool, mode_refresh: bool, step: int, is_prefill_block: bool,

@@ -14,6 +14,8 @@ cudaError_t launch_router_topk(const uint16_t *, const float *, int, int, int, i
 int router_tok(int T, int H, int E);
 size_t router_smem(int tok, int H, int E);
 extern const size_t kRouterMaxSmemBytes;
+cudaError_t launch_refresh_placement(const uint32_t *, int, int, int32_t *, int, int32_t *, int32_t *, cudaStream_t);
+cudaError_t launch_promote_copies(const void *, void *, uint64_t, const int32_t *, const int32_t *, int, cudaStream_t);
 cudaError_t launch_route_min_weight(int32_t *, float *, const int32_t *, int, int, int, float, cudaStream_t);
 cudaError_t launch_permute(const int32_t *, int, int, int32_t *, int32_t *, int32_t *, int32_t *, uint32_t *,
                            cudaStream_t);
@@ -203,10 +205,11 @@ moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *x, int32
     const int R = T * k;
     int use = path;
     if (use == MOE_FFN_AUTO) {
-        // measured on B200 (Gemma-shaped layer): the tensor-core kernels win from
-        // 4 tokens x top-8 for bf16/int8 weights and above 8 tokens for int4; one
-        // token stays on the GEMV kernels
-        const int min_routes = v.fmt == MOE_W_INT4 ? 65 : 32;
+        // measured on B200 (Gemma-shaped layer, top-8): the tensor-core kernels
+        // win from 4 tokens for bf16 weights and from about 12 tokens for int8 /
+        // int4 (at 8 tokens the GEMV is faster: 115 vs 154 us int4, 128 vs 140 us
+        // int8; at 16 the tensor cores: 203 vs 224, 194 vs 224)
+        const int min_routes = v.fmt == MOE_W_BF16 ? 32 : 96;
         use = (R >= min_routes && ffn_tc_supports(v.fmt, v.H, v.I, v.stride)) ? MOE_FFN_TC : MOE_FFN_GEMV;
     }
     if (use == MOE_FFN_TC && !ffn_tc_supports(v.fmt, v.H, v.I, v.stride))
@@ -342,6 +345,29 @@ moe_status moe_take_device_errors(uint32_t *code, uint32_t *info) {
         return set_error(MOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (warp %u)", c & 0xFFFu);
     if (c) return set_error(MOE_ERR_CUDA, "a tensor-core kernel failed an index check (site %u, value %u)", c & 0xFFFu, i);
     return MOE_OK;
+}
+
+moe_status moe_refresh_device(const uint32_t *hits, int32_t E, int32_t budget, int32_t *slot_table,
+                              int32_t n_slots, int32_t *promo, int32_t *status, moe_stream_t stream) {
+    CHECK_ARG(E >= 1 && E <= kMaxE, "E=%d outside [1, %d]", E, kMaxE);
+    CHECK_ARG(n_slots >= 0 && n_slots <= kMaxE, "n_slots=%d outside [0, %d]", n_slots, kMaxE);
+    CHECK_ARG(budget >= 0 && budget <= n_slots, "budget=%d outside [0, n_slots=%d]", budget, n_slots);
+    CHECK_ARG(hits && slot_table && promo && status, "moe_refresh_device: NULL pointer");
+    return cuda_status(launch_refresh_placement(hits, E, budget, slot_table, n_slots, promo, status,
+                                                (cudaStream_t)stream),
+                       "moe_refresh_device launch");
+}
+
+moe_status moe_promote_copies(const void *home, void *pool, uint64_t expert_bytes, const int32_t *promo,
+                              const int32_t *status, int32_t max_promo, moe_stream_t stream) {
+    CHECK_ARG(max_promo >= 0, "max_promo=%d is negative", max_promo);
+    if (max_promo == 0) return MOE_OK;
+    CHECK_ARG(home && pool && promo && status, "moe_promote_copies: NULL pointer");
+    CHECK_ARG(expert_bytes > 0 && expert_bytes % 16 == 0, "expert_bytes=%llu must be a positive multiple of 16",
+              (unsigned long long)expert_bytes);
+    CHECK_ARG(aligned16(home) && aligned16(pool), "home and pool must be 16-byte aligned");
+    return cuda_status(launch_promote_copies(home, pool, expert_bytes, promo, status, max_promo, (cudaStream_t)stream),
+                       "moe_promote_copies launch");
 }
 
 moe_status moe_copy_to_slots(const void *home, void *pool, uint64_t expert_bytes, const int32_t *experts,

@@ -172,3 +172,14 @@ def test_hits_window_matches_oracle():
     assert np.array_equal(moe.moe_hits_window(ring), oracle.hits_window(ring))
     with pytest.raises(moe.MoeError):
         moe.moe_hits_window(np.zeros((0, 128), np.uint32))
+
+
+def test_device_refresh_rejects_bad_arguments_before_launch():
+    L = moe._lib
+    assert L.moe_refresh_device(256, 128, 19, 256, 18, 256, 256, None) == moe.MOE_ERR_INVALID_ARG  # budget > slots
+    assert L.moe_refresh_device(256, 0, 0, 256, 0, 256, 256, None) == moe.MOE_ERR_INVALID_ARG      # E = 0
+    assert L.moe_refresh_device(256, 2000, 1, 256, 4, 256, 256, None) == moe.MOE_ERR_INVALID_ARG   # E > 1024
+    assert L.moe_refresh_device(None, 128, 1, 256, 4, 256, 256, None) == moe.MOE_ERR_INVALID_ARG   # NULL hits
+    assert L.moe_promote_copies(256, 256, 100, 256, 256, 4, None) == moe.MOE_ERR_INVALID_ARG       # size % 16
+    assert L.moe_promote_copies(264, 256, 256, 256, 256, 4, None) == moe.MOE_ERR_INVALID_ARG       # unaligned
+    assert L.moe_promote_copies(256, 256, 256, 256, 256, 0, None) == moe.MOE_OK                    # nothing to do

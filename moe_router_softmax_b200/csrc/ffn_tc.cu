@@ -114,6 +114,13 @@ struct TcParams {
 };
 
 // ---------------------------------------------------------------- PTX helpers
+// Programmatic dependent launch: the next kernel in the stream may be scheduled
+// as soon as every CTA of this one has signalled (here: at its start), and
+// griddepcontrol.wait blocks until the previous kernel has completed and its
+// writes are visible.  Both are no-ops for a kernel launched without the
+// programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -366,6 +373,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = PHASE == 1 ? p.L.I / 64 : (p.L.H + kBlockM - 1) / kBlockM;
+    // The next launch (phase 2 after phase 1, the combine after phase 2) may
+    // take over SMs as this grid's CTAs finish; it waits for this grid's
+    // results itself where it reads them.
+    pdl_launch_dependents();
     const int nk = (p.K + KS - 1) / KS;  // stages; the last may hold fewer atoms (p.K is a multiple of 64)
     auto atoms_at = [&](int kk) { return min(ATOMS, (p.K - kk * KS) / kBlockK); };
 
@@ -406,11 +417,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     const uint32_t tmem = s_tmem;
     const int n_act = s_items.n_act, total = s_items.total;
     const int n_block = s_items.n_block, b_slots = s_items.b_slots;
-    // A small route block leaves each MMA little work, and consecutive MMAs
-    // into one accumulator wait on each other's result; the four 16-wide K
-    // steps of a 64-wide atom then go to nacc separate partial accumulators
-    // (n_block columns apart inside the accumulator's kNMax columns), which the
-    // epilogue adds up.
+    // With a small route block the four 16-wide K steps of a 64-wide atom go
+    // to nacc separate partial accumulators (n_block columns apart inside the
+    // accumulator's kNMax columns), which the epilogue adds up, so that
+    // consecutive MMAs do not update the same small tile.
     const int nacc = n_block <= kNMax / 4 ? 4 : (n_block <= kNMax / 2 ? 2 : 1);
     const uint32_t b_atom_bytes = (uint32_t)n_block * 128;       // one 64-wide atom of a B slot
     const uint32_t b_slot_bytes = b_atom_bytes * ATOMS;
@@ -458,6 +468,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     } else if (warp == kWarpB) {
         // ------------------------------------------------ B producer: routes
         if (lane == 0) {
+            // the B operand (xs from k_gather_rows, or h from phase 1) is the one
+            // input the previous launch writes: wait for it here, while the
+            // other roles already stream weights
+            pdl_wait();
             int stage = 0;
             uint32_t phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
@@ -742,6 +756,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ sorted_route,
                               const int32_t *__restrict__ offsets, int E, int k, int H, int R,
                               uint16_t *__restrict__ xs) {
+    pdl_launch_dependents();
     const int per = H / 8;
     const int n_valid = __ldg(offsets + E);
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)R * per;
@@ -812,8 +827,18 @@ cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUten
         if (err != cudaSuccess) return err;
         attr[dev] = true;
     }
-    kern<<<n_sm, tc_threads<FMT>(), smem, s>>>(mh, mp, mb, p);
-    return cudaGetLastError();
+    // programmatic dependent launch: see pdl_launch_dependents / pdl_wait
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)n_sm);
+    cfg.blockDim = dim3((unsigned)tc_threads<FMT>());
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mh, mp, mb, p);
 }
 
 }  // namespace

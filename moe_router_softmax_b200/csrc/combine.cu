@@ -10,6 +10,10 @@ namespace {
 __global__ void __launch_bounds__(256) k_combine(const float *__restrict__ rows, const int32_t *__restrict__ route_pos,
                                                  const float *__restrict__ w, int T, int k, int H,
                                                  uint16_t *__restrict__ y) {
+    // programmatic dependent launch: wait for the previous kernel before
+    // touching memory, then let the next one be scheduled
+    pdl_wait();
+    pdl_launch_dependents();
     const int q4 = H >> 2;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (int64_t)T * q4) return;
@@ -37,8 +41,7 @@ cudaError_t launch_combine(const float *rows, const int32_t *route_pos, const fl
                            uint16_t *y, cudaStream_t s) {
     const int64_t n = (int64_t)T * (H / 4);
     if (n == 0) return cudaSuccess;
-    k_combine<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(rows, route_pos, w, T, k, H, y);
-    return cudaGetLastError();
+    return launch_pdl(k_combine, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, rows, route_pos, w, T, k, H, y);
 }
 
 }  // namespace moe

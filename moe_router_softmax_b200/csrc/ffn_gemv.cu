@@ -276,6 +276,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
     const int upi = groups * UPG;              // units per item
     const int tiles = (n_units + upi - 1) / upi;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // programmatic dependent launch: phase 1 waits for the permutation before
+    // anything else; phase 2 may be scheduled as soon as phase 1 has started
+    // (it waits for h itself, after requesting its weights into L2)
+    if (PHASE == 1) pdl_wait();
+    pdl_launch_dependents();
 
     // active experts and the prefix of their item counts (one warp)
     if (warp == 0) {
@@ -321,6 +326,23 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
         }
         a = lo;
     }
+    if (PHASE == 2 && threadIdx.x == 0) {
+        // launched while phase 1 may still run: request this CTA's weight rows
+        // into L2 first (they do not depend on phase 1), then wait for h
+        const uint64_t row_bytes = (uint64_t)nchunks * 16;
+        int pa = a;
+        for (int it = it_begin; it < it_end; ++it) {
+            while (s_base[pa + 1] <= it) ++pa;
+            const int tile = (it - s_base[pa]) % tiles;
+            const int r0 = tile * upi, r1 = min(n_units, r0 + upi);
+            const uint8_t *w = expert_blob(p.L, s_act[pa]) + p.L.off.q2 + (uint64_t)r0 * row_bytes;
+            for (uint64_t off = 0, n = (uint64_t)(r1 - r0) * row_bytes; off < n; off += 32768) {
+                const uint32_t bytes = (uint32_t)(n - off < 32768 ? n - off : 32768);
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(w + off), "r"(bytes) : "memory");
+            }
+        }
+    }
+    if (PHASE == 2) pdl_wait();
     const int li = lane & (lg - 1);
     const int gi = warp * (32 / lg) + lane / lg;
     int cur_key = -1;
@@ -381,8 +403,8 @@ cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
         cached_smem[dev] = (int)smem;
     }
     const int per_sm = cached_per_sm[dev];
-    kern<<<n_sm * per_sm, kThreads, smem, s>>>(p);
-    return cudaGetLastError();
+    // programmatic dependent launch (see the kernel's first lines)
+    return launch_pdl(kern, dim3((unsigned)(n_sm * per_sm)), dim3(kThreads), smem, s, p);
 }
 
 template <int FMT>

@@ -114,13 +114,6 @@ struct TcParams {
 };
 
 // ---------------------------------------------------------------- PTX helpers
-// Programmatic dependent launch: the next kernel in the stream may be scheduled
-// as soon as every CTA of this one has signalled (here: at its start), and
-// griddepcontrol.wait blocks until the previous kernel has completed and its
-// writes are visible.  Both are no-ops for a kernel launched without the
-// programmatic-serialization attribute.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -756,6 +749,9 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ sorted_route,
                               const int32_t *__restrict__ offsets, int E, int k, int H, int R,
                               uint16_t *__restrict__ xs) {
+    // programmatic dependent launch: wait for the previous kernel before
+    // touching memory, then let the next one be scheduled
+    pdl_wait();
     pdl_launch_dependents();
     const int per = H / 8;
     const int n_valid = __ldg(offsets + E);
@@ -827,18 +823,8 @@ cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUten
         if (err != cudaSuccess) return err;
         attr[dev] = true;
     }
-    // programmatic dependent launch: see pdl_launch_dependents / pdl_wait
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)n_sm);
-    cfg.blockDim = dim3((unsigned)tc_threads<FMT>());
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mh, mp, mb, p);
+    // programmatic dependent launch (the B producer waits for the previous launch)
+    return launch_pdl(kern, dim3((unsigned)n_sm), dim3((unsigned)tc_threads<FMT>()), smem, s, mh, mp, mb, p);
 }
 
 }  // namespace
@@ -877,8 +863,9 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     {
         const int64_t n = (int64_t)R * (H / 8);
         const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)n_sm * 8);
-        k_gather_rows<<<blocks, 256, 0, s>>>(x, sorted_route, offsets, L.E, k, H, R, xs);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        err = launch_pdl(k_gather_rows, dim3((unsigned)blocks), dim3(256), 0, s, x, sorted_route, offsets, L.E, k, H, R,
+                         xs);
+        if (err != cudaSuccess) return err;
     }
     // 2. tensor maps: weights (home and pool, as rows of one matrix), activations
     const bool bf = fmt == MOE_W_BF16;

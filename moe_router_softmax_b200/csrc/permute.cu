@@ -29,6 +29,10 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t *__restrict__ id
     int *s_scan = smem + kWarps * E;    // [1024] scan scratch
     __shared__ int s_total;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // programmatic dependent launch: wait for the previous kernel before
+    // touching memory, then let the next one be scheduled
+    pdl_wait();
+    pdl_launch_dependents();
 
     for (int i = tid; i < kWarps * E; i += blockDim.x) s_w[i] = 0;
     __syncthreads();
@@ -137,8 +141,8 @@ cudaError_t launch_permute(const int32_t *ids, int R, int E, int32_t *counts, in
         if (err != cudaSuccess) return err;
         cached[dev] = smem;
     }
-    k_permute<<<1, 1024, smem, s>>>(ids, R, E, counts, offsets, sorted_route, route_pos, hits);
-    return cudaGetLastError();
+    return launch_pdl(k_permute, dim3(1), dim3(1024), smem, s, ids, R, E, counts, offsets, sorted_route, route_pos,
+                      hits);
 }
 
 cudaError_t launch_expert_hits(const int32_t *ids, int64_t n, int E, uint32_t *hits, cudaStream_t s) {

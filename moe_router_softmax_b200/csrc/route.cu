@@ -138,6 +138,10 @@ __device__ __forceinline__ void route_token_warp(Load load, int E, int k, int32_
 template <int VPL>
 __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ logits, int T, int E, int k,
                                                     int32_t *__restrict__ ids, float *__restrict__ w) {
+    // programmatic dependent launch: wait for the previous kernel before
+    // touching memory, then let the next one be scheduled
+    pdl_wait();
+    pdl_launch_dependents();
     const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
     if (t >= T) return;
     const float *l = logits + (size_t)t * E;
@@ -363,13 +367,12 @@ cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t 
     if (T == 0) return cudaSuccess;
     const int vpl = (E + 31) / 32;
     dim3 block(256), grid((unsigned)((T + 7) / 8));
-    if (vpl <= 1) k_route_topk<1><<<grid, block, 0, s>>>(logits, T, E, k, ids, w);
-    else if (vpl <= 2) k_route_topk<2><<<grid, block, 0, s>>>(logits, T, E, k, ids, w);
-    else if (vpl <= 4) k_route_topk<4><<<grid, block, 0, s>>>(logits, T, E, k, ids, w);
-    else if (vpl <= 8) k_route_topk<8><<<grid, block, 0, s>>>(logits, T, E, k, ids, w);
-    else if (vpl <= 16) k_route_topk<16><<<grid, block, 0, s>>>(logits, T, E, k, ids, w);
-    else k_route_topk<32><<<grid, block, 0, s>>>(logits, T, E, k, ids, w);
-    return cudaGetLastError();
+    if (vpl <= 1) return launch_pdl(k_route_topk<1>, grid, block, 0, s, logits, T, E, k, ids, w);
+    if (vpl <= 2) return launch_pdl(k_route_topk<2>, grid, block, 0, s, logits, T, E, k, ids, w);
+    if (vpl <= 4) return launch_pdl(k_route_topk<4>, grid, block, 0, s, logits, T, E, k, ids, w);
+    if (vpl <= 8) return launch_pdl(k_route_topk<8>, grid, block, 0, s, logits, T, E, k, ids, w);
+    if (vpl <= 16) return launch_pdl(k_route_topk<16>, grid, block, 0, s, logits, T, E, k, ids, w);
+    return launch_pdl(k_route_topk<32>, grid, block, 0, s, logits, T, E, k, ids, w);
 }
 
 }  // namespace moe

@@ -48,9 +48,6 @@ import numpy as np  # noqa: E402
 NCU_TRAFFIC_BYTES = {
     # profiles/ffn_gemv_bf16_T64.md: phase 1 1.0059 GB + 4.04 MB, phase 2 0.5027 GB + 5.28 MB
     ("decode-bf16", 64, "gemv"): 1.5180e9,
-    # profiles/ffn_tc_bf16_decode_T64.md: phase 1 1.002597 GB + 4.92 MB, phase 2 0.500371 GB + 8.40 MB
-    ("decode-bf16", 64, "auto"): 1.5163e9,
-    ("decode-bf16", 64, "tc"): 1.5163e9,
     # profiles/ffn_tc_int4_decode_T64.md: 268.4 + 3.96 + 133.6 + 5.43 MB
     ("int4-decode", 64, "auto"): 4.1132e8,
     ("int4-decode", 64, "tc"): 4.1132e8,

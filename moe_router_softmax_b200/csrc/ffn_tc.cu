@@ -71,15 +71,15 @@ constexpr int kXPitch = 17;                               // exchange row pitch 
 // For int8 / int4 the A ring lives in tensor memory instead (kASmem = 0): the
 // dequant warps store the bf16 tiles with tcgen05.st and the MMAs read A from
 // TMEM, so the expanded weights never pass through shared memory.
-// A stage covers kKS of K (kKS / 64 swizzle atoms): one 64-wide atom for bf16;
-// two for the int formats, so that the single MMA-issuing thread pays one
-// barrier wait and one pair of commits per 8 MMAs instead of per 4 (each
-// tcgen05 instruction and each barrier wait costs that thread tens of
-// nanoseconds, which bounds a decode batch's small MMAs).
+// A stage covers kKS = 128 of K (two 64-wide swizzle atoms), so that the
+// single MMA-issuing thread pays one round of barrier waits and commits per 8
+// MMAs instead of per 4 (each tcgen05 instruction and each barrier wait costs
+// that thread tens of nanoseconds, which otherwise bounds a decode batch's
+// small MMAs).
 // kSub stages share one raw stage of kRawRowBytes per row (kSubBytes each).
 template <int FMT> struct TcFmt;
 template <> struct TcFmt<MOE_W_BF16> {
-    static constexpr int kKS = 64, kSub = 1, kSubBytes = 0, kAStages = 8, kASmem = 1, kRawStages = 0;
+    static constexpr int kKS = 128, kSub = 1, kSubBytes = 0, kAStages = 4, kASmem = 1, kRawStages = 0;
     static constexpr int kBRegion = 64 * 1024, kTmemCols = kAccCols;
 };
 template <> struct TcFmt<MOE_W_INT8> {
@@ -343,7 +343,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     // 1024-byte aligned carve-up: A ring | B region | raw ring | exchange | barriers
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
-    uint8_t *sB = sA + (TcFmt<FMT>::kASmem ? SA * kATileBytes : 0);
+    uint8_t *sB = sA + (TcFmt<FMT>::kASmem ? SA * ATOMS * kATileBytes : 0);
     uint8_t *sRaw = sB + TcFmt<FMT>::kBRegion;
     float *sX = reinterpret_cast<float *>(sRaw + SR * RAW);       // [2][64][kXPitch] gate/up exchange
     uint64_t *bars = reinterpret_cast<uint64_t *>(sX + 2 * 64 * kXPitch);
@@ -447,11 +447,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     }
                 } else {
                     for (int kk = 0; kk < nk; ++kk) {
+                        const int na = atoms_at(kk);
                         if (!mbar_wait(&a_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
-                        mbar_arrive_expect_tx(&a_full[stage], kATileBytes);
-                        uint8_t *dst = sA + stage * kATileBytes;
-                        tma_load_2d(dst, ma, &a_full[stage], kk * kBlockK, ya0);
-                        tma_load_2d(dst + kATileBytes / 2, ma, &a_full[stage], kk * kBlockK, ya1);
+                        mbar_arrive_expect_tx(&a_full[stage], (uint32_t)na * kATileBytes);
+                        for (int a = 0; a < na; ++a) {
+                            uint8_t *dst = sA + (stage * ATOMS + a) * kATileBytes;
+                            tma_load_2d(dst, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya0);
+                            tma_load_2d(dst + kATileBytes / 2, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya1);
+                        }
                         if (++stage == SA) { stage = 0; phase ^= 1; }
                     }
                 }
@@ -519,11 +522,16 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                                                (kk | a | (j / nacc)) != 0);
                         }
                     } else {
-                        const uint32_t a0 = smem_u32(sA + sa * kATileBytes);
+                        const uint32_t a0 = smem_u32(sA + sa * ATOMS * kATileBytes);
+                        const int na = atoms_at(kk);
+                        for (int a = 0; a < na; ++a) {
 #pragma unroll
-                        for (int j = 0; j < kBlockK / 16; ++j)
-                            tc_mma_bf16(d + (uint32_t)((j % nacc) * n_block), sw128_desc(a0 + 32 * j),
-                                        sw128_desc(b0 + 32 * j), idesc, (kk | (j / nacc)) != 0);
+                            for (int j = 0; j < kBlockK / 16; ++j)
+                                tc_mma_bf16(d + (uint32_t)((j % nacc) * n_block),
+                                            sw128_desc(a0 + a * kATileBytes + 32 * j),
+                                            sw128_desc(b0 + a * b_atom_bytes + 32 * j), idesc,
+                                            (kk | a | (j / nacc)) != 0);
+                        }
                     }
                     tc_commit(&a_empty[sa]);
                     tc_commit(&b_empty[sb]);
@@ -798,7 +806,8 @@ bool encode_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int ele
 
 template <int FMT>
 constexpr size_t smem_bytes() {
-    return 1024 + (size_t)(TcFmt<FMT>::kASmem ? TcFmt<FMT>::kAStages : 0) * kATileBytes + TcFmt<FMT>::kBRegion +
+    return 1024 + (size_t)(TcFmt<FMT>::kASmem ? TcFmt<FMT>::kAStages * (TcFmt<FMT>::kKS / kBlockK) : 0) * kATileBytes +
+           TcFmt<FMT>::kBRegion +
            (size_t)TcFmt<FMT>::kRawStages * kRawBytes<FMT>() + 2 * 64 * kXPitch * 4 +
            (size_t)(2 * TcFmt<FMT>::kAStages + 2 * kMaxBSlots + 2 * kAccBufs + 4 + 2 * TcFmt<FMT>::kRawStages) * 8;
 }

@@ -48,6 +48,9 @@ import numpy as np  # noqa: E402
 NCU_TRAFFIC_BYTES = {
     # profiles/ffn_gemv_bf16_T64.md: phase 1 1.0059 GB + 4.04 MB, phase 2 0.5027 GB + 5.28 MB
     ("decode-bf16", 64, "gemv"): 1.5180e9,
+    # profiles/ffn_tc_bf16_decode_T64.md: phase 1 1.002456 GB + 4.92 MB, phase 2 0.500373 GB + 8.66 MB
+    ("decode-bf16", 64, "auto"): 1.5164e9,
+    ("decode-bf16", 64, "tc"): 1.5164e9,
     # profiles/ffn_tc_int4_decode_T64.md: 268.4 + 3.96 + 133.6 + 5.43 MB
     ("int4-decode", 64, "auto"): 4.1132e8,
     ("int4-decode", 64, "tc"): 4.1132e8,
@@ -313,33 +316,55 @@ def time_steps(torch, runner, steps, warmup, dist):
 
 
 def time_e2e(torch, moe, layers, batches, T, k, steps, warmup, dev):
-    """End to end through moe_layer_forward with host buffers: H2D of logits and x
-    from pinned memory, the layer, D2H of y, every step, on one stream."""
+    """End to end through moe_layer_forward with host buffers: every step copies
+    its logits and x from pinned host memory and reads y back to pinned host
+    memory.  As a serving loop would, the copies run on their own streams and
+    overlap the layer of the neighbouring step (double-buffered device buffers,
+    ordered by events): H2D of step i+1 and D2H of step i-1 while step i runs."""
     E, H = layers[0].E, layers[0].H
     host_lg = [torch.from_numpy(b[0]).pin_memory() for b in batches]
     host_x = [torch.from_numpy(b[1].view(np.int16)).pin_memory() for b in batches]
-    host_y = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    d_lg = torch.empty((T, E), dtype=torch.float32, device=dev)
-    d_x = torch.empty((T, H), dtype=torch.int16, device=dev)
-    d_y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    host_y = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(2)]
+    d_lg = [torch.empty((T, E), dtype=torch.float32, device=dev) for _ in range(2)]
+    d_x = [torch.empty((T, H), dtype=torch.int16, device=dev) for _ in range(2)]
+    d_y = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     ws = torch.empty(moe.moe_layer_forward_workspace(layers[0], T, k), dtype=torch.uint8, device=dev)
+    comp = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]   # the layer using buffer b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # y of buffer b read back
+    for b in range(2):
+        ev_done[b].record(comp)
+        ev_out[b].record(comp)
 
     def one(i):
-        b = i % len(batches)
-        d_lg.copy_(host_lg[b], non_blocking=True)
-        d_x.copy_(host_x[b], non_blocking=True)
-        moe.moe_layer_forward(layers[i % len(layers)], d_lg, d_x.view(torch.bfloat16), k, y=d_y, ws=ws)
-        host_y.copy_(d_y.view(torch.int16), non_blocking=True)
+        b, src = i & 1, i % len(batches)
+        s_in.wait_event(ev_done[b])                    # the layer two steps back is done with these inputs
+        with torch.cuda.stream(s_in):
+            d_lg[b].copy_(host_lg[src], non_blocking=True)
+            d_x[b].copy_(host_x[src], non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])                     # y of two steps back has been read
+        moe.moe_layer_forward(layers[i % len(layers)], d_lg[b], d_x[b].view(torch.bfloat16), k, y=d_y[b], ws=ws)
+        ev_done[b].record(comp)
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            host_y[b].copy_(d_y[b].view(torch.int16), non_blocking=True)
+            ev_out[b].record(s_out)
 
     for i in range(warmup):
         one(i)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
+    t0.record(comp)
     for i in range(steps):
         one(warmup + i)
-    t1.record()
+    comp.wait_stream(s_in)
+    comp.wait_stream(s_out)
+    t1.record(comp)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
     return ms, T * E * 4 + T * H * 2, T * H * 2

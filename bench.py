@@ -51,12 +51,6 @@ NCU_TRAFFIC_BYTES = {
     # profiles/ffn_tc_bf16_decode_T64.md: phase 1 1.002456 GB + 4.92 MB, phase 2 0.500373 GB + 8.66 MB
     ("decode-bf16", 64, "auto"): 1.5164e9,
     ("decode-bf16", 64, "tc"): 1.5164e9,
-    # profiles/ffn_tc_int4_decode_T64.md: 268.4 + 3.96 + 133.6 + 5.43 MB
-    ("int4-decode", 64, "auto"): 4.1132e8,
-    ("int4-decode", 64, "tc"): 4.1132e8,
-    # profiles/ffn_tc_int4_prefill_T1024.md: 315.8 + 10.9 + 146.5 + 53.6 MB
-    ("int4-prefill", 1024, "auto"): 5.2682e8,
-    ("int4-prefill", 1024, "tc"): 5.2682e8,
 }
 
 CONFIGS = {

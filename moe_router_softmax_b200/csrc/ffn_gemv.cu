@@ -258,7 +258,12 @@ __device__ __forceinline__ void run_item(const FfnParams &p, const float *xs, co
     }
 }
 
-template <int FMT, int PHASE, int RWP, int U>
+// NTMAX = 1: the one-token kernel (every expert has one route): only the
+// single-route item code is instantiated, which leaves registers for more
+// chunks of each row in flight (bf16: U = 11, a lane's whole share of a row at
+// H = 2816 / I = 704); an expert with more routes is still handled, one route
+// at a time.
+template <int FMT, int PHASE, int RWP, int U, int NTMAX>
 __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
     constexpr int UPG = PHASE == 1 ? RWP / 2 : RWP;
     constexpr int EC = Fmt<FMT>::kElems;
@@ -363,7 +368,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
         }
         const uint8_t *blob = expert_blob(p.L, e);
         const int u0 = tile * upi + gi * UPG;
-        if (nt > 4) run_item<FMT, PHASE, RWP, U, 8>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
+        if (NTMAX == 1) {
+            // route t0's activations are sub-planes t0*SP .. of xs
+            constexpr int SP = Fmt<FMT>::kElems / 4;
+            for (int t0 = 0; t0 < nt; ++t0)
+                run_item<FMT, PHASE, RWP, U, 1>(p, xs + (size_t)t0 * SP * nchunks * 4, blob, u0, row0 + t0, 1, K,
+                                                 nchunks, li, lg);
+        } else if (nt > 4) run_item<FMT, PHASE, RWP, U, 8>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
         else if (nt > 2) run_item<FMT, PHASE, RWP, U, 4>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
         else if (nt > 1) run_item<FMT, PHASE, RWP, U, 2>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
         else run_item<FMT, PHASE, RWP, U, 1>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
@@ -378,14 +389,14 @@ int pick_lg(int nchunks) {
     return lg;
 }
 
-template <int FMT, int PHASE, int RWP, int U>
+template <int FMT, int PHASE, int RWP, int U, int NTMAX>
 cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
     FfnParams p = p0;
     const int K = PHASE == 1 ? p.L.H : p.L.I;
     const int nchunks = K / Fmt<FMT>::kElems;
     p.lg = pick_lg(nchunks);
     const size_t smem = (size_t)kNTM * K * sizeof(float);
-    auto kern = k_ffn_gemv<FMT, PHASE, RWP, U>;
+    auto kern = k_ffn_gemv<FMT, PHASE, RWP, U, NTMAX>;
     // one-time set-up per device and shared-memory size (kept out of stream
     // capture: after the first call a launch is the only API call made here)
     static int cached_smem[kMaxDevices] = {}, cached_per_sm[kMaxDevices] = {};
@@ -413,9 +424,17 @@ cudaError_t launch_fmt(const FfnParams &p, int n_sm, cudaStream_t s) {
     // of each row in flight, so a lane keeps 8 x 16 bytes of weights in flight
     constexpr int RWP = 2;
     constexpr int U = 8 / RWP;
-    cudaError_t err = launch_phase<FMT, 1, RWP, U>(p, n_sm, s);
+    if (p.T == 1) {  // one token: at most one route per expert (unless ids repeat)
+        // chunks per row in flight: all 11 of a lane's share for bf16; 6 for the
+        // int formats, whose expansion needs the registers
+        constexpr int U1 = FMT == MOE_W_BF16 ? 11 : 6;
+        cudaError_t err = launch_phase<FMT, 1, RWP, U1, 1>(p, n_sm, s);
+        if (err != cudaSuccess) return err;
+        return launch_phase<FMT, 2, RWP, U1, 1>(p, n_sm, s);
+    }
+    cudaError_t err = launch_phase<FMT, 1, RWP, U, kNTM>(p, n_sm, s);
     if (err != cudaSuccess) return err;
-    return launch_phase<FMT, 2, RWP, U>(p, n_sm, s);
+    return launch_phase<FMT, 2, RWP, U, kNTM>(p, n_sm, s);
 }
 
 }  // namespace

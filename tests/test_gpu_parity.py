@@ -445,3 +445,26 @@ def test_layer_with_min_weight_matches_oracle():
     oy = oracle.combine(oracle.ffn_routes(OL, x, oi), oi, ow, E)
     assert (oi < 0).any()
     assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_one_token_with_repeated_ids(fmt):
+    """The one-token GEMV kernel assumes one route per expert but must still be
+    right when a caller's ids repeat an expert within the token (here experts 2
+    and 5 twice each, and one dropped id)."""
+    E, H, I, k = 8, 256, 128, 6
+    w13, w2 = syn.expert_weights(E, H, I, seed=12)
+    L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
+    x = syn.activations(1, H, seed=12)
+    ids = np.array([[2, 5, 2, 7, 5, -1]], np.int32)
+    w = np.array([[0.3, 0.2, 0.1, 0.15, 0.15, 0.1]], np.float32)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    counts, offsets, sr, rp = moe.moe_permute(torch.from_numpy(ids).to(DEV), E)
+    rows = moe.moe_grouped_ffn(L, xd, k, counts, offsets, sr, path=moe.MOE_FFN_GEMV)
+    y = moe.moe_combine(rows, rp, torch.from_numpy(w).to(DEV))
+    OL = oracle_layer_for(fmt, w13, w2)
+    orows = oracle.ffn_routes(OL, x, ids)
+    valid = (ids.ravel() >= 0)
+    got = rows.cpu().numpy()[rp.cpu().numpy().ravel()[valid]]
+    assert rel_err(got, orows[valid]) <= FFN_TOL
+    assert rel_err(bf16_dev_to_f64(y), oracle.combine(orows, ids, w, E)) <= FFN_TOL

@@ -121,3 +121,10 @@ def test_router_topk_k_equals_e_is_a_softmax_and_t0_is_a_noop():
     xd = torch.empty((0, H), dtype=torch.bfloat16, device=DEV)
     ids0, w0 = moe.moe_router_topk(xd, torch.from_numpy(wr).to(DEV), 4)
     assert ids0.shape == (0, 4)
+
+
+def test_no_kernel_recorded_a_device_error():
+    """The tensor-core kernels record the first failed index check or timed-out
+    wait in a device word; after every GPU test so far it must still be clear."""
+    code, info = moe.moe_take_device_errors()
+    assert code == 0, (hex(code), info)

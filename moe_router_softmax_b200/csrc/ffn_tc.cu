@@ -53,7 +53,6 @@ constexpr int kAccBufs = 2;
 constexpr int kAccCols = kNMax * kAccBufs;   // TMEM columns of the accumulators
 constexpr int kEpiWarps = 4;
 constexpr int kDeqWarps = 8;          // per group: two threads per tile row, half a row each
-constexpr int kDeqGroups = 2;         // groups take alternate stages, so two stages expand at once
 constexpr uint32_t kATileBytes = kBlockM * kBlockK * 2;   // 16 KB
 constexpr int kMaxBSlots = 32;
 constexpr int kRawRowBytes = 128;     // per raw stage row
@@ -89,6 +88,22 @@ template <> struct TcFmt<MOE_W_INT8> {
 template <> struct TcFmt<MOE_W_INT4> {
     static constexpr int kKS = 128, kSub = 2, kSubBytes = 64, kAStages = 4, kASmem = 0, kRawStages = 6;
     static constexpr int kBRegion = 96 * 1024, kTmemCols = 512;
+};
+
+// Launch configuration.  CFG 0: one CTA per SM (above).  CFG 1, for int8/int4
+// decode batches (route blocks <= 64): two CTAs per SM, each with half the
+// accumulator width, one dequant group, shallower rings and half the tensor
+// memory -- two MMA-issuing threads per SM, which is what bounds the int formats
+// at decode (measured 16-19% faster at 64 tokens; the prefill case needs the
+// wider accumulators and stays on CFG 0).
+template <int FMT, int CFG> struct TcCfg : TcFmt<FMT> {
+    static constexpr int kNMax = 128, kDeqGroups = 2, kMinBlocks = 1;
+    static constexpr int kAccCols = kNMax * kAccBufs;
+};
+template <int FMT> struct TcCfg<FMT, 1> : TcFmt<FMT> {
+    static constexpr int kNMax = 64, kDeqGroups = 1, kMinBlocks = 2;
+    static constexpr int kAccCols = kNMax * kAccBufs;
+    static constexpr int kAStages = 2, kRawStages = 3, kBRegion = 32 * 1024, kTmemCols = 256;
 };
 
 // First problem a tensor-core kernel recorded (0 = none): 0x1000 | role for
@@ -324,27 +339,30 @@ __host__ __device__ constexpr int kRawBytes() { return FMT == MOE_W_BF16 ? 0 : k
 constexpr int kWarpB = 2 + kEpiWarps;
 constexpr int kWarpDeq0 = kWarpB + 1;
 
-template <int FMT>
-__host__ __device__ constexpr int tc_threads() { return 32 * (kWarpDeq0 + (FMT == MOE_W_BF16 ? 0 : kDeqGroups * kDeqWarps)); }
+template <int FMT, int CFG>
+__host__ __device__ constexpr int tc_threads() {
+    return 32 * (kWarpDeq0 + (FMT == MOE_W_BF16 ? 0 : TcCfg<FMT, CFG>::kDeqGroups * kDeqWarps));
+}
 
-template <int FMT, int PHASE>
-__global__ void __launch_bounds__(tc_threads<FMT>(), 1)
+template <int FMT, int PHASE, int CFG>
+__global__ void __launch_bounds__(tc_threads<FMT, CFG>(), TcCfg<FMT, CFG>::kMinBlocks)
 k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ CUtensorMap map_pool,
          const __grid_constant__ CUtensorMap map_b, const TcParams p) {
-    constexpr int SA = TcFmt<FMT>::kAStages;
-    constexpr int SR = TcFmt<FMT>::kRawStages;
+    using C = TcCfg<FMT, CFG>;
+    constexpr int SA = C::kAStages;
+    constexpr int SR = C::kRawStages;
     constexpr int RAW = kRawBytes<FMT>();
-    constexpr int SUB = TcFmt<FMT>::kSub;
+    constexpr int SUB = C::kSub;
     constexpr bool kDeq = FMT != MOE_W_BF16;
-    constexpr int KS = TcFmt<FMT>::kKS, ATOMS = KS / kBlockK;
+    constexpr int KS = C::kKS, ATOMS = KS / kBlockK;
     constexpr int A_COLS = KS / 2;  // TMEM columns of one A stage (int formats: bf16 pairs)
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned carve-up: A ring | B region | raw ring | exchange | barriers
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
-    uint8_t *sB = sA + (TcFmt<FMT>::kASmem ? SA * ATOMS * kATileBytes : 0);
-    uint8_t *sRaw = sB + TcFmt<FMT>::kBRegion;
+    uint8_t *sB = sA + (C::kASmem ? SA * ATOMS * kATileBytes : 0);
+    uint8_t *sRaw = sB + C::kBRegion;
     float *sX = reinterpret_cast<float *>(sRaw + SR * RAW);       // [2][64][kXPitch] gate/up exchange
     uint64_t *bars = reinterpret_cast<uint64_t *>(sX + 2 * 64 * kXPitch);
     uint64_t *a_full = bars;                       // A tile ready (TMA bytes, or the dequant warps)
@@ -392,18 +410,18 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         }
         for (int r = 0; r < SR; ++r) {
             mbar_init(&r_full[r], 1);
-            mbar_init(&r_empty[r], kDeqGroups * kDeqWarps);
+            mbar_init(&r_empty[r], C::kDeqGroups * kDeqWarps);
         }
         s_abort = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                     "r"(TcFmt<FMT>::kTmemCols)
+                     "r"(C::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    build_items(p, m_tiles, TcFmt<FMT>::kBRegion, ATOMS, s_act, s_base, &s_items);
+    build_items(p, m_tiles, C::kBRegion, ATOMS, s_act, s_base, &s_items);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -412,9 +430,9 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     const int n_block = s_items.n_block, b_slots = s_items.b_slots;
     // With a small route block the four 16-wide K steps of a 64-wide atom go
     // to nacc separate partial accumulators (n_block columns apart inside the
-    // accumulator's kNMax columns), which the epilogue adds up, so that
+    // accumulator's C::kNMax columns), which the epilogue adds up, so that
     // consecutive MMAs do not update the same small tile.
-    const int nacc = n_block <= kNMax / 4 ? 4 : (n_block <= kNMax / 2 ? 2 : 1);
+    const int nacc = n_block <= C::kNMax / 4 ? 4 : (n_block <= C::kNMax / 2 ? 2 : 1);
     const uint32_t b_atom_bytes = (uint32_t)n_block * 128;       // one 64-wide atom of a B slot
     const uint32_t b_slot_bytes = b_atom_bytes * ATOMS;
 
@@ -498,7 +516,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                 const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, &s_abort)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)(acc * kNMax);
+                const uint32_t d = tmem + (uint32_t)(acc * C::kNMax);
                 const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(it.n_mma >> 3) << 17) |
                                        ((uint32_t)(kBlockM >> 4) << 24);
                 bool ok = true;
@@ -510,9 +528,9 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     tc_fence_after();
                     const uint32_t b0 = smem_u32(sB + sb * b_slot_bytes);
                     if (kDeq) {
-                        // A stage sa: TMEM columns kAccCols + A_COLS sa .., 32 per atom,
+                        // A stage sa: TMEM columns C::kAccCols + A_COLS sa .., 32 per atom,
                         // 8 per 16-wide K step
-                        const uint32_t a_t = tmem + (uint32_t)(kAccCols + sa * A_COLS);
+                        const uint32_t a_t = tmem + (uint32_t)(C::kAccCols + sa * A_COLS);
                         const int na = atoms_at(kk);
                         for (int a = 0; a < na; ++a) {
 #pragma unroll
@@ -555,7 +573,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
             if (!mbar_wait(&tfull[acc], acc_phase, &s_abort)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kNMax);
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kNMax);
             const uint8_t *blob = expert_blob(p.L, it.e);
             float scale = 1.0f;
             if (FMT == MOE_W_INT8) {
@@ -635,7 +653,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         // lane quadrant; the eight warps of a group cover each quadrant twice
         // (both atoms of its rows).  The first warp of the group also waits for
         // the stage's B slot, so a completed a_full means A and B are both ready.
-        const int dw = warp - kWarpDeq0;              // 0 .. kDeqGroups*kDeqWarps-1
+        const int dw = warp - kWarpDeq0;              // 0 .. C::kDeqGroups*kDeqWarps-1
         const int group = dw / kDeqWarps;
         const int quad = warp & 3;
         const int r = quad * 32 + lane, hf = (dw % kDeqWarps) / 4;
@@ -654,7 +672,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             for (int kk = 0; kk < nk; ++kk, ++step) {
                 const int sub = kk % SUB;
                 const bool raw_last = sub == SUB - 1 || kk == nk - 1;  // last stage of this raw stage
-                if ((int)(step % kDeqGroups) != group) {   // the other group's stage
+                if ((int)(step % C::kDeqGroups) != group) {   // the other group's stage
                     if (++stage == SA) { stage = 0; phase ^= 1; }
                     if (++bstage == b_slots) { bstage = 0; bphase ^= 1; }
                     if (raw_last) {
@@ -678,7 +696,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     // spread over all banks
                     const uint8_t *src = sRaw + rstage * RAW + r * kRawRowBytes;
                     // first 16-byte chunk of this thread's atom: 64 codes = 32 (int4) / 64 (int8) bytes
-                    const int cj0 = sub * (TcFmt<FMT>::kSubBytes / 16) + hf * (FMT == MOE_W_INT4 ? 2 : 4);
+                    const int cj0 = sub * (C::kSubBytes / 16) + hf * (FMT == MOE_W_INT4 ? 2 : 4);
                     uint32_t o[32];  // bf16 pairs (weights 64 hf + 2j, +1 in the low, high half)
                     if (FMT == MOE_W_INT4) {
                         // bf16 128 + n (n in the low mantissa bits of 128.0 = 0x4300),
@@ -723,7 +741,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                             }
                         }
                     }
-                    const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(kAccCols + stage * A_COLS + 32 * hf);
+                    const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(C::kAccCols + stage * A_COLS + 32 * hf);
                     tmem_st16(ta, o);
                     tmem_st16(ta + 16, o + 16);
                     tmem_st_wait();
@@ -747,7 +765,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TcFmt<FMT>::kTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
                      : "memory");
     }
 }
@@ -804,24 +822,30 @@ bool encode_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int ele
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT>
+template <int FMT, int CFG>
 constexpr size_t smem_bytes() {
-    return 1024 + (size_t)(TcFmt<FMT>::kASmem ? TcFmt<FMT>::kAStages * (TcFmt<FMT>::kKS / kBlockK) : 0) * kATileBytes +
-           TcFmt<FMT>::kBRegion +
-           (size_t)TcFmt<FMT>::kRawStages * kRawBytes<FMT>() + 2 * 64 * kXPitch * 4 +
-           (size_t)(2 * TcFmt<FMT>::kAStages + 2 * kMaxBSlots + 2 * kAccBufs + 4 + 2 * TcFmt<FMT>::kRawStages) * 8;
+    using C = TcCfg<FMT, CFG>;
+    return 1024 + (size_t)(C::kASmem ? C::kAStages * (C::kKS / kBlockK) : 0) * kATileBytes + C::kBRegion +
+           (size_t)C::kRawStages * kRawBytes<FMT>() + 2 * 64 * kXPitch * 4 +
+           (size_t)(2 * C::kAStages + 2 * kMaxBSlots + 2 * kAccBufs + 4 + 2 * C::kRawStages) * 8;
 }
 // dynamic + static shared memory (s_act, s_base, ...: 9216 bytes) within the
-// 232448-byte per-block limit
-static_assert(smem_bytes<MOE_W_BF16>() + 9216 <= 232448, "bf16 tensor-core kernel exceeds shared memory");
-static_assert(smem_bytes<MOE_W_INT8>() + 9216 <= 232448, "int8 tensor-core kernel exceeds shared memory");
-static_assert(smem_bytes<MOE_W_INT4>() + 9216 <= 232448, "int4 tensor-core kernel exceeds shared memory");
+// 232448-byte per-block limit; two CTAs per SM (with 1 KB reserved by the
+// system each) within the SM's 233472 bytes
+static_assert(smem_bytes<MOE_W_BF16, 0>() + 9216 <= 232448, "bf16 tensor-core kernel exceeds shared memory");
+static_assert(smem_bytes<MOE_W_INT8, 0>() + 9216 <= 232448, "int8 tensor-core kernel exceeds shared memory");
+static_assert(smem_bytes<MOE_W_INT4, 0>() + 9216 <= 232448, "int4 tensor-core kernel exceeds shared memory");
+static_assert(2 * (smem_bytes<MOE_W_INT8, 1>() + 9216 + 1024) <= 233472, "int8 two-CTA config exceeds shared memory");
+static_assert(2 * (smem_bytes<MOE_W_INT4, 1>() + 9216 + 1024) <= 233472, "int4 two-CTA config exceeds shared memory");
+static_assert(2 * TcCfg<MOE_W_INT4, 1>::kTmemCols <= 512 && TcCfg<MOE_W_INT4, 1>::kAccCols +
+                  TcCfg<MOE_W_INT4, 1>::kAStages * TcCfg<MOE_W_INT4, 1>::kKS / 2 <= TcCfg<MOE_W_INT4, 1>::kTmemCols,
+              "two-CTA config exceeds tensor memory");
 
-template <int FMT, int PHASE>
+template <int FMT, int PHASE, int CFG>
 cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUtensorMap &mb, const TcParams &p,
                        int n_sm, cudaStream_t s) {
-    auto kern = k_ffn_tc<FMT, PHASE>;
-    const size_t smem = smem_bytes<FMT>();
+    auto kern = k_ffn_tc<FMT, PHASE, CFG>;
+    const size_t smem = smem_bytes<FMT, CFG>();
     static bool attr[kMaxDevices] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -833,7 +857,8 @@ cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUten
         attr[dev] = true;
     }
     // programmatic dependent launch (the B producer waits for the previous launch)
-    return launch_pdl(kern, dim3((unsigned)n_sm), dim3((unsigned)tc_threads<FMT>()), smem, s, mh, mp, mb, p);
+    return launch_pdl(kern, dim3((unsigned)(n_sm * TcCfg<FMT, CFG>::kMinBlocks)), dim3((unsigned)tc_threads<FMT, CFG>()),
+                      smem, s, mh, mp, mb, p);
 }
 
 }  // namespace
@@ -909,7 +934,9 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     // rows hold all of an expert's routes in one block (smaller blocks would
     // re-stream the weights of busier experts); the kernels shrink it to the
     // busiest expert's count
-    p.n_block = std::min(kNMax, (std::max(T, 1) + 15) / 16 * 16);
+    // int formats with a decode batch (every route block <= 64) run two CTAs per SM
+    const bool two = !bf && T <= TcCfg<MOE_W_INT4, 1>::kNMax;
+    p.n_block = std::min(two ? TcCfg<MOE_W_INT4, 1>::kNMax : kNMax, (std::max(T, 1) + 15) / 16 * 16);
     p.h = h;
     p.rows = rows;
     // every pointer the kernels write through must be set (host-side guard)
@@ -922,9 +949,11 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
         p.n_units = 2 * I;
         p.rows_per_blob = (int64_t)(L.stride / rb);
         p.q_row_off = (int64_t)(L.off.q13 / rb);
-        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 1>(mh1, mp1, mb1, p, n_sm, s);
-        else if (fmt == MOE_W_INT8) err = launch_one<MOE_W_INT8, 1>(mh1, mp1, mb1, p, n_sm, s);
-        else err = launch_one<MOE_W_INT4, 1>(mh1, mp1, mb1, p, n_sm, s);
+        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 1, 0>(mh1, mp1, mb1, p, n_sm, s);
+        else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 1, 1>(mh1, mp1, mb1, p, n_sm, s)
+                                              : launch_one<MOE_W_INT8, 1, 0>(mh1, mp1, mb1, p, n_sm, s);
+        else err = two ? launch_one<MOE_W_INT4, 1, 1>(mh1, mp1, mb1, p, n_sm, s)
+                       : launch_one<MOE_W_INT4, 1, 0>(mh1, mp1, mb1, p, n_sm, s);
         if (err != cudaSuccess) return err;
     }
     // phase 2
@@ -934,9 +963,11 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
         p.n_units = H;
         p.rows_per_blob = (int64_t)(L.stride / rb);
         p.q_row_off = (int64_t)(L.off.q2 / rb);
-        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 2>(mh2, mp2, mb2, p, n_sm, s);
-        else if (fmt == MOE_W_INT8) err = launch_one<MOE_W_INT8, 2>(mh2, mp2, mb2, p, n_sm, s);
-        else err = launch_one<MOE_W_INT4, 2>(mh2, mp2, mb2, p, n_sm, s);
+        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 2, 0>(mh2, mp2, mb2, p, n_sm, s);
+        else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 2, 1>(mh2, mp2, mb2, p, n_sm, s)
+                                              : launch_one<MOE_W_INT8, 2, 0>(mh2, mp2, mb2, p, n_sm, s);
+        else err = two ? launch_one<MOE_W_INT4, 2, 1>(mh2, mp2, mb2, p, n_sm, s)
+                       : launch_one<MOE_W_INT4, 2, 0>(mh2, mp2, mb2, p, n_sm, s);
     }
     return err;
 }

@@ -53,6 +53,10 @@ NCU_TRAFFIC_BYTES = {
     ("decode-bf16", 64, "tc"): 1.5164e9,
 }
 
+# routes from which the library's AUTO path takes the tensor-core FFN (bf16, int8,
+# int4), for counting launches: gather + 2 tensor-core launches, else 2 GEMV launches
+TC_MIN_ROUTES = {0: 24, 1: 32, 2: 40}
+
 CONFIGS = {
     # name: (weight format, logits kind, tokens, extra batches swept)
     "decode-bf16": ("bf16", "normal", 64, [1, 8]),
@@ -248,7 +252,7 @@ class Runner:
     def launches_per_step(self):
         """route, permute, FFN (2 GEMV launches, or gather + 2 tensor-core launches), combine"""
         R = self.T * self.k
-        auto_tc = R >= (32 if self.layers[0].fmt == self.moe.MOE_W_BF16 else 96)
+        auto_tc = R >= TC_MIN_ROUTES[self.layers[0].fmt]
         tc = self.path == self.moe.MOE_FFN_TC or (self.path == self.moe.MOE_FFN_AUTO and auto_tc)
         return 4 + (3 if tc else 2)
 
@@ -895,7 +899,8 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
         "sweep": sweep,
         "hbm_peak_gbs": hbm_peak,
         "gpu_launches": steps_done * L * (4 + (3 if (path == moe.MOE_FFN_TC or
-                                                      (path == moe.MOE_FFN_AUTO and T * k >= 96)) else 2))
+                                                      (path == moe.MOE_FFN_AUTO and T * k >= TC_MIN_ROUTES[s4.fmt]))
+                                                     else 2))
                         + (steps_done // 8) * L * (2 if device_refresh else 0),
         "clocks": clk,
     }

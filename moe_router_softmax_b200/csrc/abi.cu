@@ -205,11 +205,11 @@ moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *x, int32
     const int R = T * k;
     int use = path;
     if (use == MOE_FFN_AUTO) {
-        // measured on B200 (Gemma-shaped layer, top-8): the tensor-core kernels
-        // win from 4 tokens for bf16 weights and from about 12 tokens for int8 /
-        // int4 (at 8 tokens the GEMV is faster: 115 vs 154 us int4, 128 vs 140 us
-        // int8; at 16 the tensor cores: 203 vs 224, 194 vs 224)
-        const int min_routes = v.fmt == MOE_W_BF16 ? 32 : 96;
+        // measured on B200 (Gemma-shaped layer, top-8, FFN alone): the
+        // tensor-core kernels win from 3 tokens for bf16 (56.9 vs 61.9 us; at 2
+        // tokens the GEMV: 44.4 vs 51.0), from 4 for int8 (63.2 vs 67.5) and from
+        // about 5 for int4 (6 tokens: 90.8 vs 98.1); one token stays on the GEMV
+        const int min_routes = v.fmt == MOE_W_BF16 ? 24 : (v.fmt == MOE_W_INT8 ? 32 : 40);
         use = (R >= min_routes && ffn_tc_supports(v.fmt, v.H, v.I, v.stride)) ? MOE_FFN_TC : MOE_FFN_GEMV;
     }
     if (use == MOE_FFN_TC && !ffn_tc_supports(v.fmt, v.H, v.I, v.stride))

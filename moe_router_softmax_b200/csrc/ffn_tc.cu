@@ -11,29 +11,33 @@
 // a plain 2-D TMA box.  For bf16 weights TMA writes the A tile straight into
 // the 128-byte-swizzled K-major layout the MMA reads from shared memory.
 // int8/int4 codes land raw (128-byte swizzled, so the dequant warps read them
-// without bank conflicts) and eight dequant warps expand each stage into bf16
-// (int8 codes exactly, with the per-row scale applied in the epilogue; int4 as
-// bf16(q * s) with the group scale, one rounding) and store it in tensor
-// memory, where the MMA takes its A operand: the expanded weights never touch
+// without bank conflicts); a group of eight dequant warps expands each stage
+// into bf16 (int8 codes exactly, with the per-row scale applied in the
+// epilogue; int4 as bf16(q * s) with the group scale, one rounding) and stores
+// it in tensor memory, where the MMA takes its A operand: the expanded weights
+// never touch
 // shared memory, whose bandwidth the MMAs' operand reads would otherwise share
 // with the expansion.
 //
-// One persistent CTA per SM; warp roles:
+// Persistent CTAs (one per SM, or two for int8/int4 decode batches: TcCfg);
+// warp roles:
 //   warp 0      TMA producer of A: the weight tiles (bf16) or the raw codes
 //               (int8 / int4)
 //   warp 1      TMEM allocation and the single-thread MMA issuer
 //   warps 2..5  epilogue (TMEM -> registers -> global); warp w reads TMEM
 //               lanes 32*(w%4) .. +31
 //   warp 6      TMA producer of B: the routes' activation tiles
-//   warps 7..22 dequantisation (int8 / int4 only): two groups of eight warps
-//               taking alternate stages
+//   warps 7..   dequantisation (int8 / int4 only): groups of eight warps taking
+//               alternate stages (two groups, or one with two CTAs per SM)
 // Pipelines: separate rings for A, B and (int formats) raw codes, each with
 // full / empty mbarriers, so a slow operand never holds the other's slots; B
-// slots are sized by the launch's route block, so small decode blocks get many
-// stages in flight; two TMEM accumulators (full / empty) let the epilogue of
-// one item overlap the main loop of the next.  Every mbarrier wait is bounded
-// (and suspends in hardware while it waits); on timeout the kernel records an
-// error word and every role drains out.
+// slots are sized by the busiest expert's route count, so small decode blocks
+// get many stages in flight; two TMEM accumulators (full / empty) let the
+// epilogue of one item overlap the main loop of the next.  Launches are
+// programmatic dependent launches: only the B producer waits for the previous
+// kernel.  Every mbarrier wait is bounded (and suspends in hardware while it
+// waits); on timeout the kernel records an error word and every role drains
+// out.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -47,26 +51,26 @@ namespace moe {
 namespace {
 
 constexpr int kBlockM = 128;          // weight rows per tile (TMEM lanes)
-constexpr int kBlockK = 64;           // bf16 elements per MMA stage = one 128-byte swizzle row
+constexpr int kBlockK = 64;           // bf16 elements per swizzle atom = one 128-byte swizzle row
 constexpr int kNMax = 128;            // max routes per block (TMEM columns per accumulator)
 constexpr int kAccBufs = 2;
 constexpr int kAccCols = kNMax * kAccBufs;   // TMEM columns of the accumulators
 constexpr int kEpiWarps = 4;
-constexpr int kDeqWarps = 8;          // per group: two threads per tile row, half a row each
+constexpr int kDeqWarps = 8;          // per group: two threads per tile row, one 64-wide atom each
 constexpr uint32_t kATileBytes = kBlockM * kBlockK * 2;   // 16 KB
 constexpr int kMaxBSlots = 32;
 constexpr int kRawRowBytes = 128;     // per raw stage row
 constexpr long long kWaitCycles = 4000000000ll;           // ~2 s at 2 GHz
 constexpr int kXPitch = 17;                               // exchange row pitch (floats): no bank conflicts
 
-// Three rings of shared-memory stages, each with its own full / empty
-// mbarriers, so no operand's load latency holds another's slots:
-//  A:   kAStages weight tiles of 128 rows x 64 bf16 (bf16 weights: TMA into
+// Three rings of stages, each with its own full / empty mbarriers, so no
+// operand's load latency holds another's slots:
+//  A:   kAStages weight tiles of 128 rows x kKS bf16 (bf16 weights: TMA into
 //       shared memory; int8/int4: the dequant warps, into tensor memory);
-//  B:   up to kMaxBSlots activation tiles of n_block rows x 64 bf16 (TMA), as
-//       many as fit in kBRegion bytes for this launch's block size;
+//  B:   up to kMaxBSlots activation tiles of n_block rows x kKS bf16 (TMA), as
+//       many as fit in kBRegion bytes for this launch's route block;
 //  raw: kRawStages stages of 128 code bytes per row (int formats: 256 int4 or
-//       128 int8 weights, kSub MMA stages each), whole 128-byte runs of a row.
+//       128 int8 weights, kSub A stages each), whole 128-byte runs of a row.
 // For int8 / int4 the A ring lives in tensor memory instead (kASmem = 0): the
 // dequant warps store the bf16 tiles with tcgen05.st and the MMAs read A from
 // TMEM, so the expanded weights never pass through shared memory.
@@ -75,7 +79,7 @@ constexpr int kXPitch = 17;                               // exchange row pitch 
 // MMAs instead of per 4 (each tcgen05 instruction and each barrier wait costs
 // that thread tens of nanoseconds, which otherwise bounds a decode batch's
 // small MMAs).
-// kSub stages share one raw stage of kRawRowBytes per row (kSubBytes each).
+// kSub A stages share one raw stage of kRawRowBytes per row (kSubBytes each).
 template <int FMT> struct TcFmt;
 template <> struct TcFmt<MOE_W_BF16> {
     static constexpr int kKS = 128, kSub = 1, kSubBytes = 0, kAStages = 4, kASmem = 1, kRawStages = 0;

@@ -15,9 +15,8 @@
 // into bf16 (int8 codes exactly, with the per-row scale applied in the
 // epilogue; int4 as bf16(q * s) with the group scale, one rounding) and stores
 // it in tensor memory, where the MMA takes its A operand: the expanded weights
-// never touch
-// shared memory, whose bandwidth the MMAs' operand reads would otherwise share
-// with the expansion.
+// never touch shared memory, whose bandwidth the MMAs' operand reads would
+// otherwise share with the expansion.
 //
 // Persistent CTAs (one per SM, or two for int8/int4 decode batches: TcCfg);
 // warp roles:

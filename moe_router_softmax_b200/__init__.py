@@ -6,7 +6,7 @@ the name of the C entry point it calls, checks and marshals its arguments
 ``MoeError`` with ``moe_last_error()`` when the call fails.  Every step of the
 layer runs in the library's kernels; PyTorch only provides device memory and
 streams.  There is no fallback: if the shared library is missing, importing this
-package raises ImportError (build it with ``moe_router_softmax_b200.build.build()``).
+package raises ImportError (build it with ``python moe_router_softmax_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -20,7 +20,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built: run python -m moe_router_softmax_b200.build")
+    raise ImportError(f"{LIB_PATH} is not built: run python moe_router_softmax_b200/build.py "
+                      "(or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

@@ -64,6 +64,16 @@ __device__ float exp_p(float x) {
     return __fmul_rn(p, pow2_bits(ni));
 }
 
+// A 32-bit key whose unsigned order is the logit order of ranks_before: NaN
+// below every number (key 0, and every NaN alike), -0 equal to +0, otherwise
+// the IEEE bits made monotone (negative: all bits flipped; positive: sign set).
+// Equal keys are then ordered by expert id separately.
+__device__ __forceinline__ uint32_t rank_key(float v) {
+    if (v != v) return 0u;
+    const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // (va, ea) ranks before (vb, eb): larger logit, then lower id; NaN last.
 __device__ __forceinline__ bool ranks_before(float va, int ea, float vb, int eb) {
     bool na = va != va, nb = vb != vb;
@@ -92,7 +102,7 @@ __device__ __forceinline__ void route_token_warp(Load load, int E, int k, int32_
     float my_v = 0.0f;
     int my_e = 0;
     for (int j = 0; j < k; ++j) {
-        // best available value held by this lane
+        // best available value held by this lane (ties to the lower id: i ascending)
         bool has = false;
         float bv = 0.0f;
         int be = 0;
@@ -107,22 +117,17 @@ __device__ __forceinline__ void route_token_warp(Load load, int E, int k, int32_
                 }
             }
         }
-        // warp arg-best
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            bool oh = __shfl_xor_sync(0xffffffffu, (int)has, off) != 0;
-            if (oh && (!has || ranks_before(ov, oe, bv, be))) {
-                has = true;
-                bv = ov;
-                be = oe;
-            }
-        }
-        if (lane == (be & 31)) avail &= ~(1u << (be >> 5));
+        // warp arg-best in two reductions: the largest rank key, then the lowest
+        // expert id among the lanes holding it
+        const uint32_t key = has ? rank_key(bv) : 0u;
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const int cand = (has && key == kmax) ? be : 0x7fffffff;
+        const int win = __reduce_min_sync(0xffffffffu, cand);
+        const float wv = __shfl_sync(0xffffffffu, bv, win & 31);
+        if (lane == (win & 31)) avail &= ~(1u << (win >> 5));
         if (lane == j) {
-            my_v = bv;
-            my_e = be;
+            my_v = wv;
+            my_e = win;
         }
     }
     const float m = __shfl_sync(0xffffffffu, my_v, 0);

@@ -319,6 +319,22 @@ def time_steps(torch, runner, steps, warmup, dist):
     return ms, ffn_ms
 
 
+def time_eager(torch, runner, steps, warmup):
+    """The same steps launched one by one from Python (no CUDA graph), between
+    two events: the eager counterpart of time_steps."""
+    for i in range(warmup):
+        runner.step(i)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        runner.step(warmup + i)
+    t1.record()
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1)
+
+
 def time_e2e(torch, moe, layers, batches, T, k, steps, warmup, dev):
     """End to end through moe_layer_forward with host buffers: every step copies
     its logits and x from pinned host memory and reads y back to pinned host
@@ -433,6 +449,15 @@ def cpu_baseline(moe, torch, cfg_fmt, layers, batches, T, k, seconds, first_toke
     else:
         return None  # the quantised formats need the source bf16 weights; bf16 is the benchmarked config
     OL = oracle.Layer(fmt, E, H, I, np.zeros(eb, np.uint8), pool=pool, slot_table=slot)
+    # one thread first (a short sample), then every host thread
+    oracle.set_threads(1)
+    n1, t1 = 0, time.perf_counter()
+    while True:
+        oracle.moe_layer(OL, lg[n1 % T:n1 % T + 1], x[n1 % T:n1 % T + 1], k)
+        n1 += 1
+        e1 = time.perf_counter() - t1
+        if e1 >= min(seconds / 3, 5.0) or first_token_only:
+            break
     oracle.set_threads(os.cpu_count() or 1)
     threads = oracle.get_threads()
     n, t0 = 0, time.perf_counter()
@@ -446,7 +471,9 @@ def cpu_baseline(moe, torch, cfg_fmt, layers, batches, T, k, seconds, first_toke
     del home_host
     return {"value": n / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{n} token evaluations cycling through the {T} tokens of one batch ({n * k} routes), "
-                      f"whole layer (route, per-route fp64 FFN, combine), {el:.1f} s"}
+                      f"whole layer (route, per-route fp64 FFN, combine), {el:.1f} s",
+            "single_thread": {"value": round(n1 / e1, 3), "unit": "tokens/s", "cores": 1,
+                              "sample": f"{n1} token evaluations, {e1:.1f} s"}}
 
 
 def main():
@@ -533,6 +560,9 @@ def main():
             r["frac_of_hbm"] = round(r["hbm_gbs"] / hbm_peak, 4)
             router[f"T{Tr}"] = r
 
+    eager_steps = min(args.steps, 500)
+    eager_ms = float("nan") if args.quick else time_eager(torch, runner, eager_steps, args.warmup)
+    eager_ms = max_over_ranks(dist, eager_ms, dev)
     e2e_ms, h2d, d2h = (float("nan"), 0, 0) if args.quick else time_e2e(torch, moe, layers, batches, T, k,
                                                                          args.steps, args.warmup, dev)
     e2e_ms = max_over_ranks(dist, e2e_ms, dev)
@@ -590,6 +620,10 @@ def main():
         }),
         "sweep": sweep_out,
         "router_topk": router,
+        "eager": None if args.quick else {
+            "tokens_per_s": round(world * T * eager_steps / (eager_ms / 1e3), 1),
+            "ms_per_step": round(eager_ms / eager_steps, 5), "steps": eager_steps,
+            "note": "the same steps launched from Python one by one (no CUDA graph)"},
         "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": runner.launches_per_step() * args.steps,

@@ -253,7 +253,7 @@ __device__ __forceinline__ float gelu_tanh(float v) {
 // expert then fits one block, and a decode batch whose experts hold a handful of
 // routes gets small B slots, so many B stages are in flight.
 struct Items {
-    int n_act, total, m_tiles, n_block, b_slots;
+    int n_act, total, m_tiles, n_block, b_rows, b_slots;
 };
 
 __device__ void build_items(const TcParams &p, int m_tiles, int b_region, int atoms, int *s_act, int *s_base,
@@ -292,7 +292,11 @@ __device__ void build_items(const TcParams &p, int m_tiles, int b_region, int at
             it->total = run;
             it->m_tiles = m_tiles;
             it->n_block = n_block;
-            it->b_slots = min(kMaxBSlots, b_region / (n_block * 128 * atoms));
+            // B slot rows: a block over 32 routes is loaded in 64-row boxes (two to
+            // four TMA instructions per stage instead of up to sixteen)
+            const int b_rows = n_block <= 32 ? n_block : (n_block + 63) & ~63;
+            it->b_rows = b_rows;
+            it->b_slots = min(kMaxBSlots, b_region / (b_rows * 128 * atoms));
         }
     }
 }
@@ -350,7 +354,7 @@ __host__ __device__ constexpr int tc_threads() {
 template <int FMT, int PHASE, int CFG>
 __global__ void __launch_bounds__(tc_threads<FMT, CFG>(), TcCfg<FMT, CFG>::kMinBlocks)
 k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ CUtensorMap map_pool,
-         const __grid_constant__ CUtensorMap map_b, const TcParams p) {
+         const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_b64, const TcParams p) {
     using C = TcCfg<FMT, CFG>;
     constexpr int SA = C::kAStages;
     constexpr int SR = C::kRawStages;
@@ -436,7 +440,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     // accumulator's C::kNMax columns), which the epilogue adds up, so that
     // consecutive MMAs do not update the same small tile.
     const int nacc = n_block <= C::kNMax / 4 ? 4 : (n_block <= C::kNMax / 2 ? 2 : 1);
-    const uint32_t b_atom_bytes = (uint32_t)n_block * 128;       // one 64-wide atom of a B slot
+    const uint32_t b_atom_bytes = (uint32_t)s_items.b_rows * 128;  // one 64-wide atom of a B slot
     const uint32_t b_slot_bytes = b_atom_bytes * ATOMS;
 
     if (warp == 0) {
@@ -494,14 +498,19 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
                 const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 bool ok = true;
+                // up to 32 routes: 16-row boxes; more: 64-row boxes (rows past
+                // the block are another expert's or out of range and zero-filled;
+                // the slot holds them, the MMAs read only the first n_mma)
+                const bool big = it.n_mma > 32 && p.R >= 64;  // the 64-row map exists from 64 rows
+                const int rows_ld = big ? (it.n_mma + 63) & ~63 : it.n_mma;
                 for (int kk = 0; kk < nk; ++kk) {
                     const int na = atoms_at(kk);
                     if (!mbar_wait(&b_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&b_full[stage], (uint32_t)(na * it.n_mma * 128));
+                    mbar_arrive_expect_tx(&b_full[stage], (uint32_t)(na * rows_ld * 128));
                     uint8_t *db = sB + stage * b_slot_bytes;
                     for (int a = 0; a < na; ++a)
-                        for (int j = 0; j < it.n_mma; j += 16)
-                            tma_load_2d(db + a * b_atom_bytes + j * 128, &map_b, &b_full[stage],
+                        for (int j = 0; j < rows_ld; j += big ? 64 : 16)
+                            tma_load_2d(db + a * b_atom_bytes + j * 128, big ? &map_b64 : &map_b, &b_full[stage],
                                         (kk * ATOMS + a) * kBlockK, it.row0 + j);
                     if (++stage == b_slots) { stage = 0; phase ^= 1; }
                 }
@@ -845,8 +854,8 @@ static_assert(2 * TcCfg<MOE_W_INT4, 1>::kTmemCols <= 512 && TcCfg<MOE_W_INT4, 1>
               "two-CTA config exceeds tensor memory");
 
 template <int FMT, int PHASE, int CFG>
-cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUtensorMap &mb, const TcParams &p,
-                       int n_sm, cudaStream_t s) {
+cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUtensorMap &mb, const CUtensorMap &mb64,
+                       const TcParams &p, int n_sm, cudaStream_t s) {
     auto kern = k_ffn_tc<FMT, PHASE, CFG>;
     const size_t smem = smem_bytes<FMT, CFG>();
     static bool attr[kMaxDevices] = {};
@@ -861,7 +870,7 @@ cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUten
     }
     // programmatic dependent launch (the B producer waits for the previous launch)
     return launch_pdl(kern, dim3((unsigned)(n_sm * TcCfg<FMT, CFG>::kMinBlocks)), dim3((unsigned)tc_threads<FMT, CFG>()),
-                      smem, s, mh, mp, mb, p);
+                      smem, s, mh, mp, mb, mb64, p);
 }
 
 }  // namespace
@@ -910,7 +919,7 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     const int eb = bf ? 2 : 1;
     const CUtensorMapSwizzle swa = CU_TENSOR_MAP_SWIZZLE_128B;  // weight tiles and raw code tiles alike
     const uint32_t raw_inner = kRawRowBytes;
-    CUtensorMap mh1, mp1, mh2, mp2, mb1, mb2;
+    CUtensorMap mh1, mp1, mh2, mp2, mb1, mb2, mbb1, mbb2;
     for (int ph = 1; ph <= 2; ++ph) {
         const int K = ph == 1 ? H : I;
         const uint64_t row_elems = bf ? (uint64_t)K : (fmt == MOE_W_INT8 ? (uint64_t)K : (uint64_t)K / 2);
@@ -923,9 +932,14 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
         // (only rows of slots in use are ever addressed)
         if (!encode_2d(mp, L.pool ? L.pool : L.home, dt, eb, row_elems, home_rows, box_inner, 64, swa))
             return cudaErrorInvalidValue;
-        CUtensorMap *mb = ph == 1 ? &mb1 : &mb2;
+        CUtensorMap *mb = ph == 1 ? &mb1 : &mb2, *mbb = ph == 1 ? &mbb1 : &mbb2;
         if (!encode_2d(mb, ph == 1 ? (const void *)xs : (const void *)h, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
                        (uint64_t)K, (uint64_t)R, kBlockK, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        // 64-row boxes for route blocks over 32 (only used when a block that large
+        // exists, i.e. R > 32)
+        if (!encode_2d(mbb, ph == 1 ? (const void *)xs : (const void *)h, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                       (uint64_t)K, (uint64_t)R, kBlockK, R >= 64 ? 64 : 16, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
     TcParams p{};
@@ -952,11 +966,11 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
         p.n_units = 2 * I;
         p.rows_per_blob = (int64_t)(L.stride / rb);
         p.q_row_off = (int64_t)(L.off.q13 / rb);
-        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 1, 0>(mh1, mp1, mb1, p, n_sm, s);
-        else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 1, 1>(mh1, mp1, mb1, p, n_sm, s)
-                                              : launch_one<MOE_W_INT8, 1, 0>(mh1, mp1, mb1, p, n_sm, s);
-        else err = two ? launch_one<MOE_W_INT4, 1, 1>(mh1, mp1, mb1, p, n_sm, s)
-                       : launch_one<MOE_W_INT4, 1, 0>(mh1, mp1, mb1, p, n_sm, s);
+        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 1, 0>(mh1, mp1, mb1, mbb1, p, n_sm, s);
+        else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 1, 1>(mh1, mp1, mb1, mbb1, p, n_sm, s)
+                                              : launch_one<MOE_W_INT8, 1, 0>(mh1, mp1, mb1, mbb1, p, n_sm, s);
+        else err = two ? launch_one<MOE_W_INT4, 1, 1>(mh1, mp1, mb1, mbb1, p, n_sm, s)
+                       : launch_one<MOE_W_INT4, 1, 0>(mh1, mp1, mb1, mbb1, p, n_sm, s);
         if (err != cudaSuccess) return err;
     }
     // phase 2
@@ -966,11 +980,11 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
         p.n_units = H;
         p.rows_per_blob = (int64_t)(L.stride / rb);
         p.q_row_off = (int64_t)(L.off.q2 / rb);
-        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 2, 0>(mh2, mp2, mb2, p, n_sm, s);
-        else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 2, 1>(mh2, mp2, mb2, p, n_sm, s)
-                                              : launch_one<MOE_W_INT8, 2, 0>(mh2, mp2, mb2, p, n_sm, s);
-        else err = two ? launch_one<MOE_W_INT4, 2, 1>(mh2, mp2, mb2, p, n_sm, s)
-                       : launch_one<MOE_W_INT4, 2, 0>(mh2, mp2, mb2, p, n_sm, s);
+        if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 2, 0>(mh2, mp2, mb2, mbb2, p, n_sm, s);
+        else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 2, 1>(mh2, mp2, mb2, mbb2, p, n_sm, s)
+                                              : launch_one<MOE_W_INT8, 2, 0>(mh2, mp2, mb2, mbb2, p, n_sm, s);
+        else err = two ? launch_one<MOE_W_INT4, 2, 1>(mh2, mp2, mb2, mbb2, p, n_sm, s)
+                       : launch_one<MOE_W_INT4, 2, 0>(mh2, mp2, mb2, mbb2, p, n_sm, s);
     }
     return err;
 }

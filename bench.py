@@ -272,16 +272,22 @@ class Runner:
         return out
 
 
+FFN_SAMPLE_EVERY = 5
+
+
 def _capture(torch, runner, first, n):
     """One CUDA graph of n consecutive steps, with an external event pair around
-    each step's grouped-FFN launches (event record nodes inside the graph)."""
+    the grouped-FFN launches of every FFN_SAMPLE_EVERY-th step (event record
+    nodes inside the graph).  An event node between two kernels also cuts their
+    programmatic-launch edge, so only the sampled steps carry them."""
     g = torch.cuda.CUDAGraph()
-    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           for _ in range(n)]
+    sampled = [j for j in range(n) if j % FFN_SAMPLE_EVERY == FFN_SAMPLE_EVERY // 2] or [0]
+    evs = {j: (torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for j in sampled}
     with torch.cuda.graph(g):
         for j in range(n):
-            runner.step(first + j, evs[j])
-    return g, evs
+            runner.step(first + j, evs.get(j))
+    return g, list(evs.values())
 
 
 def time_steps(torch, runner, steps, warmup, dist):

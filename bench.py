@@ -431,6 +431,74 @@ def time_router(torch, moe, T, E, H, k, dev, n=200):
             "hbm_gbs": round(alg / (us / 1e6) / 1e9, 1), "router_copies": copies}
 
 
+def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
+    """Each step of the path on its own, replayed n times from a CUDA graph on
+    the decode batch's shapes: average us per call and algorithmic GB/s (inputs
+    read + outputs written).  The quantisers run on one expert's w13 [2I, H]."""
+    import synthetic as syn
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(23)
+    lg = torch.from_numpy(syn.router_logits(T, E, "normal", seed=23)).to(dev)
+    ids, w = moe.moe_route_topk(lg, k)
+    perm = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
+            torch.empty(T * k, dtype=torch.int32, device=dev), torch.empty(T * k, dtype=torch.int32, device=dev))
+    moe.moe_permute(ids, E, out=perm)
+    rows = torch.randn((T * k, H), generator=g, device=dev, dtype=torch.float32)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    hits = torch.zeros(E, dtype=torch.int32, device=dev)
+    ids2, w2 = ids.clone(), w.clone()
+    table = torch.full((E,), -1, dtype=torch.int32, device=dev)
+    table[:18] = torch.arange(18, dtype=torch.int32, device=dev)
+    wq = (torch.randn((2 * I, H), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    q8, s8 = moe.moe_quantize_int8(wq)
+    q4, s4 = moe.moe_quantize_int4(wq)
+    thits = torch.randint(0, 9, (E,), generator=g, device=dev, dtype=torch.int32)
+    rtable = table.clone()
+    promo = torch.zeros((18, 2), dtype=torch.int32, device=dev)
+    status = torch.zeros(3, dtype=torch.int32, device=dev)
+    pool = torch.empty(18 * layer.expert_bytes, dtype=torch.uint8, device=dev)
+    R = T * k
+    cases = [
+        ("route_topk", lambda: moe.moe_route_topk(lg, k, ids=ids, w=w), T * E * 4 + R * 8),
+        ("route_min_weight (0.6)", lambda: moe.moe_route_min_weight(ids2, w2, E, 0.6, slot_table=table), R * 16 + E * 4),
+        ("permute + hits", lambda: moe.moe_permute(ids, E, hits=hits, out=perm), R * 4 + R * 8 + E * 12),
+        ("combine", lambda: moe.moe_combine(rows, perm[3], w, y), R * H * 4 + R * 8 + T * H * 2),
+        ("quantize_int8 (one w13)", lambda: moe.moe_quantize_int8(wq, q8, s8), 2 * I * H * 3 + 2 * I * 4),
+        ("quantize_int4 (one w13)", lambda: moe.moe_quantize_int4(wq, q4, s4), 2 * I * H * 2 + I * H + 2 * I * (H // 64) * 2),
+        ("refresh_device (18 slots)", lambda: moe.moe_refresh_device(thits, 18, rtable, 18, promo=promo, status=status),
+         E * 8),
+        ("promote_copies (listed blobs)", lambda: moe.moe_promote_copies(layer.home, pool, layer.expert_bytes, promo,
+                                                                       status, 18), None),
+    ]
+    out = {}
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for name, fn, nbytes in cases:
+            fn()
+            stream.synchronize()
+            if name.startswith("refresh_device"):
+                rtable.copy_(table)  # the first call above changed it; replays refresh from the same table
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for _ in range(n):
+                    fn()
+            graph.replay()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            stream.synchronize()
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+            b.synchronize()
+            us = a.elapsed_time(b) * 1e3 / n
+            if nbytes is None:  # promotions listed by the last refresh
+                nbytes = 2 * int(status[0].item()) * layer.expert_bytes
+            out[name] = {"us": round(us, 2), "alg_bytes": int(nbytes), "gbs": round(nbytes / (us / 1e6) / 1e9, 1)}
+            del graph
+    return out
+
+
 def cpu_baseline(moe, torch, cfg_fmt, layers, batches, T, k, seconds, first_token_only=False):
     """The oracle (as it stands) on a bounded sample: whole tokens of batch 0 of
     layer 0, one at a time, until `seconds` have passed."""
@@ -559,6 +627,12 @@ def main():
             "ffn_frac_of_hbm": round((dd * eb + Ts * H * 2) / (f2 / 1e3) / 1e9 / hbm_peak, 4),
         }
 
+    kernels = None
+    if not args.quick and args.config != "tiny":
+        try:
+            kernels = time_kernels(torch, moe, layers[0], T, E, H, I, k, dev)
+        except Exception as exc:  # keep the headline line even if a side measurement fails
+            kernels = {"error": f"{type(exc).__name__}: {exc}"}
     router = {}
     if args.config != "tiny":
         for Tr in ([T] if args.quick else sorted({1, T, 1024})):
@@ -626,6 +700,7 @@ def main():
         }),
         "sweep": sweep_out,
         "router_topk": router,
+        "kernels": kernels,
         "eager": None if args.quick else {
             "tokens_per_s": round(world * T * eager_steps / (eager_ms / 1e3), 1),
             "ms_per_step": round(eager_ms / eager_steps, 5), "steps": eager_steps,

@@ -458,6 +458,10 @@ def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
     promo = torch.zeros((18, 2), dtype=torch.int32, device=dev)
     status = torch.zeros(3, dtype=torch.int32, device=dev)
     pool = torch.empty(18 * layer.expert_bytes, dtype=torch.uint8, device=dev)
+    # a fixed promotion list for the copy timing: experts 18..35 into slots 0..17
+    cpromo = torch.stack([torch.arange(18, 36, dtype=torch.int32, device=dev),
+                          torch.arange(18, dtype=torch.int32, device=dev)], dim=1).contiguous()
+    cstatus = torch.tensor([18, 18, 0], dtype=torch.int32, device=dev)
     R = T * k
     cases = [
         ("route_topk", lambda: moe.moe_route_topk(lg, k, ids=ids, w=w), T * E * 4 + R * 8),
@@ -468,8 +472,8 @@ def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
         ("quantize_int4 (one w13)", lambda: moe.moe_quantize_int4(wq, q4, s4), 2 * I * H * 2 + I * H + 2 * I * (H // 64) * 2),
         ("refresh_device (18 slots)", lambda: moe.moe_refresh_device(thits, 18, rtable, 18, promo=promo, status=status),
          E * 8),
-        ("promote_copies (listed blobs)", lambda: moe.moe_promote_copies(layer.home, pool, layer.expert_bytes, promo,
-                                                                       status, 18), None),
+        ("promote_copies (18 blobs)", lambda: moe.moe_promote_copies(layer.home, pool, layer.expert_bytes, cpromo,
+                                                                   cstatus, 18), 2 * 18 * layer.expert_bytes),
     ]
     out = {}
     stream = torch.cuda.Stream(dev)
@@ -492,8 +496,6 @@ def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
             b.record(stream)
             b.synchronize()
             us = a.elapsed_time(b) * 1e3 / n
-            if nbytes is None:  # promotions listed by the last refresh
-                nbytes = 2 * int(status[0].item()) * layer.expert_bytes
             out[name] = {"us": round(us, 2), "alg_bytes": int(nbytes), "gbs": round(nbytes / (us / 1e6) / 1e9, 1)}
             del graph
     return out

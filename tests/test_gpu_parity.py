@@ -104,8 +104,10 @@ def _special_matrix(rows, K, seed):
     return w
 
 
-@pytest.mark.parametrize("rows,K", [(1408, 2816), (2816, 704), (64, 256), (3, 64)])
+@pytest.mark.parametrize("rows,K", [(1408, 2816), (2816, 704), (64, 256), (3, 64), (5, 100), (3, 4104)])
 def test_quantize_int8_bit_exact(rows, K):
+    """(5, 100) and (3, 4104) take the element-loop kernel (K not a multiple of 8,
+    or more than 16 chunks per lane); the others the register-resident one."""
     w = _special_matrix(rows, K, rows)
     q, s = moe.moe_quantize_int8(torch.from_numpy(w.view(np.int16)).to(DEV))
     oq, os_ = oracle.quantize_int8(w)

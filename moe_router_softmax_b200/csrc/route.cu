@@ -173,7 +173,6 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
 // are added by a butterfly (xor 16, 8, 4, 2, 1).
 constexpr int kRouterCluster = 8;
 constexpr int kRouterThreads = 256;
-constexpr int kRouterWarps = kRouterThreads / 32;
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -181,8 +180,11 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-template <int TOK, int VPL>
-__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouterThreads)
+// NT threads per CTA: 256 (eight warps, two experts each), or for one token
+// 512 (sixteen warps, one expert each, all of a lane's chunks of the row in
+// flight at once: one DRAM round trip instead of three at H = 2816).
+template <int TOK, int VPL, int NT>
+__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(NT)
     k_router_topk(const uint16_t *__restrict__ x, const float *__restrict__ wr, int T, int H, int E, int k,
                   float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ w) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -201,13 +203,13 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouter
     if (e_hi > e_lo) {
         const char *slice = reinterpret_cast<const char *>(wr + (size_t)e_lo * H);
         const size_t bytes = (size_t)(e_hi - e_lo) * H * 4;
-        for (size_t off = (size_t)threadIdx.x * 128; off < bytes; off += (size_t)kRouterThreads * 128)
+        for (size_t off = (size_t)threadIdx.x * 128; off < bytes; off += (size_t)NT * 128)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(slice + off));
     }
 
     // the group's activation rows (zero past the last token)
     const int h4 = H / 4;
-    for (int i = threadIdx.x; i < TOK * h4; i += kRouterThreads) {
+    for (int i = threadIdx.x; i < TOK * h4; i += NT) {
         const int t = i / h4, c = i - t * h4;
         uint2 v = make_uint2(0u, 0u);
         if (t < nt) v = __ldg(reinterpret_cast<const uint2 *>(x + (size_t)(t0 + t) * H) + c);
@@ -215,12 +217,14 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouter
     }
     __syncthreads();
 
-    // projection: warp w takes experts e_lo + 2w, +1, then + 2*kRouterWarps, ...
-    // U chunks of 128 h per lane are loaded before they are used, so U loads of
-    // each operand are in flight (the sums still run in increasing h)
-    constexpr int U = TOK <= 8 ? 8 : 4;
-    for (int e0 = e_lo + 2 * warp; e0 < e_hi; e0 += 2 * kRouterWarps) {
-        const bool two = e0 + 1 < e_hi;
+    // projection: warp w takes experts e_lo + EPW w (and the next one when EPW
+    // is 2), then + EPW * NW, ...; U chunks of 128 h per lane are loaded before
+    // they are used, so U loads of each operand are in flight (the sums still run
+    // in increasing h)
+    constexpr int NW = NT / 32, EPW = NT >= 512 ? 1 : 2;
+    constexpr int U = NT >= 512 ? 22 : (TOK <= 8 ? 8 : 4);
+    for (int e0 = e_lo + EPW * warp; e0 < e_hi; e0 += EPW * NW) {
+        const bool two = EPW == 2 && e0 + 1 < e_hi;
         const float *w0 = wr + (size_t)e0 * H;
         const float *w1 = wr + (size_t)(two ? e0 + 1 : e0) * H;
         float a0[TOK], a1[TOK];
@@ -234,7 +238,7 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouter
                 p[u] = q[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (h < H) {
                     p[u] = __ldg(reinterpret_cast<const float4 *>(w0 + h));
-                    q[u] = __ldg(reinterpret_cast<const float4 *>(w1 + h));
+                    if (EPW == 2) q[u] = __ldg(reinterpret_cast<const float4 *>(w1 + h));
                 }
             }
 #pragma unroll
@@ -250,10 +254,12 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouter
                         a0[t] = __fmaf_rn(x1, p[u].y, a0[t]);
                         a0[t] = __fmaf_rn(x2, p[u].z, a0[t]);
                         a0[t] = __fmaf_rn(x3, p[u].w, a0[t]);
-                        a1[t] = __fmaf_rn(x0, q[u].x, a1[t]);
-                        a1[t] = __fmaf_rn(x1, q[u].y, a1[t]);
-                        a1[t] = __fmaf_rn(x2, q[u].z, a1[t]);
-                        a1[t] = __fmaf_rn(x3, q[u].w, a1[t]);
+                        if (EPW == 2) {
+                            a1[t] = __fmaf_rn(x0, q[u].x, a1[t]);
+                            a1[t] = __fmaf_rn(x1, q[u].y, a1[t]);
+                            a1[t] = __fmaf_rn(x2, q[u].z, a1[t]);
+                            a1[t] = __fmaf_rn(x3, q[u].w, a1[t]);
+                        }
                     }
                 }
             }
@@ -261,7 +267,7 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouter
 #pragma unroll
         for (int t = 0; t < TOK; ++t) {
             a0[t] = warp_sum(a0[t]);
-            a1[t] = warp_sum(a1[t]);
+            if (EPW == 2) a1[t] = warp_sum(a1[t]);
         }
         if (lane == 0) {
 #pragma unroll
@@ -290,10 +296,10 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouter
     cluster.sync();
 }
 
-template <int TOK, int VPL>
+template <int TOK, int VPL, int NT = kRouterThreads>
 cudaError_t launch_router(const uint16_t *x, const float *wr, int T, int H, int E, int k, float *logits,
                           int32_t *ids, float *w, cudaStream_t s) {
-    auto kern = k_router_topk<TOK, VPL>;
+    auto kern = k_router_topk<TOK, VPL, NT>;
     static bool attr[kMaxDevices] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -305,7 +311,7 @@ cudaError_t launch_router(const uint16_t *x, const float *wr, int T, int H, int 
         attr[dev] = true;
     }
     dim3 grid(kRouterCluster, (unsigned)((T + TOK - 1) / TOK));
-    kern<<<grid, kRouterThreads, router_smem(TOK, H, E), s>>>(x, wr, T, H, E, k, logits, ids, w);
+    kern<<<grid, NT, router_smem(TOK, H, E), s>>>(x, wr, T, H, E, k, logits, ids, w);
     return cudaGetLastError();
 }
 
@@ -315,7 +321,7 @@ cudaError_t launch_router_vpl(const uint16_t *x, const float *wr, int T, int H, 
     const int tok = router_tok(T, H, E);
     if (router_smem(tok, H, E) > kRouterMaxSmem) return cudaErrorInvalidValue;
     if (tok == 16) return launch_router<16, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
-    if (tok == 1) return launch_router<1, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
+    if (tok == 1) return launch_router<1, VPL, 512>(x, wr, T, H, E, k, logits, ids, w, s);
     if (tok == 2) return launch_router<2, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
     if (tok == 4) return launch_router<4, VPL>(x, wr, T, H, E, k, logits, ids, w, s);
     return launch_router<8, VPL>(x, wr, T, H, E, k, logits, ids, w, s);

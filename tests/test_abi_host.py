@@ -183,3 +183,42 @@ def test_device_refresh_rejects_bad_arguments_before_launch():
     assert L.moe_promote_copies(256, 256, 100, 256, 256, 4, None) == moe.MOE_ERR_INVALID_ARG       # size % 16
     assert L.moe_promote_copies(264, 256, 256, 256, 256, 4, None) == moe.MOE_ERR_INVALID_ARG       # unaligned
     assert L.moe_promote_copies(256, 256, 256, 256, 256, 0, None) == moe.MOE_OK                    # nothing to do
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover
+    given = None
+
+
+if given is not None:
+    @st.composite
+    def _placement_case(draw):
+        E = draw(st.integers(1, 64))
+        n_slots = draw(st.integers(0, E))
+        budget = draw(st.integers(0, n_slots))
+        hits = np.array(draw(st.lists(st.integers(0, 5), min_size=E, max_size=E)), np.uint32)
+        n_res = draw(st.integers(0, n_slots))
+        experts = draw(st.permutations(list(range(E))))[:n_res]
+        slots = draw(st.permutations(list(range(n_slots))))[:n_res] if n_slots else []
+        slot_of = np.full(E, -1, np.int32)
+        slot_of[list(experts)] = list(slots)
+        return hits, slot_of, n_slots, budget
+
+    @settings(max_examples=300, deadline=None)
+    @given(_placement_case())
+    def test_placement_property_matches_oracle(case):
+        """Generated hit histograms and slot tables (empty and full pools, zero
+        budget, all-zero hits, ties): the library's host placement equals the
+        oracle's, and the residency invariants hold."""
+        hits, slot_of, n_slots, budget = case
+        target = moe.moe_refresh_target(hits, budget)
+        assert np.array_equal(target, oracle.refresh_target(hits, budget))
+        so, pr, de = moe.moe_apply_placement(slot_of, n_slots, target)
+        oso, opr, ode = oracle.apply_placement(slot_of, n_slots, target)
+        assert np.array_equal(so, oso) and np.array_equal(pr, opr) and np.array_equal(de, ode)
+        held = so[so >= 0]
+        assert len(set(held.tolist())) == len(held) and (held < n_slots).all()
+        assert all(so[t] >= 0 for t in target)
+        assert len(held) == int((slot_of >= 0).sum()) - len(de) + len(pr)
+        assert set(pr.tolist()).isdisjoint(de.tolist())

@@ -66,7 +66,9 @@ typedef enum {
 /* Expert weight formats (prain README.md, "Expert formats"). */
 typedef enum { MOE_W_BF16 = 0, MOE_W_INT8 = 1, MOE_W_INT4 = 2 } moe_wfmt;
 
-/* Kernel path for the grouped FFN: AUTO picks by routes per call. */
+/* Kernel path for the grouped FFN.  AUTO takes the tensor-core kernels from
+ * T*k >= 24 / 32 / 40 routes (bf16 / int8 / int4 weights), the GEMV kernels
+ * below that (measured crossovers on B200 at the Gemma shape, top-8). */
 typedef enum { MOE_FFN_AUTO = 0, MOE_FFN_GEMV = 1, MOE_FFN_TC = 2 } moe_ffn_path;
 
 /*
@@ -188,7 +190,12 @@ MOE_API moe_status moe_expert_hits(const int32_t *ids, int64_t n, int32_t E, uin
  * ws: device workspace of at least moe_grouped_ffn_workspace() bytes.
  * moe_grouped_ffn_path forces a kernel path (MOE_FFN_GEMV: split-K GEMV
  * kernels; MOE_FFN_TC: tcgen05 tensor-core kernels); MOE_ERR_UNSUPPORTED if
- * the forced path does not handle the format.
+ * the forced path does not handle the format.  Asynchronous on `stream`; the
+ * kernels are launched with programmatic stream serialization (each waits for
+ * the previous kernel in the stream before reading its results), which is
+ * transparent to callers and to CUDA graph capture.  A tensor-core kernel that
+ * finds an inconsistent route block or gives up a bounded wait records it for
+ * moe_take_device_errors() and skips the affected work.
  */
 MOE_API size_t moe_grouped_ffn_workspace(const moe_layer *layer, int32_t T, int32_t k);
 MOE_API moe_status moe_grouped_ffn(const moe_layer *layer, const uint16_t *x, int32_t T, int32_t k,

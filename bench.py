@@ -48,15 +48,13 @@ import numpy as np  # noqa: E402
 NCU_TRAFFIC_BYTES = {
     # profiles/ffn_gemv_bf16_T64.md: phase 1 1.0059 GB + 4.04 MB, phase 2 0.5027 GB + 5.28 MB
     ("decode-bf16", 64, "gemv"): 1.5180e9,
-    # profiles/ffn_tc_bf16_decode_T64.md: phase 1 1.002456 GB + 4.92 MB, phase 2 0.500373 GB + 8.66 MB
-    ("decode-bf16", 64, "auto"): 1.5164e9,
-    ("decode-bf16", 64, "tc"): 1.5164e9,
-    # profiles/ffn_tc_int4_decode_T64.md: 268.9 + 4.06 + 133.6 + 5.22 MB
-    ("int4-decode", 64, "auto"): 4.1179e8,
-    ("int4-decode", 64, "tc"): 4.1179e8,
-    # profiles/ffn_tc_int4_prefill_T1024.md: 315.8 + 11.4 + 146.5 + 52.1 MB
-    ("int4-prefill", 1024, "auto"): 5.2580e8,
-    ("int4-prefill", 1024, "tc"): 5.2580e8,
+    # profiles/ffn_tc_dram_traffic.md (current kernels): read + write of both launches
+    ("decode-bf16", 64, "auto"): 1.5134e9,
+    ("decode-bf16", 64, "tc"): 1.5134e9,
+    ("int4-decode", 64, "auto"): 4.0771e8,
+    ("int4-decode", 64, "tc"): 4.0771e8,
+    ("int4-prefill", 1024, "auto"): 5.2211e8,
+    ("int4-prefill", 1024, "tc"): 5.2211e8,
 }
 
 # routes from which the library's AUTO path takes the tensor-core FFN (bf16, int8,

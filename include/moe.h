@@ -168,7 +168,8 @@ MOE_API moe_status moe_route_min_weight(int32_t *ids, float *w, const int32_t *s
  * route, -1 for a dropped route).  Routes whose id is outside [0,E) are
  * dropped.  hits (uint32 [E], nullable) is incremented by counts (the
  * per-layer expert-hit histogram, expert_pool.rs count_hits).  One CTA; uses
- * 32*E*4 + 8 KiB of shared memory.
+ * 32*E*4 + 8 KiB of shared memory.  T == 0 is the empty grouping: counts and
+ * offsets, where given, are set to zero (nothing else is touched).
  */
 MOE_API moe_status moe_permute(const int32_t *ids, int32_t T, int32_t k, int32_t E, int32_t *counts,
                        int32_t *offsets, int32_t *sorted_route, int32_t *route_pos, uint32_t *hits,
@@ -352,6 +353,64 @@ MOE_API int32_t moe_should_refresh(int32_t offload_enabled, int32_t mode_refresh
  * layers is 0). */
 MOE_API int64_t moe_budget_from_vram(int64_t free_bytes, int64_t reserve_bytes, int64_t expert_bytes,
                              int64_t layers, int64_t max_per_layer, int64_t E);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism across GPUs.  Rank d of N holds local experts
+ * [d*El, (d+1)*El) of a layer, El = E / N (E a multiple of N); one process per
+ * GPU.  This is the multi-GPU form of the pages' remote-expert runtime
+ * (Winery-Strata remote_experts.cpp: a secondary GPU owns a claimed subset of
+ * the experts; RemoteExperts::begin stages the rows routed to it and
+ * RemoteExperts::finish returns the compact result rows to their routes).
+ * Per layer call, on every rank:
+ *   1. moe_route_topk + moe_permute over all E experts.  The expert-sorted rows
+ *      for rank d are the contiguous range [offsets[d*El], offsets[(d+1)*El]).
+ *   2. moe_gather_rows(x, index = sorted_route, divisor = k) packs the routed
+ *      tokens' rows in that order.
+ *   3. An all-to-all of counts (El per rank pair) gives recv_counts [N][El];
+ *      moe_ep_splits turns both into the row splits of the exchanges.
+ *   4. An all-to-all of the packed rows (splits from step 3).
+ *   5. The owner labels the received rows with moe_ep_recv_ids, groups them
+ *      with moe_permute (k = 1, E = El), runs moe_grouped_ffn on its own El
+ *      experts, and puts the fp32 result rows back in arrival order with
+ *      moe_gather_rows(rows, index = route_pos, divisor = 1).
+ *   6. The reverse all-to-all returns them; they land in the sender's sorted
+ *      order, where one GPU's moe_grouped_ffn would have written them.
+ *   7. moe_combine.
+ * The exchanges are the caller's (NCCL all-to-all); nothing here waits on
+ * another GPU.
+ */
+
+/*
+ * dst row i = src row (index[i] / divisor) for i in [0, n), copied as
+ * row_bytes bytes; rows whose index is negative or points at or past src_rows
+ * are left untouched.  src [src_rows][row_bytes] and dst [n][row_bytes] are
+ * device memory, 16-byte aligned; row_bytes a positive multiple of 16;
+ * divisor >= 1.  Errors: MOE_ERR_INVALID_ARG (launches nothing).
+ */
+MOE_API moe_status moe_gather_rows(const void *src, int32_t src_rows, int32_t row_bytes, const int32_t *index,
+                                   int32_t n, int32_t divisor, void *dst, moe_stream_t stream);
+
+/*
+ * Local expert of each received row: rows arrive grouped by source rank s and,
+ * inside a source, by local expert e, recv_counts[s*El + e] rows each
+ * (recv_counts int32 [N][El], device).  ids int32 [n] (device) gets e for
+ * every row below the total of recv_counts, -1 for the rest.  N*El <= 1024.
+ * Negative counts are read as 0.
+ */
+MOE_API moe_status moe_ep_recv_ids(const int32_t *recv_counts, int32_t N, int32_t El, int32_t *ids, int32_t n,
+                                   moe_stream_t stream);
+
+/*
+ * Row splits of the two row exchanges (host, pure CPU).  counts: HOST [E], this
+ * rank's routes per expert (moe_permute's counts); recv_counts: HOST [N][El],
+ * what every source sends here per local expert.  send_rows[d] = rows this rank
+ * sends to rank d = sum of counts over d's experts; recv_rows[s] = rows it
+ * receives from s = sum of recv_counts[s].  The reverse exchange swaps the two.
+ * Errors: MOE_ERR_INVALID_ARG if E is not a multiple of N, a count is negative
+ * or a total does not fit in int32.
+ */
+MOE_API moe_status moe_ep_splits(const int32_t *counts, int32_t E, const int32_t *recv_counts, int32_t N,
+                                 int32_t *send_rows, int32_t *recv_rows);
 
 #ifdef __cplusplus
 }

@@ -38,6 +38,7 @@ EXPORTS = [
     "moe_pack_expert", "moe_copy_to_slots", "moe_refresh_target", "moe_apply_placement",
     "moe_should_refresh", "moe_budget_from_vram", "moe_grouped_ffn_noalloc", "moe_take_device_errors",
     "moe_route_min_weight", "moe_router_topk", "moe_hits_window", "moe_refresh_device", "moe_promote_copies",
+    "moe_gather_rows", "moe_ep_recv_ids", "moe_ep_splits",
 ]
 
 
@@ -86,6 +87,9 @@ _SIG = {
     "moe_hits_window": (i32, [P, i32, i32, P]),
     "moe_refresh_device": (i32, [P, i32, i32, P, i32, P, P, P]),
     "moe_promote_copies": (i32, [P, P, u64, P, P, i32, P]),
+    "moe_gather_rows": (i32, [P, i32, i32, P, i32, i32, P, P]),
+    "moe_ep_recv_ids": (i32, [P, i32, i32, P, i32, P]),
+    "moe_ep_splits": (i32, [P, i32, P, i32, P, P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -403,6 +407,46 @@ def moe_grouped_ffn_noalloc(layer: MoeLayer, x: torch.Tensor, k: int, counts, of
                                         _dev(sorted_route, torch.int32, "sorted_route"),
                                         _dev(rows, torch.float32, "rows"), _stream(stream)))
     return rows
+
+
+def moe_gather_rows(src: torch.Tensor, index: torch.Tensor, divisor: int = 1, dst: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """dst[i] = src[index[i] // divisor] for the rows of a 2-D tensor (rows with a
+    negative or out-of-range index are left as they are in dst)."""
+    n = index.numel()
+    if dst is None:
+        dst = torch.empty((max(n, 1), src.shape[1]), dtype=src.dtype, device=src.device)
+    row_bytes = src.shape[1] * src.element_size()
+    if dst.shape[1] * dst.element_size() != row_bytes or dst.shape[0] < n:
+        raise ValueError("dst must have at least index.numel() rows of the same size as src's")
+    _check(_lib.moe_gather_rows(_dev(src, None, "src"), src.shape[0], row_bytes, _dev(index, torch.int32, "index"),
+                                n, int(divisor), _dev(dst, None, "dst"), _stream(stream)))
+    return dst[:n] if dst.shape[0] != n else dst
+
+
+def moe_ep_recv_ids(recv_counts: torch.Tensor, n: int, ids: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Local expert id (int32 [n]) of each received row; recv_counts int32 [N, El]."""
+    N, El = recv_counts.shape
+    if ids is None:
+        ids = torch.empty(max(n, 1), dtype=torch.int32, device=recv_counts.device)[:n]
+    _check(_lib.moe_ep_recv_ids(_dev(recv_counts, torch.int32, "recv_counts"), N, El, _dev(ids, torch.int32, "ids"),
+                                int(n), _stream(stream)))
+    return ids
+
+
+def moe_ep_splits(counts: np.ndarray, recv_counts: np.ndarray):
+    """Host: (send_rows, recv_rows), int32 [N] each, from this rank's counts [E]
+    and the received per-expert counts [N, El]."""
+    c, pc = _host(np.ravel(counts), np.int32)
+    r, pr = _host(recv_counts, np.int32)
+    if r.ndim != 2 or r.shape[0] * r.shape[1] != c.size:
+        raise ValueError("recv_counts must be [N, E / N]")
+    N = r.shape[0]
+    send = np.zeros(N, np.int32)
+    recv = np.zeros(N, np.int32)
+    _check(_lib.moe_ep_splits(pc, c.size, pr, N, send.ctypes.data_as(ctypes.c_void_p),
+                              recv.ctypes.data_as(ctypes.c_void_p)))
+    return send, recv
 
 
 # ------------------------------------------------------------------ helpers

@@ -168,7 +168,14 @@ moe_status moe_permute(const int32_t *ids, int32_t T, int32_t k, int32_t E, int3
     moe_status st = check_shape(E, k, 64, 64);
     if (st != MOE_OK) return st;
     if ((st = check_tk(T, k)) != MOE_OK) return st;
-    if (T == 0) return MOE_OK;
+    if (T == 0) {
+        // an empty grouping: zero counts and offsets where the caller gave them
+        cudaError_t e = cudaSuccess;
+        if (counts) e = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), (cudaStream_t)stream);
+        if (e == cudaSuccess && offsets)
+            e = cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), (cudaStream_t)stream);
+        return cuda_status(e, "moe_permute: clearing counts and offsets");
+    }
     CHECK_ARG(ids && counts && offsets && sorted_route && route_pos, "moe_permute: NULL pointer");
     return cuda_status(launch_permute(ids, T * k, E, counts, offsets, sorted_route, route_pos, hits,
                                       (cudaStream_t)stream),

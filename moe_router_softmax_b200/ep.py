@@ -153,7 +153,9 @@ class ExpertParallelLayer:
 
 def local_layer_of(layer: MoeLayer, rank: int, world: int) -> MoeLayer:
     """The rank's share of a layer whose E blobs are all in `layer.home`: a view of
-    its El consecutive blobs (no copy)."""
+    its El consecutive blobs (no copy).  A rank that should hold only its own
+    experts builds them directly instead: make_layer(fmt, w13[d*El:(d+1)*El],
+    w2[d*El:(d+1)*El])."""
     El = layer.E // world
     eb = layer.expert_bytes
     home = layer.home[rank * El * eb:(rank + 1) * El * eb]

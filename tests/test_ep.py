@@ -26,6 +26,7 @@ sys.path.insert(0, os.path.join(ROOT, "tests"))
 import oracle  # noqa: E402
 import synthetic as syn  # noqa: E402
 import moe_router_softmax_b200 as moe  # noqa: E402
+from ep_support import _bits, host_ops, lockstep  # noqa: E402
 
 
 # ------------------------------------------------------------------ splits
@@ -98,60 +99,46 @@ def test_ep_layer_checks_the_partition():
         ExpertParallelLayer(local, 8, 2, 2)
 
 
-# ------------------------------------------------------- host stand-ins
+def _host_local_layer(full, fmt, rank, El, H, I):
+    eb = full.expert_bytes
+    return oracle.Layer(fmt, El, H, I, full.home[rank * El * eb:(rank + 1) * El * eb].copy())
 
-def _bits(x: torch.Tensor) -> np.ndarray:
-    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
 
+@pytest.mark.parametrize("seed", range(8))
+def test_ep_lockstep_on_host_equals_one_process_oracle(seed):
+    """Random partitions (N in 1..8, El in 1..3), token counts (0 included), k and
+    skewed logits, every rank in one process: each rank's output equals the
+    one-process oracle bit for bit, and the owners' hits add up to the global
+    histogram."""
+    import gpu_support as gs
+    from moe_router_softmax_b200.ep import ExpertParallelLayer
 
-def host_ops(E_full_layer_fmt):
-    """Host versions of the kernels with the binding's signatures (test only)."""
-
-    def route_topk(logits, k):
-        ids, w = oracle.route_topk(logits.numpy(), k)
-        return torch.from_numpy(ids), torch.from_numpy(w)
-
-    def permute(ids, E, hits=None):
-        c, o, s, p = oracle.permute(ids.numpy(), E)
-        if hits is not None:
-            hits += torch.from_numpy(c.astype(np.int64)).to(hits.dtype)
-        return tuple(torch.from_numpy(a) for a in (c, o, s, p))
-
-    def gather_rows(src, index, divisor=1):
-        idx = index.long()
-        out = torch.zeros((idx.numel(), src.shape[1]), dtype=src.dtype)
-        ok = (idx >= 0) & (idx // divisor < src.shape[0])
-        out[ok] = src[idx[ok] // divisor]
-        return out
-
-    def recv_ids(recv_counts, n):
-        N, El = recv_counts.shape
-        lab = np.repeat(np.tile(np.arange(El, dtype=np.int32), N), recv_counts.numpy().ravel().clip(0))
-        out = np.full(n, -1, np.int32)
-        out[:min(n, lab.size)] = lab[:n]
-        return torch.from_numpy(out)
-
-    def grouped_ffn(layer, x, k, counts, offsets, sorted_route):
-        xb = _bits(x)
-        off = offsets.numpy()
-        sr = sorted_route.numpy()
-        rows = np.zeros((sr.size, layer.H), np.float32)
-        for e in range(layer.E):
-            for i in range(off[e], off[e + 1]):
-                rows[i] = oracle.expert_ffn(layer, e, xb[sr[i] // k]).astype(np.float32)
-        return torch.from_numpy(rows)
-
-    def combine(rows, route_pos, w):
-        T, k = w.shape
-        rp = route_pos.numpy()
-        r = np.zeros((T * k, rows.shape[1]), np.float64)
-        r[rp >= 0] = rows.numpy()[rp[rp >= 0]].astype(np.float64)
-        ids = np.where(rp.reshape(T, k) >= 0, 0, -1).astype(np.int32)
-        return torch.from_numpy(oracle.combine(r, ids, w.numpy(), 1))
-
-    return SimpleNamespace(moe_route_topk=route_topk, moe_permute=permute, moe_gather_rows=gather_rows,
-                           moe_ep_recv_ids=recv_ids, moe_ep_splits=moe.moe_ep_splits, moe_grouped_ffn=grouped_ffn,
-                           moe_combine=combine)
+    rng = np.random.default_rng(seed)
+    N = [1, 2, 3, 4, 8, 2, 5, 3][seed]
+    El = int(rng.integers(1, 4))
+    E, H, I = N * El, 64, 64
+    k = int(rng.integers(1, min(E, 4) + 1))
+    fmt = [oracle.BF16, oracle.INT8, oracle.INT4][seed % 3]
+    w13, w2 = syn.expert_weights(E, H, I, seed=seed)
+    full = gs.oracle_layer_for(fmt, w13, w2)
+    eps = [ExpertParallelLayer(_host_local_layer(full, fmt, d, El, H, I), E, d, N, ops=host_ops()) for d in range(N)]
+    Ts = [int(t) for t in rng.integers(0, 7, size=N)]
+    bias = rng.normal(0.0, 2.0, size=E).astype(np.float32)       # some experts, and so some owners, favoured
+    xs = [torch.from_numpy(syn.activations(T, H, seed=10 * seed + d).view(np.int16)).view(torch.bfloat16)
+          for d, T in enumerate(Ts)]
+    lgs = [np.ascontiguousarray(syn.router_logits(T, E, "normal", seed=20 * seed + d) + bias) for d, T in enumerate(Ts)]
+    hits = [torch.zeros(El, dtype=torch.int64) for _ in range(N)]
+    ys, sts = lockstep(eps, [torch.from_numpy(g) for g in lgs], xs, k, hits)
+    all_ids = []
+    for d in range(N):
+        ids, w = oracle.route_topk(lgs[d], k)
+        all_ids.append(ids.ravel())
+        rows = oracle.ffn_routes(full, _bits(xs[d]), ids).astype(np.float32).astype(np.float64)
+        assert np.array_equal(ys[d].numpy(), oracle.combine(rows, ids, w, E)), d
+        assert sum(sts[d].send_rows) == Ts[d] * k
+    assert sum(sum(st.recv_rows) for st in sts) == sum(Ts) * k
+    want = np.bincount(np.concatenate(all_ids + [np.zeros(0, np.int64)]).astype(np.int64), minlength=E)
+    assert np.concatenate([h.numpy() for h in hits]).tolist() == want.tolist()
 
 
 def _case(fmt, E, H, I, rank, T, kind):
@@ -178,7 +165,7 @@ def _ep_worker(rank, world, port, fmt, kind, q):
         El = E // world
         eb = full.expert_bytes
         local = oracle.Layer(fmt, El, H, I, full.home[rank * El * eb:(rank + 1) * El * eb].copy())
-        ep = ExpertParallelLayer(local, E, rank, world, TorchExchange(), ops=host_ops(fmt))
+        ep = ExpertParallelLayer(local, E, rank, world, TorchExchange(), ops=host_ops())
         hits = torch.zeros(El, dtype=torch.int64)
         y = ep.forward(logits, x, k, hits=hits).numpy()
         ids, w = oracle.route_topk(logits.numpy(), k)

@@ -20,6 +20,7 @@ import oracle
 import synthetic as syn
 import moe_router_softmax_b200 as moe
 from moe_router_softmax_b200.ep import ExpertParallelLayer, TorchExchange, local_layer_of
+from ep_support import lockstep
 from gpu_support import (FFN_TOL, bf16_dev_to_f64, device_weights_from_host, host_bits, oracle_blob,
                          oracle_layer_for, rel_err)
 
@@ -72,30 +73,6 @@ def test_permute_of_no_tokens_is_the_empty_grouping():
 
 
 # ------------------------------------------------------ lockstep ranks
-
-def lockstep(eps, logits, xs, k, hits=None):
-    """One layer call of every rank in `eps`; the all-to-alls are device copies."""
-    N, El, H = len(eps), eps[0].El, eps[0].H
-    sts = [ep.begin(lg, x, k) for ep, lg, x in zip(eps, logits, xs)]
-    for d, st in enumerate(sts):
-        st.recv_counts = torch.stack([sts[s].counts.view(N, El)[d] for s in range(N)]).contiguous()
-    for ep, st in zip(eps, sts):
-        ep.plan(st)
-    send_off = [np.concatenate([[0], np.cumsum(st.send_rows)]).astype(int) for st in sts]
-    for d, st in enumerate(sts):
-        parts = [sts[s].xs[send_off[s][d]:send_off[s][d + 1]] for s in range(N)]
-        st.xr = torch.cat(parts).contiguous()
-    for d, (ep, st) in enumerate(zip(eps, sts)):
-        ep.serve(st, None if hits is None else hits[d])
-    recv_off = [np.concatenate([[0], np.cumsum(st.recv_rows)]).astype(int) for st in sts]
-    for s, st in enumerate(sts):
-        st.rows_back = torch.zeros((max(st.T * k, 1), H), dtype=torch.float32, device=DEV)
-        parts = [sts[d].rows_out[recv_off[d][s]:recv_off[d][s + 1]] for d in range(N)]
-        n = sum(p.shape[0] for p in parts)
-        if n:
-            st.rows_back[:n] = torch.cat(parts)
-    return [ep.finish(st) for ep, st in zip(eps, sts)], sts
-
 
 def _dev_bf16(bits):
     return torch.from_numpy(bits.view(np.int16)).to(DEV).view(torch.bfloat16)

@@ -16,12 +16,13 @@ come back only after 29 other layers' worth of traffic.  The batches of 1 and
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--config decode-bf16|decode-int8|int4-decode|int4-prefill|tiny]
-                  [--tokens T]
+                  [--tokens T] [--parallel replicas|ep]
 
-Multi-GPU (N > 1, launched by torchrun): the layer does not shard across GPUs
-in this build, so every rank runs an independent replica of the same
-workload (weak scaling, no collective on the data path); the timing is the
-max over ranks.
+Multi-GPU (N > 1, launched by torchrun): by default every rank runs an
+independent replica of the same workload (weak scaling, no collective on the
+data path); the timing is the max over ranks.  --parallel ep splits the experts
+over the ranks instead (each rank routes its own tokens; NCCL all-to-all
+dispatch and return).
 
 --impl reference times the CPU oracle (plain C, every host core) on a bounded
 sample of the same workload on rank 0; it is the baseline, not the target.
@@ -89,6 +90,9 @@ def parse():
                     help="stack30: placement refresh on the device (graph-captured, copies overlapped) or on the host")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"],
                     help="grouped-FFN kernels: AUTO picks by routes per call")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
+                    help="N > 1: independent replicas (default), or expert parallelism (each rank holds E/N "
+                         "experts, NCCL all-to-all dispatch and return)")
     return ap.parse_args()
 
 
@@ -564,6 +568,8 @@ def main():
         return reference_arm(args, fmt_name, kind, T, E, H, I, k, world, rank)
     if args.config == "stack30":
         return stack_main(args, T, E, H, I, k, world, rank, local)
+    if args.parallel == "ep":
+        return ep_main(args, fmt_name, kind, T, E, H, I, k, world, rank, local)
 
     import torch
 
@@ -716,6 +722,91 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------ expert parallelism
+
+def ep_main(args, fmt_name, kind, T, E, H, I, k, world, rank, local):
+    """Expert parallelism: rank d holds experts [d*E/N, (d+1)*E/N) of each of the
+    rotated layer copies and routes its own T tokens per step; routed rows go to
+    their owners and back by NCCL all-to-all.  Eager steps (the split sizes are read
+    on the host every step); timed on the device, max over ranks."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as tdist
+
+    import moe_router_softmax_b200 as moe
+    from moe_router_softmax_b200.ep import ExpertParallelLayer, TorchExchange
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if "MASTER_ADDR" not in os.environ:          # one process without torchrun
+        sock = socket.socket()
+        sock.bind(("127.0.0.1", 0))
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(sock.getsockname()[1]), RANK="0",
+                          WORLD_SIZE="1")
+        sock.close()
+    tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if E % world:
+        raise SystemExit(f"E={E} is not a multiple of {world} ranks")
+    El = E // world
+    n_layers = args.layers if args.config != "tiny" else 2
+    layers = build_layers(moe, torch, fmt_name, El, H, I, n_layers, dev, seed=rank)
+    eps = [ExpertParallelLayer(L, E, rank, world, TorchExchange()) for L in layers]
+    batches = make_batches(torch, kind, T, E, H, 8, dev, seed=rank)
+    steps, warmup = args.steps, max(args.warmup, 3)
+
+    def step(i):
+        b = batches[i % len(batches)]
+        return eps[i % n_layers].forward(b[2], b[3], k)
+
+    for i in range(warmup):
+        step(i)
+    clocks = ClockSampler(local)
+    clocks.start()
+    tdist.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        step(warmup + i)
+    t1.record()
+    torch.cuda.synchronize(dev)
+    tdist.barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(tdist, t0.elapsed_time(t1), dev)
+    line = {
+        "metric": "MoE layer tokens/s and expert-weight HBM GB/s (% of roofline) at decode/prefill",
+        "value": round(whole_job_rate(T * steps, world, ms), 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(ms / steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": fmt_name,
+        "data": "synthetic (seeded; Gemma-4-26B-A4B-shaped layer, random weights)",
+        "config": {
+            "workload": f"moe-layer-{fmt_name}-{'prefill' if T > 64 else 'decode'}-T{T}",
+            "experts": E, "hidden": H, "intermediate": I, "top_k": k, "tokens_per_rank": T,
+            "weights": fmt_name, "logits": kind, "layers_rotated": n_layers,
+            "l2": f"inputs larger than L2: each step reads a different one of {n_layers} layer copies "
+                  f"({n_layers * El * moe.moe_expert_bytes(moe.FMT[fmt_name], H, I) / 1e9:.1f} GB per rank)",
+            "parallelism": f"expert parallel x{world} ({El} experts per rank, NCCL all-to-all)",
+        },
+        "roofline": None,
+        "gpu_launches": None,
+        "clocks": clk,
+        "note": "eager steps with one device-to-host read of the split sizes per step",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    tdist.barrier()
+    tdist.destroy_process_group()
 
 
 # ----------------------------------------------------------- the layer stack

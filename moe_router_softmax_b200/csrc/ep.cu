@@ -19,9 +19,9 @@ namespace {
 // dst row i = src row (index[i] / divisor), copied in 16-byte chunks, for
 // 0 <= index[i] / divisor < src_rows; every other row of dst is left as it is.
 // One CTA per row, grid-stride over rows.
-__global__ void __launch_bounds__(128) k_gather_rows(const uint4 *__restrict__ src, int src_rows, int chunks,
-                                                     const int32_t *__restrict__ index, int n, int divisor,
-                                                     uint4 *__restrict__ dst) {
+__global__ void __launch_bounds__(128) k_ep_gather_rows(const uint4 *__restrict__ src, int src_rows, int chunks,
+                                                        const int32_t *__restrict__ index, int n, int divisor,
+                                                        uint4 *__restrict__ dst) {
     pdl_wait();
     pdl_launch_dependents();
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
@@ -115,7 +115,7 @@ moe_status moe_gather_rows(const void *src, int32_t src_rows, int32_t row_bytes,
     cudaError_t e = sm_count(&n_sm);
     if (e == cudaSuccess) {
         const int grid = n < n_sm * 16 ? n : n_sm * 16;
-        e = launch_pdl(k_gather_rows, dim3(grid), dim3(128), 0, (cudaStream_t)stream,
+        e = launch_pdl(k_ep_gather_rows, dim3(grid), dim3(128), 0, (cudaStream_t)stream,
                        static_cast<const uint4 *>(src), (int)src_rows, (int)(row_bytes / 16), index, (int)n,
                        (int)divisor, static_cast<uint4 *>(dst));
     }

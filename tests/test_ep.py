@@ -8,6 +8,8 @@
   the oracle (route, permute, per-route FFN, combine), so each rank's output must
   equal, bit for bit, the oracle's one-process layer on that rank's tokens -- a
   row sent to the wrong owner, or returned to the wrong place, changes it.
+* The same phases for random partitions (1 to 8 ranks) driven in lockstep from
+  one process, with the same host stand-ins and the same bit-exact bar.
 """
 import os
 import sys

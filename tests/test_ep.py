@@ -99,6 +99,8 @@ def test_ep_layer_checks_the_partition():
         ExpertParallelLayer(local, 16, 0, 2)
     with pytest.raises(ValueError, match="rank"):
         ExpertParallelLayer(local, 8, 2, 2)
+    with pytest.raises(RuntimeError, match="exchange"):
+        ExpertParallelLayer(local, 8, 0, 2).forward(None, None, 2)
 
 
 def _host_local_layer(full, fmt, rank, El, H, I):

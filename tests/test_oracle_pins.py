@@ -344,6 +344,64 @@ def test_int4_zero_group():
     assert s[0, 0] == 0 and np.all(q == 0x88)
 
 
+def _torch_bf16_bits(u32: np.ndarray) -> np.ndarray:
+    """fp32 bit patterns -> bf16 bit patterns by torch's own conversion."""
+    f = torch.from_numpy(np.ascontiguousarray(u32, np.uint32).view(np.float32).copy())
+    return f.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_bf16_rounding_matches_torch_conversion():
+    """The oracle's fp32 -> bf16 rounding (it fixes every int4 scale: prain README,
+    'Expert formats', bf16 scale per 64 weights) equals torch's float32 ->
+    bfloat16 conversion bit for bit: exact ties with an even and an odd kept
+    part, one ulp either side of a tie, subnormals, values that round up to
+    +-inf, +-0, +-inf, the largest finite values, and random patterns.  NaN stays
+    NaN.  A truncating or ties-away rounding fails here."""
+    pats = []
+    rng = np.random.default_rng(7)
+    hi = rng.integers(0, 1 << 16, size=3000, dtype=np.uint32)
+    for lo in (0x8000, 0x7FFF, 0x8001, 0x0000, 0xFFFF, 0x0001):
+        pats.append((hi << 16) | lo)                      # ties, both parities of hi; one ulp around them
+    pats.append(rng.integers(0, 1 << 32, size=20000, dtype=np.uint64).astype(np.uint32))
+    sub = rng.integers(1, 0x00800000, size=2000, dtype=np.uint32)
+    pats.append(sub)                                      # positive subnormals
+    pats.append(sub | 0x80000000)                         # negative subnormals
+    pats.append(np.array([0x00008000, 0x00018000, 0x007F8000, 0x007FFFFF, 0x00800000, 0x80008000,
+                          0x7F7F7FFF, 0x7F7F8000, 0x7F7FFFFF, 0x7F7E8000, 0xFF7F8000, 0xFF7FFFFF,
+                          0x7F800000, 0xFF800000, 0x00000000, 0x80000000, 0x3F808000, 0x3F818000],
+                         np.uint32))
+    u = np.concatenate(pats).astype(np.uint32)
+    nan = (u & 0x7FFFFFFF) > 0x7F800000
+    f = u.view(np.float32)
+    got = np.array([oracle.bf16_rne(float(v)) for v in f], np.uint16)
+    ref = _torch_bf16_bits(u)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # the overflow cases really reach infinity, and ties really go to even
+    assert oracle.bf16_rne(struct.unpack("<f", struct.pack("<I", 0x7F7F8000))[0]) == 0x7F80
+    assert oracle.bf16_rne(struct.unpack("<f", struct.pack("<I", 0x3F808000))[0]) == 0x3F80
+    assert oracle.bf16_rne(struct.unpack("<f", struct.pack("<I", 0x3F818000))[0]) == 0x3F82
+    qn = np.array([0x7FC00000, 0xFFC00001, 0x7F800001, 0xFF812345], np.uint32)
+    for v in qn.view(np.float32):
+        b = oracle.bf16_rne(float(v))
+        assert (b & 0x7F80) == 0x7F80 and (b & 0x007F) != 0      # still a NaN
+
+
+def test_int4_candidate_scales_are_torch_rounded():
+    """Every candidate scale of the clip search is the bf16 rounding of the fp32
+    r_i * absmax / 7 (ratios r_i = 0.70, 0.72, ..., 1.00; fp32 multiply, then
+    fp32 divide), recomputed here with torch's float32 arithmetic and its
+    bfloat16 conversion."""
+    for seed in range(6):
+        w64 = syn.normal_bf16((64,), 0.02 * (1 + seed), 41, seed)
+        amax = torch.tensor(float(np.abs(syn.bf16_to_f32(w64)).max()), dtype=torch.float32)
+        s_c, _ = oracle.int4_candidates(w64)
+        for i in range(16):
+            r = torch.tensor((70 + 2 * i) / 100, dtype=torch.float32)
+            t = (r * amax) / torch.tensor(7.0, dtype=torch.float32)
+            want = t.to(torch.bfloat16).to(torch.float32).item()
+            assert struct.pack("<f", float(s_c[i])) == struct.pack("<f", want), (seed, i)
+
+
 # ------------------------------------------------------------------ expert FFN
 
 def _tiny_layer(fmt, E=4, h=128, i=64, seed=0):

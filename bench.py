@@ -43,19 +43,14 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# grouped-FFN kernels from one ncu capture, per workload; None until captured
-# for the kernels as they stand (see profiles/).
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, summed
+# over the grouped-FFN launches of one call) from one-pass ncu captures of the
+# kernels as they stand, keyed by (workload, --path): (bytes, what was captured).
+# A workload without an entry reports null.
 NCU_TRAFFIC_BYTES = {
-    # profiles/ffn_gemv_bf16_T64.md: phase 1 1.0059 GB + 4.04 MB, phase 2 0.5027 GB + 5.28 MB
-    ("decode-bf16", 64, "gemv"): 1.5180e9,
-    # profiles/ffn_tc_dram_traffic.md (current kernels): read + write of both launches
-    ("decode-bf16", 64, "auto"): 1.5134e9,
-    ("decode-bf16", 64, "tc"): 1.5134e9,
-    ("int4-decode", 64, "auto"): 4.0771e8,
-    ("int4-decode", 64, "tc"): 4.0771e8,
-    ("int4-prefill", 1024, "auto"): 5.2211e8,
-    ("int4-prefill", 1024, "tc"): 5.2211e8,
+    ("moe-layer-bf16-decode-T64", "auto"): (1.5134e9, "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum "
+                                                      "--clock-control none: gather + both tcgen05 launches, "
+                                                      "bench.py --config decode-bf16 --quick --layers 2"),
 }
 
 # routes from which the library's AUTO path takes the tensor-core FFN (bf16, int8,
@@ -86,6 +81,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--quick", action="store_true", help="main batch only: no sweep, no e2e, no CPU baseline")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="decode-bf16: skip the int8 / int4 / stack workloads reported under 'configs'")
     ap.add_argument("--stack-refresh", default="device", choices=["device", "host"],
                     help="stack30: placement refresh on the device (graph-captured, copies overlapped) or on the host")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"],
@@ -274,14 +271,16 @@ class Runner:
         return out
 
 
-FFN_SAMPLE_EVERY = 5
+FFN_SAMPLE_EVERY = 1
 
 
 def _capture(torch, runner, first, n):
     """One CUDA graph of n consecutive steps, with an external event pair around
     the grouped-FFN launches of every FFN_SAMPLE_EVERY-th step (event record
-    nodes inside the graph).  An event node between two kernels also cuts their
-    programmatic-launch edge, so only the sampled steps carry them."""
+    nodes inside the graph; every step, so a 20-step run gives 20 pairs).  An
+    event node between two kernels also cuts their programmatic-launch edge: the
+    permute -> FFN and FFN -> combine hand-offs of a sampled step wait for the
+    previous kernel to finish (the FFN's own launches keep theirs)."""
     g = torch.cuda.CUDAGraph()
     sampled = [j for j in range(n) if j % FFN_SAMPLE_EVERY == FFN_SAMPLE_EVERY // 2] or [0]
     evs = {j: (torch.cuda.Event(enable_timing=True, external=True),
@@ -554,6 +553,64 @@ def cpu_baseline(moe, torch, cfg_fmt, layers, batches, T, k, seconds, first_toke
                               "sample": f"{n1} token evaluations, {e1:.1f} s"}}
 
 
+def ffn_roofline(T, k, H, I, eb, distinct, ffn_ms, peaks, traffic):
+    """Roofline object of the grouped FFN (the dominant kernel) for one workload:
+    algorithmic bytes = distinct routed experts x expert_bytes + T*H*2 (x); flops
+    = 2*T*k*3*H*I.  Decode batches (T <= 64) are bound by HBM, the prefill batch
+    by the tensor pipe (against the sustained bf16 peak; its HBM fraction is
+    reported beside it).  `ffn_ms` is the average of the live event pairs."""
+    hbm_peak, _, tf_sust, src = peaks
+    alg_bytes = distinct * eb + T * H * 2
+    gbs = alg_bytes / (ffn_ms / 1e3) / 1e9
+    flops = 2.0 * T * k * 3 * H * I
+    tflops = flops / (ffn_ms / 1e3) / 1e12
+    tr = None if traffic is None else traffic[0]
+    tr_src = None if traffic is None else traffic[1]
+    if T > 64:
+        return {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_sust, "unit": "TFLOP/s",
+                "frac": round(tflops / tf_sust, 4), "traffic": tr, "traffic_capture": tr_src,
+                "peak_source": f"{src} sustained bf16 (bf16_tflops_sustained)",
+                "alg_flops_per_launch": flops,
+                "hbm": {"achieved_gbs": round(gbs, 1), "peak": hbm_peak, "frac": round(gbs / hbm_peak, 4),
+                        "alg_bytes_per_launch": int(alg_bytes)},
+                "avg_launch_us": round(ffn_ms * 1e3, 2)}
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(gbs / hbm_peak, 4), "traffic": tr, "traffic_capture": tr_src,
+            "peak_source": f"{src} (hbm_gbs)", "alg_bytes_per_launch": int(alg_bytes),
+            "avg_launch_us": round(ffn_ms * 1e3, 2)}
+
+
+def run_layer_config(ctx, layers, kind, T, name, seed=0):
+    """One layer workload: T tokens per step over the rotated layer copies, steps
+    replayed from CUDA graphs with an event pair around every grouped-FFN call.
+    Returns (summary dict, runner, step ms list)."""
+    moe, torch, args, dev, dist, world = ctx["moe"], ctx["torch"], ctx["args"], ctx["dev"], ctx["dist"], ctx["world"]
+    L0 = layers[0]
+    E, H, I, k = L0.E, L0.H, L0.I, ctx["k"]
+    batches = make_batches(torch, kind, T, E, H, 8, dev, seed=seed)
+    runner = Runner(moe, torch, layers, batches, T, k, dev, ctx["path"])
+    distinct = runner.distinct_experts()
+    ms, ffn_ms = time_steps(torch, runner, args.steps, args.warmup, dist)
+    ms = max_over_ranks(dist, ms, dev)
+    eb = L0.expert_bytes
+    d_avg = sum(distinct[(args.warmup + i) % len(distinct)] for i in range(args.steps)) / args.steps
+    f_avg = sum(ffn_ms) / len(ffn_ms)
+    fmt_name = {0: "bf16", 1: "int8", 2: "int4"}[L0.fmt]
+    workload = f"moe-layer-{fmt_name}-{'prefill' if T > 64 else 'decode'}-T{T}"
+    traffic = NCU_TRAFFIC_BYTES.get((workload, args.path))
+    out = {
+        "workload": workload, "logits": kind,
+        "tokens_per_s": round(world * T * args.steps / (ms / 1e3), 1),
+        "us_per_step": round(ms / args.steps * 1e3, 2),
+        "ffn_us": round(f_avg * 1e3, 2), "ffn_event_pairs": len(ffn_ms),
+        "distinct_experts": round(d_avg, 2),
+        "layer_hbm_gbs": round((d_avg * eb + T * H * 4 + T * E * 4) / (ms / args.steps / 1e3) / 1e9, 1),
+        "roofline": ffn_roofline(T, k, H, I, eb, d_avg, f_avg, ctx["peaks"], traffic),
+        "gpu_launches": runner.launches_per_step() * args.steps,
+    }
+    return out, runner, ms, batches
+
+
 def main():
     args = parse()
     fmt_name, kind, T0, sweep = CONFIGS[args.config]
@@ -587,51 +644,24 @@ def main():
         dist = tdist
 
     n_layers = args.layers if args.config != "tiny" else 2
-    layers = build_layers(moe, torch, fmt_name, E, H, I, n_layers, dev)
-    batches = make_batches(torch, kind, T, E, H, 8, dev)
     path = {"auto": moe.MOE_FFN_AUTO, "gemv": moe.MOE_FFN_GEMV, "tc": moe.MOE_FFN_TC}[args.path]
-    runner = Runner(moe, torch, layers, batches, T, k, dev, path)
-    distinct = runner.distinct_experts()
+    peaks = measured_peaks()
+    ctx = {"moe": moe, "torch": torch, "args": args, "dev": dev, "dist": dist, "world": world, "k": k,
+           "path": path, "peaks": peaks}
+    layers = build_layers(moe, torch, fmt_name, E, H, I, n_layers, dev)
 
     clocks = ClockSampler(local)
     clocks.start()
-    ms, ffn_ms = time_steps(torch, runner, args.steps, args.warmup, dist)
+    head, runner, ms, batches = run_layer_config(ctx, layers, kind, T, "headline")
     clk = clocks.stop()
-
-    ms = max_over_ranks(dist, ms, dev)
     ms_step = ms / args.steps
     value = whole_job_rate(T * args.steps, world, ms)
-
-    # roofline of the dominant kernel (the grouped FFN: two launches per step)
     eb = moe.moe_expert_bytes(moe.FMT[fmt_name], H, I)
-    avg_distinct = sum(distinct[(args.warmup + i) % len(distinct)] for i in range(args.steps)) / args.steps
-    alg_bytes = avg_distinct * eb + T * H * 2
-    ffn_avg_ms = sum(ffn_ms) / len(ffn_ms)
-    achieved = alg_bytes / (ffn_avg_ms / 1e3) / 1e9
-    hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
-    flops = 2.0 * T * k * 3 * H * I
-    tflops = flops / (ffn_avg_ms / 1e3) / 1e12
-    tensor_bound = T > 64
-    traffic = NCU_TRAFFIC_BYTES.get((args.config, T, args.path))
-    layer_bytes = avg_distinct * eb + T * H * 2 * 2 + T * E * 4
 
     sweep_out = {}
     for Ts in ([] if args.quick else sweep):
-        b2 = make_batches(torch, kind, Ts, E, H, 8, dev, seed=Ts)
-        r2 = Runner(moe, torch, layers, b2, Ts, k, dev, path)
-        d2 = r2.distinct_experts()
-        ms2, ffn2 = time_steps(torch, r2, args.steps, args.warmup, dist)
-        ms2 = max_over_ranks(dist, ms2, dev)
-        dd = sum(d2) / len(d2)
-        f2 = sum(ffn2) / len(ffn2)
-        sweep_out[f"T{Ts}"] = {
-            "tokens_per_s": round(world * Ts * args.steps / (ms2 / 1e3), 1),
-            "us_per_step": round(ms2 / args.steps * 1e3, 2),
-            "ffn_us": round(f2 * 1e3, 2),
-            "distinct_experts": round(dd, 2),
-            "ffn_hbm_gbs": round((dd * eb + Ts * H * 2) / (f2 / 1e3) / 1e9, 1),
-            "ffn_frac_of_hbm": round((dd * eb + Ts * H * 2) / (f2 / 1e3) / 1e9 / hbm_peak, 4),
-        }
+        s_out, _, _, _ = run_layer_config(ctx, layers, kind, Ts, f"T{Ts}", seed=Ts)
+        sweep_out[f"T{Ts}"] = s_out
 
     kernels = None
     if not args.quick and args.config != "tiny":
@@ -643,7 +673,7 @@ def main():
     if args.config != "tiny":
         for Tr in ([T] if args.quick else sorted({1, T, 1024})):
             r = time_router(torch, moe, Tr, E, H, k, dev)
-            r["frac_of_hbm"] = round(r["hbm_gbs"] / hbm_peak, 4)
+            r["frac_of_hbm"] = round(r["hbm_gbs"] / peaks[0], 4)
             router[f"T{Tr}"] = r
 
     eager_steps = min(args.steps, 500)
@@ -656,6 +686,13 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
         cpu = cpu_baseline(moe, torch, fmt_name, layers, batches, T, k, args.cpu_seconds)
+
+    # the other workloads of the same layer shape, each with its own roofline:
+    # int8 decode with skewed routing, int4 decode and prefill, and the 30-layer
+    # stacks behind cache slots (int4 and bf16 both resident)
+    configs = None
+    if args.config == "decode-bf16" and not args.quick and not args.headline_only:
+        configs = other_configs(ctx, layers, E, H, I, k, n_layers)
 
     line = {
         "metric": "MoE layer tokens/s and expert-weight HBM GB/s (% of roofline) at decode/prefill",
@@ -671,7 +708,7 @@ def main():
         "dtype": fmt_name,
         "data": "synthetic (seeded; Gemma-4-26B-A4B-shaped layer, random weights)",
         "config": {
-            "workload": f"moe-layer-{fmt_name}-{'prefill' if T > 64 else 'decode'}-T{T}",
+            "workload": head["workload"],
             "ffn_path": args.path,
             "experts": E, "hidden": H, "intermediate": I, "top_k": k, "tokens": T,
             "weights": fmt_name, "logits": kind, "layers_rotated": n_layers,
@@ -679,32 +716,12 @@ def main():
                   f"({n_layers * E * eb / 1e9:.1f} GB of expert blobs)",
             "parallelism": f"replicas x{world}",
         },
-        "layer_hbm_gbs": round(layer_bytes / (ms_step / 1e3) / 1e9, 1),
-        "roofline": ({
-            "bound": "tensor",
-            "kernel": "grouped FFN on tcgen05 (gather, w13+GELU gate, w2; 3 launches)",
-            "achieved": round(tflops, 1),
-            "peak": tf_sust,
-            "peak_source": f"{peak_src} sustained bf16 (MEASURED_PEAKS.json bf16_tflops_sustained)",
-            "unit": "TFLOP/s",
-            "frac": round(tflops / tf_sust, 4),
-            "traffic": traffic,
-            "alg_flops_per_launch": flops,
-            "hbm": {"achieved_gbs": round(achieved, 1), "peak": hbm_peak, "frac": round(achieved / hbm_peak, 4)},
-            "avg_launch_us": round(ffn_avg_ms * 1e3, 2),
-        } if tensor_bound else {
-            "bound": "hbm",
-            "kernel": "grouped FFN (tcgen05: gather, w13+GELU gate, w2; GEMV: w13+GELU gate, w2)",
-            "achieved": round(achieved, 1),
-            "peak": hbm_peak,
-            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
-            "unit": "GB/s",
-            "frac": round(achieved / hbm_peak, 4),
-            "traffic": traffic,
-            "alg_bytes_per_launch": int(alg_bytes),
-            "avg_launch_us": round(ffn_avg_ms * 1e3, 2),
-        }),
+        "layer_hbm_gbs": head["layer_hbm_gbs"],
+        "roofline": dict(head["roofline"], kernel="grouped FFN (tcgen05: gather, w13+GELU gate, w2; "
+                                                 "GEMV: w13+GELU gate, w2)",
+                         ffn_event_pairs=head["ffn_event_pairs"]),
         "sweep": sweep_out,
+        "configs": configs,
         "router_topk": router,
         "kernels": kernels,
         "eager": None if args.quick else {
@@ -713,7 +730,7 @@ def main():
             "note": "the same steps launched from Python one by one (no CUDA graph)"},
         "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": runner.launches_per_step() * args.steps,
+        "gpu_launches": head["gpu_launches"],
         "clocks": clk,
         "cpu_baseline": cpu,
     }
@@ -722,6 +739,62 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def other_configs(ctx, bf16_layers, E, H, I, k, n_layers):
+    """int8 decode (skewed logits) at T = 1, 8, 64; int4 decode T = 64 and prefill
+    T = 1024; the 30-layer int4 and bf16 stacks at T = 1, 8, 64.  Each layer
+    workload runs the same --steps/--warmup with its own live FFN events."""
+    moe, torch, dev = ctx["moe"], ctx["torch"], ctx["dev"]
+    out = {}
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    l8 = build_layers(moe, torch, "int8", E, H, I, n_layers, dev)
+    for Ts in (64, 8, 1):
+        out[f"int8-decode-T{Ts}"] = run_layer_config(ctx, l8, "biased", Ts, f"int8-T{Ts}", seed=100 + Ts)[0]
+    del l8
+    torch.cuda.empty_cache()
+    l4 = build_layers(moe, torch, "int4", E, H, I, n_layers, dev)
+    out["int4-decode-T64"] = run_layer_config(ctx, l4, "normal", 64, "int4-T64", seed=200)[0]
+    out["int4-prefill-T1024"] = run_layer_config(ctx, l4, "normal", 1024, "int4-T1024", seed=300)[0]
+    out["stack30"] = stack_configs(ctx, l4, bf16_layers, E, H, I, k)
+    del l4
+    torch.cuda.empty_cache()
+    out["clocks"] = clocks.stop()
+    return out
+
+
+def stack_configs(ctx, l4, l16, E, H, I, k):
+    """The 30-layer stacks of the layers already in HBM (int4 and bf16 both
+    resident), 18 cache slots per layer, Zipf(1.1) routing, device placement
+    refresh every 8 steps, 256 decode steps at T = 1, 8, 64."""
+    moe, torch, dev = ctx["moe"], ctx["torch"], ctx["dev"]
+    L, slots, steps = min(30, len(l4), len(l16)), 18, 256
+    s4 = Stack(moe, torch, "int4", E, H, I, L, slots, dev, homes=l4[:L])
+    s16 = Stack(moe, torch, "bf16", E, H, I, L, slots, dev, homes=l16[:L])
+    hbm = ctx["peaks"][0]
+    out = {"layers": L, "slots_per_layer": slots, "refresh_every": 8, "steps": steps,
+           "refresh": "on the device, promotion copies on a second stream; one CUDA graph per 8-step window"}
+    for name, st in (("int4", s4), ("bf16", s16)):
+        for Ts in (1, 8, 64):
+            ms, n, alg = stack_steps_device(torch, moe, st, Ts, k, steps, 8, seed=11 + Ts, path=ctx["path"])
+            ms = max_over_ranks(ctx["dist"], ms, dev)
+            ms_step = ms / n
+            share = st.stats["resident_route_share"]
+            out[f"{name}-T{Ts}"] = {
+                "tokens_per_s": round(ctx["world"] * Ts * n / (ms / 1e3), 1), "ms_per_step": round(ms_step, 4),
+                "roofline": {"bound": "hbm", "unit": "GB/s", "peak": hbm,
+                             "achieved": round(alg / (ms_step / 1e3) / 1e9, 1),
+                             "frac": round(alg / (ms_step / 1e3) / 1e9 / hbm, 4),
+                             "alg_bytes_per_step": int(alg),
+                             "note": "whole step of 30 layers (route, permute, FFN, combine, refresh, copies) "
+                                     "against the distinct routed experts' bytes"},
+                "placement": {"refreshes": st.stats["refreshes"], "promotions": st.stats["promotions"],
+                              "demotions": st.stats["demotions"],
+                              "routes_on_resident_slots": round(sum(share) / len(share), 4) if share else None},
+            }
+    del s4, s16
+    return out
 
 
 # ------------------------------------------------------ expert parallelism
@@ -818,9 +891,9 @@ class Stack:
     mirrors the device slot table.  Initial residents are experts 0..slots-1
     (expert_pool.rs, ExpertPool::new)."""
 
-    def __init__(self, moe, torch, fmt_name, E, H, I, L, slots, dev, seed=0):
+    def __init__(self, moe, torch, fmt_name, E, H, I, L, slots, dev, seed=0, homes=None):
         self.moe, self.torch = moe, torch
-        self.homes = build_layers(moe, torch, fmt_name, E, H, I, L, dev, seed=seed)
+        self.homes = homes if homes is not None else build_layers(moe, torch, fmt_name, E, H, I, L, dev, seed=seed)
         self.fmt = moe.FMT[fmt_name]
         self.E, self.H, self.I, self.L, self.slots = E, H, I, L, slots
         self.eb = self.homes[0].expert_bytes
@@ -954,7 +1027,10 @@ def stack_steps_device(torch, moe, stack, T, k, steps, warmup, seed, refresh_eve
     forward), so that a window of `refresh_every` steps is one CUDA graph with
     no host round trip and the copies overlap the following layers' compute.
     `steps` and `warmup` are rounded up to whole windows.  Returns (total ms,
-    steps timed)."""
+    steps timed, algorithmic bytes per timed step: the distinct routed experts'
+    blobs of every layer plus each layer's x, y and logits).  The distinct
+    experts come from a host top-k of the same logits (continuous draws: no
+    ties)."""
     import synthetic as syn
 
     dev = stack.layers[0].home.device
@@ -965,10 +1041,15 @@ def stack_steps_device(torch, moe, stack, T, k, steps, warmup, seed, refresh_eve
     n = steps + warmup
     lg_all = torch.empty((n, L, T, E), dtype=torch.float32, device=dev)
     x_all = torch.empty((n, T, H), dtype=torch.bfloat16, device=dev)
+    distinct = 0
     for st in range(n):
-        lg_all[st] = torch.from_numpy(np.stack([syn.router_logits(T, E, "zipf", seed=seed, layer=l, step=st)
-                                                for l in range(L)])).to(dev)
+        lg_h = np.stack([syn.router_logits(T, E, "zipf", seed=seed, layer=l, step=st) for l in range(L)])
+        if st >= warmup:
+            top = np.argpartition(-lg_h, k - 1, axis=2)[:, :, :k].reshape(L, -1)
+            distinct += sum(np.unique(top[l]).size for l in range(L))
+        lg_all[st] = torch.from_numpy(lg_h).to(dev)
         x_all[st] = torch.from_numpy(syn.activations(T, H, seed=seed, layer=st).view(np.int16)).to(dev).view(torch.bfloat16)
+    alg_step = distinct / steps * stack.eb + L * (T * H * 4 + T * E * 4)
     lg_stage = torch.empty((W, L, T, E), dtype=torch.float32, device=dev)
     x_stage = torch.empty((W, T, H), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(moe.moe_grouped_ffn_workspace(stack.layers[0], T, k), dtype=torch.uint8, device=dev)
@@ -1054,7 +1135,7 @@ def stack_steps_device(torch, moe, stack, T, k, steps, warmup, seed, refresh_eve
     stack.stats = {"refreshes": windows, "promotions": int(a[0]), "demotions": int(a[1]),
                    "resident_route_share": [float(a[2]) / float(a[3])] if a[3] else []}
     del g
-    return t0.elapsed_time(t1), steps
+    return t0.elapsed_time(t1), steps, alg_step
 
 
 def stack_main(args, T, E, H, I, k, world, rank, local):
@@ -1076,7 +1157,7 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
 
     def run_stack(st, Ts, seed):
         if device_refresh:
-            return stack_steps_device(torch, moe, st, Ts, k, steps, warmup, seed=seed, path=path)
+            return stack_steps_device(torch, moe, st, Ts, k, steps, warmup, seed=seed, path=path)[:2]
         return stack_steps(torch, moe, st, Ts, k, steps, warmup, seed=seed, path=path), steps
 
     resident_gb = (sum(h.home.numel() for h in s4.homes) + sum(h.home.numel() for h in s16.homes) +

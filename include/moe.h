@@ -23,6 +23,8 @@
  *    call says "host".  bf16 data is passed as raw 16-bit words (uint16_t).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Device
  *    calls are asynchronous on it; the library never synchronises.
+ *    (moe_stream_t is void * and bf16 is uint16_t so that this header needs no
+ *    CUDA headers; a cudaStream_t and __nv_bfloat16 data pass unchanged.)
  *  - The library never allocates device memory.  Calls that need scratch take
  *    a caller-owned workspace whose size the matching *_workspace() query gives.
  *  - Arguments are checked on the host before any launch.  A bad argument
@@ -77,6 +79,14 @@ typedef enum { MOE_FFN_AUTO = 0, MOE_FFN_GEMV = 1, MOE_FFN_TC = 2 } moe_ffn_path
  * slot_table[e] >= 0, else from   home + e * expert_bytes
  * (remote_experts.cpp: a cached expert is found by slot_of and read from its
  * device slot).  slot_table may be NULL (every expert read from home).
+ * pool_slots is the number of blobs in pool (a pool may hold more slots than
+ * the layer has experts: prain's 540 cache slots are shared by all layers).  It
+ * is an addition to the pages' interface: the slot table lives on the device,
+ * so the kernels need the pool's extent to bound what they read.  Required
+ * (>= 1) with a slot table; ignored without one.  A slot_table entry at or past
+ * pool_slots is refused on the device: the kernels skip that expert's routes
+ * (their output rows are not written) and record the fault for
+ * moe_take_device_errors() (MOE_ERR_CUDA, info = the bad slot id).
  * Blob layout of one expert, row-major, no padding:
  *   bf16: W13[2I][H] bf16 | W2[H][I] bf16
  *   int8: Q13[2I][H] i8 | S13[2I] f32 | Q2[H][I] i8 | S2[H] f32
@@ -92,6 +102,7 @@ typedef struct {
     const void *pool;          /* slot blobs, stride expert_bytes, device; may be NULL if unused */
     const void *home;          /* E blobs, stride expert_bytes, device */
     uint64_t expert_bytes;     /* blob stride: >= moe_expert_bytes(), multiple of 256 */
+    int32_t pool_slots;        /* blobs in pool (>= 1 when slot_table is set) */
 } moe_layer;
 
 /* Library version string and the last error of this thread ("" if none). */
@@ -188,7 +199,13 @@ MOE_API moe_status moe_expert_hits(const int32_t *ids, int64_t n, int32_t E, uin
  *   (h rounded to bf16);  rows[s] = W2_e h  (fp32 accumulate)
  * with gelu_tanh(v) = 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))).
  * rows fp32 [T*k][H] in sorted order; rows past offsets[E] are not written.
- * ws: device workspace of at least moe_grouped_ffn_workspace() bytes.
+ * ws: device workspace of at least moe_grouped_ffn_workspace() bytes.  The
+ * query follows the scratch-size queries of remote_experts.cpp
+ * (moe_hit_grouped_scratch_bytes / native_expert_scratch_bytes: the caller asks
+ * how much scratch a grouped call needs, then owns it): here the larger of the
+ * GEMV kernels' need (h, T*k*I*2 bytes) and the tensor-core kernels' (h plus x
+ * gathered into sorted-route order, T*k*H*2 bytes), so one workspace serves
+ * either path.
  * moe_grouped_ffn_path forces a kernel path (MOE_FFN_GEMV: split-K GEMV
  * kernels; MOE_FFN_TC: tcgen05 tensor-core kernels); MOE_ERR_UNSUPPORTED if
  * the forced path does not handle the format.  Asynchronous on `stream`; the
@@ -211,16 +228,22 @@ MOE_API moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *
  * Grouped FFN without a caller-provided workspace, for callers that cannot
  * allocate device memory (a plugin or serving runtime that passes the library
  * only its input and output buffers, or a loop that must never call
- * cudaMalloc).  Same arguments and results as moe_grouped_ffn, minus ws.  The
- * pages have no counterpart: this is a library convenience.
+ * cudaMalloc).  The pages have no counterpart: this is a library convenience.
+ * Same arguments as moe_grouped_ffn, minus ws, and the same rows up to the FFN
+ * tolerance: this entry point always runs the split-K GEMV kernels
+ * (MOE_FFN_GEMV), so its rows are bit-identical to moe_grouped_ffn's where
+ * that call picks the GEMV kernels and within 1e-2 (max-relative) where it
+ * picks the tensor cores; prefill-sized batches run slower than there.
  * Scratch: a fixed 16 MiB device array inside the library, reserved on every
- * GPU that loads it until the process exits.  Calls needing more
- * (moe_grouped_ffn_workspace() > 16 MiB, i.e. T*k*I*2 bytes) are rejected with
- * MOE_ERR_INVALID_ARG before any launch.  The first call on a device looks up
- * the array's device address (once per device, that device current); make that
- * first call before any stream capture.  Every call shares the array and leaves
- * its contents behind; calls that overlap on the GPU race on it.  No
- * allocation is made by this call.
+ * GPU that loads it until the process exits.  The layer and sizes are checked
+ * first, as in moe_grouped_ffn; then calls with T*k*I*2 > 16 MiB (the bf16
+ * intermediate) are rejected with MOE_ERR_INVALID_ARG before any launch.  The
+ * first call on a device looks up the array's device address (once per
+ * device, that device current); make that first call before any stream
+ * capture, and do not call this entry point again after a cudaDeviceReset in
+ * the same process (the address it keeps would be stale).  Every call shares
+ * the array and leaves its contents behind; calls that overlap on the GPU race
+ * on it.  No allocation is made by this call.
  */
 MOE_API moe_status moe_grouped_ffn_noalloc(const moe_layer *layer, const uint16_t *x, int32_t T, int32_t k,
                                            const int32_t *counts, const int32_t *offsets,
@@ -323,7 +346,12 @@ MOE_API moe_status moe_refresh_target(const uint32_t *hits, int32_t E, int32_t b
                               int32_t *n_target);
 
 /*
- * Paired promote/demote (apply_target_placement) on a slot table.
+ * Paired promote/demote (apply_target_placement) on a slot table.  expert_pool.rs
+ * keeps a resident set and reports only counts; a slot table also needs to know
+ * which slot each promoted expert takes, so this call adds n_slots (the pool's
+ * extent) and returns the promoted and the demoted experts separately
+ * (n_promote, n_demote; the page's paired swap makes n_demote <= n_promote,
+ * with equality while the pool is full).
  * slot_of: HOST [E], slot id or -1, updated in place.  promote = target
  * experts not resident, in target order; demote = resident experts not in the
  * target, in ascending id, at most |promote| of them (the rest stay

@@ -52,7 +52,7 @@ class _CLayer(ctypes.Structure):
     _fields_ = [
         ("fmt", ctypes.c_int32), ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
         ("slot_table", ctypes.c_void_p), ("pool", ctypes.c_void_p), ("home", ctypes.c_void_p),
-        ("expert_bytes", ctypes.c_uint64),
+        ("expert_bytes", ctypes.c_uint64), ("pool_slots", ctypes.c_int32),
     ]
 
 
@@ -150,15 +150,20 @@ class MoeLayer:
     """One MoE layer's experts: format, sizes and the device memory they live in.
 
     ``home`` holds E expert blobs (uint8, stride ``expert_bytes``); ``pool`` and
-    ``slot_table`` (int32 [E], slot id or -1) are optional.  The tensors are kept
-    alive by this object.
+    ``slot_table`` (int32 [E], slot id or -1) are optional.  ``pool_slots`` is the
+    number of blobs in ``pool`` (default: as many whole blobs as it holds).  The
+    tensors are kept alive by this object.
     """
 
     def __init__(self, fmt: int, E: int, H: int, I: int, home: torch.Tensor, pool: torch.Tensor | None = None,
-                 slot_table: torch.Tensor | None = None, expert_bytes: int | None = None):
+                 slot_table: torch.Tensor | None = None, expert_bytes: int | None = None,
+                 pool_slots: int | None = None):
         self.fmt, self.E, self.H, self.I = int(fmt), int(E), int(H), int(I)
         self.expert_bytes = int(expert_bytes or moe_expert_bytes(fmt, H, I))
         self.home, self.pool, self.slot_table = home, pool, slot_table
+        if pool_slots is None:
+            pool_slots = 0 if pool is None else pool.numel() // self.expert_bytes
+        self.pool_slots = int(pool_slots)
         self._c = _CLayer()
         self.refresh()
 
@@ -169,6 +174,7 @@ class MoeLayer:
         self._c.pool = None if self.pool is None else _dev(self.pool, torch.uint8, "pool").value
         self._c.slot_table = None if self.slot_table is None else _dev(self.slot_table, torch.int32, "slot_table").value
         self._c.expert_bytes = self.expert_bytes
+        self._c.pool_slots = self.pool_slots
         return self
 
     def ref(self):

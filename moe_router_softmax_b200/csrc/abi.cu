@@ -31,6 +31,7 @@ bool ffn_tc_supports(int fmt, int H, int I, uint64_t stride);
 cudaError_t launch_ffn_tc(const LayerView &, const uint16_t *, int, int, const int32_t *, const int32_t *,
                           const int32_t *, float *, void *, cudaStream_t);
 cudaError_t tc_take_error(unsigned *code, unsigned *info);
+cudaError_t gemv_take_error(unsigned *code, unsigned *info);
 
 static thread_local char g_err[512];
 
@@ -81,6 +82,8 @@ static moe_status layer_view(const moe_layer *l, LayerView *v) {
               (unsigned long long)o.total);
     CHECK_ARG(aligned16(l->home) && aligned16(l->pool), "home/pool must be 16-byte aligned");
     CHECK_ARG(l->slot_table == nullptr || l->pool != nullptr, "a slot table needs a pool");
+    CHECK_ARG(l->slot_table == nullptr || l->pool_slots >= 1, "a slot table needs pool_slots >= 1 (got %d)",
+              l->pool_slots);
     v->fmt = l->fmt;
     v->E = l->E;
     v->H = l->H;
@@ -89,11 +92,21 @@ static moe_status layer_view(const moe_layer *l, LayerView *v) {
     v->pool = static_cast<const uint8_t *>(l->pool);
     v->home = static_cast<const uint8_t *>(l->home);
     v->stride = l->expert_bytes;
+    v->pool_slots = l->slot_table ? l->pool_slots : 0;
     v->off = o;
     return MOE_OK;
 }
 
 static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// The grouped FFN's layer and size checks, for the entry points that share them.
+moe_status check_ffn_args(const moe_layer *layer, int T, int k) {
+    LayerView v;
+    moe_status st = layer_view(layer, &v);
+    if (st != MOE_OK) return st;
+    if ((st = check_shape(v.E, k, v.H, v.I)) != MOE_OK) return st;
+    return check_tk(T, k);
+}
 
 }  // namespace moe
 
@@ -343,14 +356,22 @@ moe_status moe_take_device_errors(uint32_t *code, uint32_t *info) {
     CHECK_ARG(code && info, "moe_take_device_errors: NULL pointer");
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_status(e, "moe_take_device_errors: device synchronise");
-    unsigned c = 0, i = 0;
+    unsigned c = 0, i = 0, cg = 0, ig = 0;
     e = tc_take_error(&c, &i);
+    if (e == cudaSuccess) e = gemv_take_error(&cg, &ig);
     if (e != cudaSuccess) return cuda_status(e, "moe_take_device_errors: read");
+    if (c == 0) {  // the tensor-core word first, then the GEMV kernels' word
+        c = cg;
+        i = ig;
+    }
     *code = c;
     *info = i;
     if (c >= 0x1000u && c < 0x2000u)
         return set_error(MOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (warp %u)", c & 0xFFFu);
-    if (c) return set_error(MOE_ERR_CUDA, "a tensor-core kernel failed an index check (site %u, value %u)", c & 0xFFFu, i);
+    if (c == 0x2005u || c == 0x2006u)
+        return set_error(MOE_ERR_CUDA, "slot %u of the slot table is past the pool; that expert's routes were skipped",
+                         i);
+    if (c) return set_error(MOE_ERR_CUDA, "a kernel failed an index check (site %u, value %u)", c & 0xFFFu, i);
     return MOE_OK;
 }
 

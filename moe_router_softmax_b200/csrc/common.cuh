@@ -102,11 +102,25 @@ struct LayerView {
     const uint8_t *pool;
     const uint8_t *home;
     uint64_t stride;
+    int pool_slots;  // blobs in pool (meaningful with a slot table)
     BlobOffsets off;
 };
 
+// Slot of expert e: -1 for home, else a pool slot below pool_slots.  A table
+// entry at or past pool_slots is out of the pool: *bad is set (and -1 returned,
+// so that an address computed from it stays inside home).
+__device__ __forceinline__ int expert_slot(const LayerView &L, int e, bool *bad) {
+    const int s = L.slot_table ? __ldg(L.slot_table + e) : -1;
+    *bad = s >= L.pool_slots && L.slot_table != nullptr;
+    return (s >= 0 && !*bad) ? s : -1;
+}
+
+// Blob of expert e through the slot table, or nullptr when its slot is out of
+// the pool (the caller skips the expert and records the fault).
 __device__ __forceinline__ const uint8_t *expert_blob(const LayerView &L, int e) {
-    int s = L.slot_table ? __ldg(L.slot_table + e) : -1;
+    bool bad;
+    const int s = expert_slot(L, e, &bad);
+    if (bad) return nullptr;
     return s >= 0 ? L.pool + (uint64_t)s * L.stride : L.home + (uint64_t)e * L.stride;
 }
 

@@ -36,9 +36,19 @@ struct FfnParams {
     uint16_t *h;                  // [R][I] bf16 (phase 1 out / phase 2 in)
     float *rows;                  // [R][H] fp32
     int lg;                       // lanes per row group (power of two, <= 32)
+    int prefetch_w2;              // phase 1 requests the active experts' w2 into L2
 };
 
 namespace {
+
+// First slot fault a GEMV kernel recorded (0 = none): 0x2005 for an expert
+// whose slot is past the pool (info = the slot id); the expert's routes are
+// skipped.  Read and cleared by moe_take_device_errors().
+__device__ unsigned int g_gemv_error;
+__device__ unsigned int g_gemv_error_info;
+__device__ __forceinline__ void record_gemv_error(unsigned code, unsigned info) {
+    if (atomicCAS(&g_gemv_error, 0u, code) == 0u) g_gemv_error_info = info;
+}
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -318,6 +328,28 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
     __syncthreads();
     const int n_act = s_nact;
     const int total = s_base[n_act];
+    if (PHASE == 1 && p.prefetch_w2 && warp == kWarps - 1) {
+        // a batch whose routed experts fit in L2 many times over (one token):
+        // phase 2 cannot start streaming w2 before phase 1's CTAs retire, so
+        // phase 1 asks for it now -- each CTA a 1/grid share of the active
+        // experts' w2 pieces (codes and scales), in 16-byte multiples -- and
+        // phase 2 then finds its weights in L2
+        const uint64_t piece = p.L.off.total - p.L.off.q2;
+        const uint64_t all = (uint64_t)n_act * piece;
+        const uint64_t share = ((all + gridDim.x - 1) / gridDim.x + 15) & ~(uint64_t)15;
+        const uint64_t beg = (uint64_t)blockIdx.x * share, end = min(all, beg + share);
+        constexpr uint64_t kChunk = 8192;
+        for (uint64_t off = beg + (uint64_t)lane * kChunk; off < end; off += 32 * kChunk) {
+            const int a = (int)(off / piece);
+            const uint64_t in = off - (uint64_t)a * piece;
+            const uint64_t n = min(min(end - off, piece - in), kChunk);
+            const uint8_t *blob = expert_blob(p.L, s_act[a]);
+            if (blob != nullptr && n >= 16)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(blob + p.L.off.q2 + in),
+                             "r"((uint32_t)(n & ~(uint64_t)15))
+                             : "memory");
+        }
+    }
     const int it_begin = (int)(((long long)total * blockIdx.x) / gridDim.x);
     const int it_end = (int)(((long long)total * (blockIdx.x + 1)) / gridDim.x);
     if (it_begin >= it_end) return;
@@ -340,7 +372,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
             while (s_base[pa + 1] <= it) ++pa;
             const int tile = (it - s_base[pa]) % tiles;
             const int r0 = tile * upi, r1 = min(n_units, r0 + upi);
-            const uint8_t *w = expert_blob(p.L, s_act[pa]) + p.L.off.q2 + (uint64_t)r0 * row_bytes;
+            const uint8_t *blob = expert_blob(p.L, s_act[pa]);
+            if (blob == nullptr) continue;  // slot out of the pool: the item is skipped below
+            const uint8_t *w = blob + p.L.off.q2 + (uint64_t)r0 * row_bytes;
             for (uint64_t off = 0, n = (uint64_t)(r1 - r0) * row_bytes; off < n; off += 32768) {
                 const uint32_t bytes = (uint32_t)(n - off < 32768 ? n - off : 32768);
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(w + off), "r"(bytes) : "memory");
@@ -359,6 +393,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
         const int n_e = __ldg(p.counts + e);
         const int row0 = __ldg(p.offsets + e) + chunk * kNTM;
         const int nt = min(kNTM, n_e - chunk * kNTM);
+        const uint8_t *blob = expert_blob(p.L, e);
+        if (blob == nullptr) {
+            // the expert's slot is past the pool: nothing of this item is read or
+            // written (the same for every thread of the CTA, so no barrier is split)
+            if (threadIdx.x == 0) record_gemv_error(0x2005u, (unsigned)__ldg(p.L.slot_table + e));
+            continue;
+        }
         const int key = a * 65536 + chunk;
         if (key != cur_key) {
             __syncthreads();
@@ -366,7 +407,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
             __syncthreads();
             cur_key = key;
         }
-        const uint8_t *blob = expert_blob(p.L, e);
         const int u0 = tile * upi + gi * UPG;
         if (NTMAX == 1) {
             // route t0's activations are sub-planes t0*SP .. of xs
@@ -441,6 +481,14 @@ cudaError_t launch_fmt(const FfnParams &p, int n_sm, cudaStream_t s) {
 
 size_t ffn_gemv_workspace(int T, int k, int I) { return (size_t)T * k * I * sizeof(uint16_t); }
 
+cudaError_t gemv_take_error(unsigned *code, unsigned *info) {
+    unsigned zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_gemv_error, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(info, g_gemv_error_info, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv_error, &zero, sizeof(unsigned));
+    return e;
+}
+
 cudaError_t launch_ffn_gemv(const LayerView &L, const uint16_t *x, int T, int k, const int32_t *counts,
                             const int32_t *offsets, const int32_t *sorted_route, float *rows, void *ws,
                             cudaStream_t s) {
@@ -457,6 +505,9 @@ cudaError_t launch_ffn_gemv(const LayerView &L, const uint16_t *x, int T, int k,
     p.sorted_route = sorted_route;
     p.h = static_cast<uint16_t *>(ws);
     p.rows = rows;
+    // w2 into L2 during phase 1 when every routed expert together is far below
+    // the L2 size (at most T*k distinct experts)
+    p.prefetch_w2 = (uint64_t)T * k * L.stride <= (uint64_t)100 << 20;
     if (L.fmt == MOE_W_BF16) return launch_fmt<MOE_W_BF16>(p, n_sm, s);
     if (L.fmt == MOE_W_INT8) return launch_fmt<MOE_W_INT8>(p, n_sm, s);
     return launch_fmt<MOE_W_INT4>(p, n_sm, s);

@@ -9,6 +9,12 @@
 // the device and can fail under fragmentation).  For them this entry point
 // keeps its scratch in a fixed, file-scope device array instead.
 //
+// It always runs the split-K GEMV kernels (their only scratch is h, T*k*I*2
+// bytes); the tensor-core kernels would also need a sorted copy of the
+// activations.  Its rows therefore equal moe_grouped_ffn's where that call picks
+// the GEMV kernels, and agree within the FFN tolerance where it picks the tensor
+// cores; prefill-sized batches run slower than through moe_grouped_ffn.
+//
 // The array is a module global: every GPU that loads the library reserves it
 // (kNoAllocScratchBytes) until the process exits, and every call shares it.
 // Nothing in it has to start at zero -- each call writes every h row it later
@@ -21,6 +27,7 @@
 
 namespace moe {
 size_t ffn_gemv_workspace(int T, int k, int I);
+moe_status check_ffn_args(const moe_layer *layer, int T, int k);
 }
 
 namespace {
@@ -33,7 +40,9 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch per device, looked up once with that
 // device current (on the host the symbol name is only a stand-in, never a
-// device pointer).
+// device pointer).  The cached address belongs to the device's primary
+// context: after a cudaDeviceReset it is stale, so the entry point must not be
+// called again in that process.
 void *g_scratch_addr[moe::kMaxDevices];
 std::mutex g_scratch_mutex;
 
@@ -65,8 +74,10 @@ extern "C" {
 moe_status moe_grouped_ffn_noalloc(const moe_layer *layer, const uint16_t *x, int32_t T, int32_t k,
                                    const int32_t *counts, const int32_t *offsets, const int32_t *sorted_route,
                                    float *rows, moe_stream_t stream) {
-    if (layer == nullptr) return moe::set_error(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_noalloc: layer is NULL");
-    if (T < 0 || k < 1) return moe::set_error(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_noalloc: T=%d k=%d", T, k);
+    // the layer and the sizes first, so that a bad argument is reported as what
+    // it is rather than as a scratch overflow
+    moe_status st = moe::check_ffn_args(layer, T, k);
+    if (st != MOE_OK) return st;
     // the GEMV kernels' scratch: the bf16 intermediate, T*k*I*2 bytes
     const size_t need = moe::ffn_gemv_workspace(T, k, layer->I);
     if (need > kNoAllocScratchBytes)
@@ -75,7 +86,7 @@ moe_status moe_grouped_ffn_noalloc(const moe_layer *layer, const uint16_t *x, in
                               "scratch holds %zu bytes (use moe_grouped_ffn with a workspace instead)",
                               (long long)T * k, layer->I, need, kNoAllocScratchBytes);
     void *scratch = nullptr;
-    moe_status st = scratch_for_current_device(&scratch);
+    st = scratch_for_current_device(&scratch);
     if (st != MOE_OK) return st;
     return moe_grouped_ffn_path(layer, x, T, k, counts, offsets, sorted_route, rows, scratch, kNoAllocScratchBytes,
                                 MOE_FFN_GEMV, stream);

@@ -125,8 +125,6 @@ struct TcParams {
     int n_block;           // cap on the route block (multiple of 16, <= kNMax)
     int K;                 // reduction length: H (phase 1) or I (phase 2)
     int n_units;           // output rows of the weight: 2I (phase 1) or H (phase 2)
-    int64_t rows_per_blob; // expert_bytes / row_bytes
-    int64_t q_row_off;     // offset of the code matrix in the blob / row_bytes
     uint16_t *h;           // [R][I] bf16: phase-1 output
     float *rows;           // [R][H] fp32: phase-2 output
 };
@@ -181,6 +179,15 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
         ::"r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+// 3-D box {x, y, z} of a weight map: x along the row, y the row of the matrix,
+// z the blob (expert or pool slot).  Coordinates past an extent read zeros.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
+                                            int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -320,22 +327,33 @@ __device__ __forceinline__ ItemInfo decode_item(const TcParams &p, const int *s_
     r.row0 = __ldg(p.offsets + r.e) + nb * n_block;
     r.n = min(n_block, n_e - nb * n_block);
     r.n_mma = (r.n + 15) & ~15;
-    if (r.n <= 0 || r.n_mma > n_block || r.row0 < 0 || r.row0 + r.n > p.R) {
-        record_error(0x2003u, (unsigned)item);
-        r.n = 0;       // nothing is written for an item that fails the check,
-        r.n_mma = 16;  // and its tiles stay inside their slots
-        r.row0 = 0;
+    bool bad_slot;
+    expert_slot(p.L, r.e, &bad_slot);
+    if (bad_slot) record_error(0x2006u, (unsigned)__ldg(p.L.slot_table + r.e));
+    if (r.n <= 0 || r.n_mma > n_block || r.row0 < 0 || r.row0 + r.n > p.R || bad_slot) {
+        if (!bad_slot) record_error(0x2003u, (unsigned)item);
+        r.n = 0;       // nothing is written for an item that fails the check (its
+        r.n_mma = 16;  // weights are read from home), and its tiles stay inside
+        r.row0 = 0;    // their slots
     }
     r.m0 = mt;  // tile index; callers scale it
     return r;
 }
 
-// Row coordinate of weight row `row` of expert e in the home / pool tensor maps.
-__device__ __forceinline__ int a_row_coord(const TcParams &p, int e, int row, bool *in_pool) {
-    const int s = p.L.slot_table ? __ldg(p.L.slot_table + e) : -1;
+// Blob coordinate (z) of expert e in the home or pool weight map.  An expert
+// whose slot is past the pool is read from home (its item writes nothing).
+__device__ __forceinline__ int a_blob_coord(const TcParams &p, int e, bool *in_pool) {
+    bool bad;
+    const int s = expert_slot(p.L, e, &bad);
     *in_pool = s >= 0;
-    const int64_t blob = s >= 0 ? s : e;
-    return (int)(blob * p.rows_per_blob + p.q_row_off + row);
+    return s >= 0 ? s : e;
+}
+
+// Blob of expert e for the scale reads; home for an expert whose slot is past
+// the pool (its item writes nothing).
+__device__ __forceinline__ const uint8_t *scale_blob(const TcParams &p, int e) {
+    const uint8_t *b = expert_blob(p.L, e);
+    return b ? b : p.L.home + (uint64_t)e * p.L.stride;
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -451,12 +469,13 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
                 const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 bool pool;
-                int ya0, ya1;  // row coordinates of the two 64-row halves of the tile
+                const int za = a_blob_coord(p, it.e, &pool);
+                int ya0, ya1;  // rows of the matrix of the two 64-row halves of the tile
                 if (PHASE == 1) {
-                    ya0 = a_row_coord(p, it.e, it.m0 * 64, &pool);
-                    ya1 = a_row_coord(p, it.e, p.L.I + it.m0 * 64, &pool);
+                    ya0 = it.m0 * 64;
+                    ya1 = p.L.I + it.m0 * 64;
                 } else {
-                    ya0 = a_row_coord(p, it.e, it.m0 * kBlockM, &pool);
+                    ya0 = it.m0 * kBlockM;
                     ya1 = ya0 + 64;
                 }
                 const CUtensorMap *ma = pool ? &map_pool : &map_home;
@@ -466,8 +485,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                         if (!mbar_wait(&r_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
                         mbar_arrive_expect_tx(&r_full[stage], (uint32_t)RAW);
                         uint8_t *dst = sRaw + stage * RAW;
-                        tma_load_2d(dst, ma, &r_full[stage], rs * kRawRowBytes, ya0);
-                        tma_load_2d(dst + 64 * kRawRowBytes, ma, &r_full[stage], rs * kRawRowBytes, ya1);
+                        tma_load_3d(dst, ma, &r_full[stage], rs * kRawRowBytes, ya0, za);
+                        tma_load_3d(dst + 64 * kRawRowBytes, ma, &r_full[stage], rs * kRawRowBytes, ya1, za);
                         if (++stage == SR) { stage = 0; phase ^= 1; }
                     }
                 } else {
@@ -477,8 +496,9 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                         mbar_arrive_expect_tx(&a_full[stage], (uint32_t)na * kATileBytes);
                         for (int a = 0; a < na; ++a) {
                             uint8_t *dst = sA + (stage * ATOMS + a) * kATileBytes;
-                            tma_load_2d(dst, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya0);
-                            tma_load_2d(dst + kATileBytes / 2, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya1);
+                            tma_load_3d(dst, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya0, za);
+                            tma_load_3d(dst + kATileBytes / 2, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya1,
+                                        za);
                         }
                         if (++stage == SA) { stage = 0; phase ^= 1; }
                     }
@@ -586,7 +606,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             if (!mbar_wait(&tfull[acc], acc_phase, &s_abort)) break;
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kNMax);
-            const uint8_t *blob = expert_blob(p.L, it.e);
+            const uint8_t *blob = scale_blob(p, it.e);
             float scale = 1.0f;
             if (FMT == MOE_W_INT8) {
                 const int wrow = PHASE == 1 ? (lrow < 64 ? it.m0 * 64 + lrow : p.L.I + it.m0 * 64 + lrow - 64)
@@ -675,7 +695,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         uint32_t step = 0;                              // stages seen, across items
         for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
             const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
-            const uint8_t *blob = expert_blob(p.L, it.e);
+            const uint8_t *blob = scale_blob(p, it.e);
             const int wrow = PHASE == 1 ? (r < 64 ? it.m0 * 64 + r : p.L.I + it.m0 * 64 + r - 64)
                                         : min(it.m0 * kBlockM + r, p.n_units - 1);
             const uint16_t *srow = reinterpret_cast<const uint16_t *>(blob + (PHASE == 1 ? p.L.off.s13 : p.L.off.s2)) +
@@ -823,6 +843,20 @@ cudaError_t get_encoder() {
     return g_encode ? cudaSuccess : cudaErrorNotSupported;
 }
 
+// 3-D map over `blobs` matrices of `rows` rows of `row_elems` elements, one
+// matrix per blob (`blob_stride` bytes apart, starting at `base`); box =
+// box_inner elements x box_rows rows of one matrix.
+bool encode_3d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t row_elems,
+               uint64_t rows, uint64_t blobs, uint64_t blob_stride, uint32_t box_inner, uint32_t box_rows,
+               CUtensorMapSwizzle sw) {
+    cuuint64_t dims[3] = {row_elems, rows, blobs};
+    cuuint64_t strides[2] = {row_elems * (uint64_t)elem_bytes, blob_stride};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return g_encode(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D map over `rows` rows of `row_bytes` bytes; box = box_inner elements x box_rows.
 bool encode_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t row_elems,
                uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
@@ -883,13 +917,11 @@ size_t ffn_tc_workspace(int T, int k, int E, int H, int I) {
 }
 
 bool ffn_tc_supports(int fmt, int H, int I, uint64_t stride) {
-    if (H % 64 || I % 64) return false;
-    // every weight row of every expert must start on a whole row of the tensor
-    // map that spans the blob buffer
-    const BlobOffsets o = blob_offsets(fmt, H, I);
-    const uint64_t rb1 = fmt == MOE_W_BF16 ? (uint64_t)H * 2 : (fmt == MOE_W_INT8 ? (uint64_t)H : (uint64_t)H / 2);
-    const uint64_t rb2 = fmt == MOE_W_BF16 ? (uint64_t)I * 2 : (fmt == MOE_W_INT8 ? (uint64_t)I : (uint64_t)I / 2);
-    return stride % rb1 == 0 && stride % rb2 == 0 && o.q2 % rb2 == 0 && get_encoder() == cudaSuccess;
+    (void)fmt;
+    // the weight maps are 3-D (row, matrix row, blob), so any blob stride that is a
+    // multiple of 16 bytes works; every row length (H or I times 2, 1 or 1/2
+    // bytes) is a multiple of 32 bytes and every matrix piece starts 16-byte aligned
+    return H % 64 == 0 && I % 64 == 0 && stride % 16 == 0 && get_encoder() == cudaSuccess;
 }
 
 cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, const int32_t *counts,
@@ -923,14 +955,17 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     for (int ph = 1; ph <= 2; ++ph) {
         const int K = ph == 1 ? H : I;
         const uint64_t row_elems = bf ? (uint64_t)K : (fmt == MOE_W_INT8 ? (uint64_t)K : (uint64_t)K / 2);
-        const uint64_t row_bytes = row_elems * eb;
         const uint32_t box_inner = bf ? kBlockK : raw_inner;
         CUtensorMap *mh = ph == 1 ? &mh1 : &mh2, *mp = ph == 1 ? &mp1 : &mp2;
-        const uint64_t home_rows = (uint64_t)L.E * L.stride / row_bytes;
-        if (!encode_2d(mh, L.home, dt, eb, row_elems, home_rows, box_inner, 64, swa)) return cudaErrorInvalidValue;
-        // the pool's extent is unknown here: map it with the home's row count
-        // (only rows of slots in use are ever addressed)
-        if (!encode_2d(mp, L.pool ? L.pool : L.home, dt, eb, row_elems, home_rows, box_inner, 64, swa))
+        // one matrix (w13 codes, or w2 codes) per blob: E blobs of home, pool_slots
+        // of the pool (home again when the layer has no slot table)
+        const uint64_t piece = ph == 1 ? L.off.q13 : L.off.q2;
+        const uint64_t mrows = ph == 1 ? 2 * (uint64_t)I : (uint64_t)H;
+        if (!encode_3d(mh, L.home + piece, dt, eb, row_elems, mrows, (uint64_t)L.E, L.stride, box_inner, 64, swa))
+            return cudaErrorInvalidValue;
+        const bool slotted = L.slot_table != nullptr && L.pool != nullptr && L.pool_slots > 0;
+        if (!encode_3d(mp, (slotted ? L.pool : L.home) + piece, dt, eb, row_elems, mrows,
+                       slotted ? (uint64_t)L.pool_slots : (uint64_t)L.E, L.stride, box_inner, 64, swa))
             return cudaErrorInvalidValue;
         CUtensorMap *mb = ph == 1 ? &mb1 : &mb2, *mbb = ph == 1 ? &mbb1 : &mbb2;
         if (!encode_2d(mb, ph == 1 ? (const void *)xs : (const void *)h, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
@@ -961,11 +996,8 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
         return cudaErrorInvalidValue;
     // phase 1
     {
-        const uint64_t rb = bf ? (uint64_t)H * 2 : (fmt == MOE_W_INT8 ? (uint64_t)H : (uint64_t)H / 2);
         p.K = H;
         p.n_units = 2 * I;
-        p.rows_per_blob = (int64_t)(L.stride / rb);
-        p.q_row_off = (int64_t)(L.off.q13 / rb);
         if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 1, 0>(mh1, mp1, mb1, mbb1, p, n_sm, s);
         else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 1, 1>(mh1, mp1, mb1, mbb1, p, n_sm, s)
                                               : launch_one<MOE_W_INT8, 1, 0>(mh1, mp1, mb1, mbb1, p, n_sm, s);
@@ -975,11 +1007,8 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     }
     // phase 2
     {
-        const uint64_t rb = bf ? (uint64_t)I * 2 : (fmt == MOE_W_INT8 ? (uint64_t)I : (uint64_t)I / 2);
         p.K = I;
         p.n_units = H;
-        p.rows_per_blob = (int64_t)(L.stride / rb);
-        p.q_row_off = (int64_t)(L.off.q2 / rb);
         if (fmt == MOE_W_BF16) err = launch_one<MOE_W_BF16, 2, 0>(mh2, mp2, mb2, mbb2, p, n_sm, s);
         else if (fmt == MOE_W_INT8) err = two ? launch_one<MOE_W_INT8, 2, 1>(mh2, mp2, mb2, mbb2, p, n_sm, s)
                                               : launch_one<MOE_W_INT8, 2, 0>(mh2, mp2, mb2, mbb2, p, n_sm, s);

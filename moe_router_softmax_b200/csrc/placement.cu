@@ -1,4 +1,4 @@
-// placement.cpp -- the expert residency pool's host logic (rlx_runtime
+// placement.cu -- the expert residency pool's host logic (rlx_runtime
 // expert_pool.rs): hit-ranked target selection, paired promote/demote on a
 // cache-slot table, the refresh schedule and the VRAM budget formula.
 // Pure host code; no CUDA.

@@ -44,13 +44,15 @@ def _null_layer(**kw):
     c.pool = kw.get("pool", None)
     c.slot_table = kw.get("slot_table", None)
     c.expert_bytes = kw.get("expert_bytes", moe.moe_expert_bytes(c.fmt, c.H, c.I))
+    c.pool_slots = kw.get("pool_slots", 0)
     return ctypes.byref(c)
 
 
 @pytest.mark.parametrize("args,frag", [
     (dict(E=0), "E=0"), (dict(E=2000), "E=2000"), (dict(H=100), "H=100"), (dict(I=96), "I=96"),
     (dict(fmt=7), "format"), (dict(expert_bytes=1000), "expert_bytes"), (dict(home=8), "aligned"),
-    (dict(slot_table=256), "pool"),
+    (dict(slot_table=256), "pool"), (dict(slot_table=256, pool=512), "pool_slots"),
+    (dict(slot_table=256, pool=512, pool_slots=-3), "pool_slots"),
 ])
 def test_ffn_rejects_bad_layers_before_launch(args, frag):
     st = moe._lib.moe_grouped_ffn(_null_layer(**args), 256, 4, 2, 256, 256, 256, 256, 256, 1 << 20, None)

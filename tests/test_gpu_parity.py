@@ -337,12 +337,10 @@ def test_gemma_layer_prefill_sampled():
 
 # ------------------------------------------------------ tensor-core FFN path
 
-def _tc_or_skip(L, lg, x, k):
-    try:
-        return _run_layer(L, lg, x, k, path=moe.MOE_FFN_TC)
-    except moe.MoeError as e:
-        assert e.status == moe.MOE_ERR_UNSUPPORTED, str(e)
-        pytest.skip(f"tensor-core path unsupported here: {e}")
+def _tc(L, lg, x, k):
+    """The layer with the tcgen05 kernels forced (they take every format at every
+    H, I that are multiples of 64: the weight maps are 3-D, blob by blob)."""
+    return _run_layer(L, lg, x, k, path=moe.MOE_FFN_TC)
 
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
@@ -357,7 +355,7 @@ def test_tc_layer_small_every_element(fmt, E, H, I, k, T):
     lg = syn.router_logits(T, E, "normal", seed=12)
     L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
     xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
-    ids, w, counts, offsets, sr, rp, rows, y = _tc_or_skip(L, torch.from_numpy(lg).to(DEV), xd, k)
+    ids, w, counts, offsets, sr, rp, rows, y = _tc(L, torch.from_numpy(lg).to(DEV), xd, k)
     oi, ow, orows, oy = oracle.moe_layer(oracle_layer_for(fmt, w13, w2), lg, x, k)
     assert np.array_equal(ids.cpu().numpy(), oi)
     g_rows = rows.cpu().numpy()[rp.cpu().numpy()]
@@ -372,7 +370,7 @@ def test_tc_gemma_layer_decode_sampled(fmt, kind, T):
     w13, w2, L = _full_layer(fmt)
     x = syn.activations(T, H, seed=300 + T)
     lg = syn.router_logits(T, E, kind, seed=400 + T)
-    ids, w, counts, offsets, sr, rp, rows, y = _tc_or_skip(
+    ids, w, counts, offsets, sr, rp, rows, y = _tc(
         L, torch.from_numpy(lg).to(DEV), torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16), k)
     oi, ow = oracle.route_topk(lg, k)
     toks = np.unique(np.r_[0, T - 1, np.random.default_rng(T).integers(0, T, size=2)])
@@ -405,9 +403,91 @@ def test_tc_and_gemv_agree_on_the_slot_table():
     x = torch.from_numpy(syn.activations(T, H, seed=2).view(np.int16)).to(DEV).view(torch.bfloat16)
     lg = torch.from_numpy(syn.router_logits(T, E, "zipf", seed=2)).to(DEV)
     a = _run_layer(L, lg, x, k, path=moe.MOE_FFN_GEMV)[-2]
-    b = _tc_or_skip(L2, lg, x, k)[-2]
+    b = _tc(L2, lg, x, k)[-2]
     n = a.shape[0]
     assert rel_err(b.cpu().numpy()[:n], a.cpu().numpy()) <= FFN_TOL
+
+
+def _pool_layers(fmt, E, H, I, w13, w2, slot_of, n_slots):
+    """The same slotted layer on both sides: device pool of n_slots blobs filled
+    from the device home, oracle pool built by the oracle's own quantiser and
+    packer, the same slot table; home of every slotted expert wiped on the device
+    so that only the pool can serve it."""
+    L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
+    eb = L.expert_bytes
+    pool = torch.zeros(n_slots * eb, dtype=torch.uint8, device=DEV)
+    held = np.nonzero(slot_of >= 0)[0]
+    moe.moe_copy_to_slots(L.home, pool, eb, held, slot_of[held])
+    home2 = L.home.clone()
+    for e in held:
+        home2[e * eb:(e + 1) * eb] = 0
+    table = torch.from_numpy(slot_of.astype(np.int32)).to(DEV)
+    Ld = moe.MoeLayer(fmt, E, H, I, home2, pool=pool, slot_table=table, pool_slots=n_slots)
+    oeb = oracle.expert_bytes(fmt, H, I)
+    ohome = np.concatenate([oracle_blob(fmt, w13[e], w2[e], H, I) for e in range(E)])
+    opool = np.zeros(n_slots * oeb, np.uint8)
+    for e in held:
+        opool[slot_of[e] * oeb:(slot_of[e] + 1) * oeb] = oracle_blob(fmt, w13[e], w2[e], H, I)
+    OL = oracle.Layer(fmt, E, H, I, ohome, pool=opool, slot_table=slot_of.astype(np.int32))
+    return Ld, OL
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("path", [moe.MOE_FFN_GEMV, moe.MOE_FFN_TC])
+def test_pool_with_more_slots_than_experts_matches_the_oracle(fmt, path):
+    """A pool holds more slots than the layer has experts (prain's 540 cache
+    slots are shared by the layers; remote_experts.cpp reads a cached expert from
+    its device slot): 8 experts, 24 slots, slot ids up to 23.  Both kernel paths
+    against the oracle on the same slot table, every row and output element."""
+    E, H, I, k, T = 8, 512, 192, 3, 45
+    w13, w2 = syn.expert_weights(E, H, I, seed=77)
+    slot_of = np.array([23, -1, 17, 5, -1, 20, 0, 11], np.int32)
+    Ld, OL = _pool_layers(fmt, E, H, I, w13, w2, slot_of, 24)
+    x = syn.activations(T, H, seed=78)
+    lg = syn.router_logits(T, E, "normal", seed=79)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    ids, w, counts, offsets, sr, rp, rows, y = _run_layer(Ld, torch.from_numpy(lg).to(DEV), xd, k, path=path)
+    assert moe.moe_take_device_errors() == (0, 0)
+    oi, ow, orows, oy = oracle.moe_layer(OL, lg, x, k)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    assert rel_err(rows.cpu().numpy()[rp.cpu().numpy()], orows) <= FFN_TOL
+    assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
+
+
+@pytest.mark.parametrize("path", [moe.MOE_FFN_GEMV, moe.MOE_FFN_TC])
+def test_slot_past_the_pool_is_refused_and_reported(path):
+    """A slot table entry at or past pool_slots is refused on the device: that
+    expert's routes are skipped (their rows keep what the caller put there), the
+    kernels record the bad slot for moe_take_device_errors, and every other
+    expert's rows still match the oracle.  The kernels resolve such an expert to
+    its home blob for any address they form, so nothing outside the buffers is
+    read."""
+    E, H, I, k, T = 8, 256, 128, 2, 40
+    w13, w2 = syn.expert_weights(E, H, I, seed=81)
+    slot_of = np.array([2, -1, 0, -1, 1, -1, -1, -1], np.int32)
+    Ld, OL = _pool_layers(2, E, H, I, w13, w2, slot_of, 3)
+    bad = slot_of.copy()
+    bad[4] = 3                               # == pool_slots: one past the end
+    Ld.slot_table.copy_(torch.from_numpy(bad))
+    x = syn.activations(T, H, seed=82)
+    lg = syn.router_logits(T, E, "normal", seed=83)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    moe.moe_take_device_errors()             # start from a clear word
+    ids, w = moe.moe_route_topk(torch.from_numpy(lg).to(DEV), k)
+    counts, offsets, sr, rp = moe.moe_permute(ids, E)
+    rows = torch.full((T * k, H), 7.0, dtype=torch.float32, device=DEV)
+    moe.moe_grouped_ffn(Ld, xd, k, counts, offsets, sr, rows=rows, path=path)
+    code, info = moe.moe_take_device_errors()
+    assert code in (0x2005, 0x2006) and info == 3
+    oi, _ = oracle.route_topk(lg, k)
+    assert int((oi == 4).sum()) > 0
+    rp_h = rp.cpu().numpy()
+    g = rows.cpu().numpy()[rp_h]
+    mine = (oi.ravel() == 4)
+    assert np.all(g[mine] == 7.0)            # skipped: untouched
+    orows = oracle.ffn_routes(OL, x, oi)
+    assert rel_err(g[~mine], orows[~mine]) <= FFN_TOL
+    assert moe.moe_take_device_errors() == (0, 0)
 
 
 # ------------------------------------------------------- [miss] min_weight

@@ -1,12 +1,17 @@
 """moe_grouped_ffn_noalloc: the grouped FFN for callers that cannot allocate
 device memory (a runtime that hands the library only input and output buffers,
 or a loop that must not call cudaMalloc).  Its scratch is a fixed device array
-inside the library instead of a caller workspace.
+inside the library instead of a caller workspace, and it always runs the split-K
+GEMV kernels.
 
-Checked through the C ABI against moe_grouped_ffn (the workspace entry point) on
-the same inputs, on two calls in a row with different batches, so the second call
-runs over the scratch contents the first one left behind.  This file is named to
-be collected last; it also passes on its own in a fresh process.
+Checked through the C ABI, on consecutive calls with different batches (so each
+later call runs over the scratch contents the earlier one left behind), against
+  - the CPU oracle, every row, at the FFN tolerance;
+  - moe_grouped_ffn_path(..., MOE_FFN_GEMV) on the same inputs: bit-identical;
+  - moe_grouped_ffn (the workspace entry point, AUTO path): within the tolerance.
+The sequence includes a one-token call, which takes the GEMV kernels' one-token
+instantiation.  This file is named to be collected last; it also passes on its
+own in a fresh process.
 """
 import ctypes
 
@@ -14,9 +19,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synthetic as syn
 import moe_router_softmax_b200 as moe
-from gpu_support import FFN_TOL, device_weights_from_host, rel_err
+from gpu_support import FFN_TOL, device_weights_from_host, oracle_layer_for, rel_err
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -32,22 +38,30 @@ def _noalloc(L, x, k, counts, offsets, sr, rows):
     assert st == moe.MOE_OK, moe.moe_last_error()
 
 
-@pytest.mark.parametrize("fmt", [moe.MOE_W_BF16, moe.MOE_W_INT4])
-def test_noalloc_matches_workspace_entry_point_twice(fmt):
+@pytest.mark.parametrize("fmt", [moe.MOE_W_BF16, moe.MOE_W_INT8, moe.MOE_W_INT4])
+def test_noalloc_matches_the_oracle_and_the_workspace_entry_point(fmt):
     E, H, I, k = 16, 1024, 320, 4
     w13, w2 = syn.expert_weights(E, H, I, seed=31)
     L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
-    for call, T in enumerate((40, 23)):
-        x = torch.from_numpy(syn.activations(T, H, seed=40 + call).view(np.int16)).to(DEV).view(torch.bfloat16)
-        lg = torch.from_numpy(syn.router_logits(T, E, "normal", seed=50 + call)).to(DEV)
-        ids, w = moe.moe_route_topk(lg, k)
+    OL = oracle_layer_for(fmt, w13, w2)
+    for call, T in enumerate((40, 1, 23)):
+        xh = syn.activations(T, H, seed=40 + call)
+        lgh = syn.router_logits(T, E, "normal", seed=50 + call)
+        x = torch.from_numpy(xh.view(np.int16)).to(DEV).view(torch.bfloat16)
+        ids, w = moe.moe_route_topk(torch.from_numpy(lgh).to(DEV), k)
         counts, offsets, sr, rp = moe.moe_permute(ids, E)
-        ref = moe.moe_grouped_ffn(L, x, k, counts, offsets, sr)
+        gemv = moe.moe_grouped_ffn(L, x, k, counts, offsets, sr, path=moe.MOE_FFN_GEMV)
+        auto = moe.moe_grouped_ffn(L, x, k, counts, offsets, sr)
         rows = torch.full((T * k, H), float("nan"), dtype=torch.float32, device=DEV)
         _noalloc(L, x, k, counts, offsets, sr, rows)
         torch.cuda.synchronize()
         n = int(offsets[-1])
-        assert rel_err(rows[:n].cpu().numpy(), ref[:n].cpu().numpy()) <= FFN_TOL
+        assert n == T * k
+        got = rows[:n].cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), gemv[:n].cpu().numpy().view(np.uint32))
+        assert rel_err(got, auto[:n].cpu().numpy()) <= FFN_TOL
+        orows = oracle.ffn_routes(OL, xh, oracle.route_topk(lgh, k)[0])
+        assert rel_err(got[rp.cpu().numpy()], orows) <= FFN_TOL
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch():
@@ -61,3 +75,8 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     st = moe._lib.moe_grouped_ffn_noalloc(L.ref(), _ptr(x), T, k, _ptr(z), _ptr(z), _ptr(z), _ptr(rows), None)
     assert st == moe.MOE_ERR_INVALID_ARG
     assert "scratch" in moe.moe_last_error()
+    # a bad layer is reported as what it is, not as a scratch overflow
+    bad = moe.MoeLayer(moe.MOE_W_BF16, E, H, 4100, home, expert_bytes=moe.moe_expert_bytes(0, H, I))
+    st = moe._lib.moe_grouped_ffn_noalloc(bad.ref(), _ptr(x), T, k, _ptr(z), _ptr(z), _ptr(z), _ptr(rows), None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    assert "I=4100" in moe.moe_last_error()

@@ -36,7 +36,6 @@ struct FfnParams {
     uint16_t *h;                  // [R][I] bf16 (phase 1 out / phase 2 in)
     float *rows;                  // [R][H] fp32
     int lg;                       // lanes per row group (power of two, <= 32)
-    int prefetch_w2;              // phase 1 requests the active experts' w2 into L2
 };
 
 namespace {
@@ -328,28 +327,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
     __syncthreads();
     const int n_act = s_nact;
     const int total = s_base[n_act];
-    if (PHASE == 1 && p.prefetch_w2 && warp == kWarps - 1) {
-        // a batch whose routed experts fit in L2 many times over (one token):
-        // phase 2 cannot start streaming w2 before phase 1's CTAs retire, so
-        // phase 1 asks for it now -- each CTA a 1/grid share of the active
-        // experts' w2 pieces (codes and scales), in 16-byte multiples -- and
-        // phase 2 then finds its weights in L2
-        const uint64_t piece = p.L.off.total - p.L.off.q2;
-        const uint64_t all = (uint64_t)n_act * piece;
-        const uint64_t share = ((all + gridDim.x - 1) / gridDim.x + 15) & ~(uint64_t)15;
-        const uint64_t beg = (uint64_t)blockIdx.x * share, end = min(all, beg + share);
-        constexpr uint64_t kChunk = 8192;
-        for (uint64_t off = beg + (uint64_t)lane * kChunk; off < end; off += 32 * kChunk) {
-            const int a = (int)(off / piece);
-            const uint64_t in = off - (uint64_t)a * piece;
-            const uint64_t n = min(min(end - off, piece - in), kChunk);
-            const uint8_t *blob = expert_blob(p.L, s_act[a]);
-            if (blob != nullptr && n >= 16)
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(blob + p.L.off.q2 + in),
-                             "r"((uint32_t)(n & ~(uint64_t)15))
-                             : "memory");
-        }
-    }
     const int it_begin = (int)(((long long)total * blockIdx.x) / gridDim.x);
     const int it_end = (int)(((long long)total * (blockIdx.x + 1)) / gridDim.x);
     if (it_begin >= it_end) return;
@@ -486,6 +463,7 @@ cudaError_t gemv_take_error(unsigned *code, unsigned *info) {
     cudaError_t e = cudaMemcpyFromSymbol(code, g_gemv_error, sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemcpyFromSymbol(info, g_gemv_error_info, sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv_error, &zero, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv_error_info, &zero, sizeof(unsigned));
     return e;
 }
 
@@ -505,9 +483,6 @@ cudaError_t launch_ffn_gemv(const LayerView &L, const uint16_t *x, int T, int k,
     p.sorted_route = sorted_route;
     p.h = static_cast<uint16_t *>(ws);
     p.rows = rows;
-    // w2 into L2 during phase 1 when every routed expert together is far below
-    // the L2 size (at most T*k distinct experts)
-    p.prefetch_w2 = (uint64_t)T * k * L.stride <= (uint64_t)100 << 20;
     if (L.fmt == MOE_W_BF16) return launch_fmt<MOE_W_BF16>(p, n_sm, s);
     if (L.fmt == MOE_W_INT8) return launch_fmt<MOE_W_INT8>(p, n_sm, s);
     return launch_fmt<MOE_W_INT4>(p, n_sm, s);

@@ -356,6 +356,14 @@ __device__ __forceinline__ const uint8_t *scale_blob(const TcParams &p, int e) {
     return b ? b : p.L.home + (uint64_t)e * p.L.stride;
 }
 
+// Storage column of K element c in the int4 kernels' B operand (xs, h): within
+// every run of 8, elements 1 and 2, 5 and 6 trade places (the order in which
+// the int4 expansion lays out A; an involution).  Identity for bf16 and int8.
+template <int FMT>
+__host__ __device__ __forceinline__ int k_order(int c) {
+    return FMT == MOE_W_INT4 ? ((c & ~3) | ((c & 1) << 1) | ((c >> 1) & 1)) : c;
+}
+
 // ---------------------------------------------------------------- the kernel
 template <int FMT>
 __host__ __device__ constexpr int kRawBytes() { return FMT == MOE_W_BF16 ? 0 : kRawRowBytes * kBlockM; }
@@ -646,7 +654,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                                     continue;
                                 }
                                 const float g = v[i] * scale, up = xrow[i];
-                                p.h[(size_t)(it.row0 + j) * p.L.I + icol] = f32_to_bf16_rne(gelu_tanh(g) * up);
+                                p.h[(size_t)(it.row0 + j) * p.L.I + k_order<FMT>(icol)] =
+                                    f32_to_bf16_rne(gelu_tanh(g) * up);
                             }
                         }
                         __syncwarp();
@@ -732,7 +741,15 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     uint32_t o[32];  // bf16 pairs (weights 64 hf + 2j, +1 in the low, high half)
                     if (FMT == MOE_W_INT4) {
                         // bf16 128 + n (n in the low mantissa bits of 128.0 = 0x4300),
-                        // minus 136 -> n - 8 exactly, times s -> one rounding
+                        // minus 136 -> n - 8 exactly, times s -> one rounding.
+                        // A word holds weights 0..7 of a run of 8 (byte j: 2j low, 2j+1
+                        // high nibble).  Masking the low and the high nibbles gives two
+                        // words of one nibble per byte, and each byte permute then pairs
+                        // two of them with the 0x43 exponent byte: pairs (0,2) (1,3)
+                        // (4,6) (5,7).  So within every run of 8 the A columns hold K
+                        // order 0 2 1 3 4 6 5 7 (swap 1<->2 and 5<->6); the B operand of
+                        // the int4 kernels (xs and h) is stored in the same order, which
+                        // leaves every dot product unchanged.
                         const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
 #pragma unroll
                         for (int c = 0; c < 2; ++c) {
@@ -740,14 +757,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                             const uint32_t words[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                // byte j of the word = weight 2j (low nibble), 2j+1 (high)
-                                const uint32_t w = words[i], w4 = w >> 4;
+                                const uint32_t lo = words[i] & 0x0F0F0F0Fu, hi = (words[i] >> 4) & 0x0F0F0F0Fu;
+                                const uint32_t pr[4] = {__byte_perm(lo, 0x43434343u, 0x4140),
+                                                        __byte_perm(hi, 0x43434343u, 0x4140),
+                                                        __byte_perm(lo, 0x43434343u, 0x4342),
+                                                        __byte_perm(hi, 0x43434343u, 0x4342)};
 #pragma unroll
                                 for (int j = 0; j < 4; ++j) {
-                                    // {w.byte j, -, (w >> 4).byte j, -}: n_lo and n_hi in the low bits of each half
-                                    const uint32_t dup =
-                                        __byte_perm(w, w4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
-                                    uint32_t v = (dup & 0x000F000Fu) | 0x43004300u;
+                                    uint32_t v = pr[j];
                                     __nv_bfloat162 q = *reinterpret_cast<__nv_bfloat162 *>(&v);
                                     q = __hmul2(__hsub2(q, bias), s2);
                                     o[16 * c + 4 * i + j] = *reinterpret_cast<uint32_t *>(&q);
@@ -803,9 +820,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 }
 
 // x rows gathered into sorted-route order: xs[s] = x[sorted_route[s] / k] for
-// s < offsets[E] (16 bytes per thread).
+// s < offsets[E] (16 bytes per thread).  With `perm` (the int4 kernels) each run
+// of 8 elements is stored in the order k_order<MOE_W_INT4> gives.
 __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ sorted_route,
-                              const int32_t *__restrict__ offsets, int E, int k, int H, int R,
+                              const int32_t *__restrict__ offsets, int E, int k, int H, int R, int perm,
                               uint16_t *__restrict__ xs) {
     // programmatic dependent launch: wait for the previous kernel before
     // touching memory, then let the next one be scheduled
@@ -823,8 +841,15 @@ __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__r
             record_error(0x2004u, (unsigned)s);
             continue;
         }
-        reinterpret_cast<uint4 *>(xs + (size_t)s * H)[c] =
-            __ldg(reinterpret_cast<const uint4 *>(x + (size_t)tok * H) + c);
+        uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)tok * H) + c);
+        if (perm) {  // elements (0,1)(2,3)(4,5)(6,7) -> (0,2)(1,3)(4,6)(5,7)
+            const uint4 v = u;
+            u.x = __byte_perm(v.x, v.y, 0x5410);
+            u.y = __byte_perm(v.x, v.y, 0x7632);
+            u.z = __byte_perm(v.z, v.w, 0x5410);
+            u.w = __byte_perm(v.z, v.w, 0x7632);
+        }
+        reinterpret_cast<uint4 *>(xs + (size_t)s * H)[c] = u;
     }
 }
 
@@ -942,7 +967,7 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
         const int64_t n = (int64_t)R * (H / 8);
         const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)n_sm * 8);
         err = launch_pdl(k_gather_rows, dim3((unsigned)blocks), dim3(256), 0, s, x, sorted_route, offsets, L.E, k, H, R,
-                         xs);
+                         (int)(L.fmt == MOE_W_INT4), xs);
         if (err != cudaSuccess) return err;
     }
     // 2. tensor maps: weights (home and pool, as rows of one matrix), activations
@@ -1023,6 +1048,7 @@ cudaError_t tc_take_error(unsigned *code, unsigned *info) {
     cudaError_t e = cudaMemcpyFromSymbol(code, g_tc_error, sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemcpyFromSymbol(info, g_tc_error_info, sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_tc_error_info, &zero, sizeof(unsigned));
     return e;
 }
 

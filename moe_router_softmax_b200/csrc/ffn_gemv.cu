@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
             const int n = (e < E) ? __ldg(p.counts + e) : 0;
             const bool act = n > 0;
             const unsigned m = __ballot_sync(0xffffffffu, act);
-            const int items = act ? tiles * ((n + kNTM - 1) / kNTM) : 0;
+            const int items = act ? tiles * ((n + NTMAX - 1) / NTMAX) : 0;
             int inc = items;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -368,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
         const int chunk = rem / tiles, tile = rem - chunk * tiles;
         const int e = s_act[a];
         const int n_e = __ldg(p.counts + e);
-        const int row0 = __ldg(p.offsets + e) + chunk * kNTM;
-        const int nt = min(kNTM, n_e - chunk * kNTM);
+        const int row0 = __ldg(p.offsets + e) + chunk * NTMAX;
+        const int nt = min(NTMAX, n_e - chunk * NTMAX);
         const uint8_t *blob = expert_blob(p.L, e);
         if (blob == nullptr) {
             // the expert's slot is past the pool: nothing of this item is read or
@@ -399,10 +399,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
 }
 
 // Lanes per row group: the largest power of two <= 32 that leaves every lane
-// at least `min_per_lane` chunks of a row (so a group is never mostly idle).
-int pick_lg(int nchunks) {
+// at least `per_lane` chunks of a row (so a group is never mostly idle).  Batches
+// with several routes per expert take 8 chunks per lane (long, reused rows); the
+// one-token kernel takes 1, so that a row is spread over more lanes and the few
+// routed experts' rows form enough work items to occupy every SM.
+int pick_lg(int nchunks, int per_lane) {
     int lg = 32;
-    while (lg > 1 && nchunks < lg * 8) lg >>= 1;
+    while (lg > 1 && nchunks < lg * per_lane) lg >>= 1;
     return lg;
 }
 
@@ -411,8 +414,8 @@ cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
     FfnParams p = p0;
     const int K = PHASE == 1 ? p.L.H : p.L.I;
     const int nchunks = K / Fmt<FMT>::kElems;
-    p.lg = pick_lg(nchunks);
-    const size_t smem = (size_t)kNTM * K * sizeof(float);
+    p.lg = pick_lg(nchunks, NTMAX == 1 ? 1 : 8);
+    const size_t smem = (size_t)NTMAX * K * sizeof(float);
     auto kern = k_ffn_gemv<FMT, PHASE, RWP, U, NTMAX>;
     // one-time set-up per device and shared-memory size (kept out of stream
     // capture: after the first call a launch is the only API call made here)

@@ -157,9 +157,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Non-blocking test of a phase (the common case: it has already completed).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait: false (and the abort flag set) if the phase did not complete in
 // time or another role already gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_test_wait(bar, parity)) return true;
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
@@ -552,6 +565,13 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             uint32_t pa = 0, pb = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
+            // K step j of an atom accumulates into partial accumulator j % nacc
+            // (columns dj[j]); it overwrites it on the atom's first use (j < nacc).
+            // nacc is 1, 2 or 4: a mask and a shift, no division per MMA.
+            const int lg_acc = nacc == 4 ? 2 : (nacc == 2 ? 1 : 0);
+            uint32_t dj[kBlockK / 16];
+#pragma unroll
+            for (int j = 0; j < kBlockK / 16; ++j) dj[j] = (uint32_t)((j & (nacc - 1)) * n_block);
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
                 const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, &s_abort)) break;
@@ -566,29 +586,31 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     // they completed a_full, so only bf16 waits for it here
                     if (!kDeq && !mbar_wait(&b_full[sb], pb, &s_abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t b0 = smem_u32(sB + sb * b_slot_bytes);
+                    // descriptors of the stage's first K step; one 16-wide K step is 32
+                    // bytes, 2 in the descriptor's start-address field (which cannot
+                    // carry: every address stays below 256 KB)
+                    const uint64_t bd = sw128_desc(smem_u32(sB + sb * b_slot_bytes));
+                    const int na = atoms_at(kk);
                     if (kDeq) {
                         // A stage sa: TMEM columns C::kAccCols + A_COLS sa .., 32 per atom,
                         // 8 per 16-wide K step
                         const uint32_t a_t = tmem + (uint32_t)(C::kAccCols + sa * A_COLS);
-                        const int na = atoms_at(kk);
                         for (int a = 0; a < na; ++a) {
+                            const uint64_t bda = bd + (uint64_t)((a * b_atom_bytes) >> 4);
 #pragma unroll
                             for (int j = 0; j < kBlockK / 16; ++j)
-                                tc_mma_bf16_ts(d + (uint32_t)((j % nacc) * n_block), a_t + 32 * a + 8 * j,
-                                               sw128_desc(b0 + a * b_atom_bytes + 32 * j), idesc,
-                                               (kk | a | (j / nacc)) != 0);
+                                tc_mma_bf16_ts(d + dj[j], a_t + 32 * a + 8 * j, bda + (uint64_t)(2 * j), idesc,
+                                               (kk | a | (j >> lg_acc)) != 0);
                         }
                     } else {
-                        const uint32_t a0 = smem_u32(sA + sa * ATOMS * kATileBytes);
-                        const int na = atoms_at(kk);
+                        const uint64_t ad = sw128_desc(smem_u32(sA + sa * ATOMS * kATileBytes));
                         for (int a = 0; a < na; ++a) {
+                            const uint64_t ada = ad + (uint64_t)((a * kATileBytes) >> 4);
+                            const uint64_t bda = bd + (uint64_t)((a * b_atom_bytes) >> 4);
 #pragma unroll
                             for (int j = 0; j < kBlockK / 16; ++j)
-                                tc_mma_bf16(d + (uint32_t)((j % nacc) * n_block),
-                                            sw128_desc(a0 + a * kATileBytes + 32 * j),
-                                            sw128_desc(b0 + a * b_atom_bytes + 32 * j), idesc,
-                                            (kk | a | (j / nacc)) != 0);
+                                tc_mma_bf16(d + dj[j], ada + (uint64_t)(2 * j), bda + (uint64_t)(2 * j), idesc,
+                                            (kk | a | (j >> lg_acc)) != 0);
                         }
                     }
                     tc_commit(&a_empty[sa]);
@@ -727,8 +749,13 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                 __nv_bfloat162 s2 = __floats2bfloat162_rn(0.0f, 0.0f);
                 if (FMT == MOE_W_INT4 && mine)
                     s2 = __bfloat162bfloat162(__ushort_as_bfloat16(__ldg(srow + kk * ATOMS + hf)));
-                // the codes have landed, and the MMAs are done with this A slot
-                if (!mbar_wait(&r_full[rstage], rphase, &s_abort)) { ok = false; break; }
+                // the codes have landed, and the MMAs are done with this A slot (a
+                // single group takes both halves of an int4 raw stage, so it waits
+                // for the codes once; two groups each wait for their own half)
+                if ((sub == 0 || C::kDeqGroups > 1) && !mbar_wait(&r_full[rstage], rphase, &s_abort)) {
+                    ok = false;
+                    break;
+                }
                 if (!mbar_wait(&a_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
                 tc_fence_after();
                 if (mine) {

@@ -399,10 +399,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
 }
 
 // Lanes per row group: the largest power of two <= 32 that leaves every lane
-// at least `per_lane` chunks of a row (so a group is never mostly idle).  Batches
-// with several routes per expert take 8 chunks per lane (long, reused rows); the
-// one-token kernel takes 1, so that a row is spread over more lanes and the few
-// routed experts' rows form enough work items to occupy every SM.
+// at least `per_lane` chunks of a row (so a group is never mostly idle).
 int pick_lg(int nchunks, int per_lane) {
     int lg = 32;
     while (lg > 1 && nchunks < lg * per_lane) lg >>= 1;
@@ -414,7 +411,7 @@ cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
     FfnParams p = p0;
     const int K = PHASE == 1 ? p.L.H : p.L.I;
     const int nchunks = K / Fmt<FMT>::kElems;
-    p.lg = pick_lg(nchunks, NTMAX == 1 ? 1 : 8);
+    p.lg = pick_lg(nchunks, 8);
     const size_t smem = (size_t)NTMAX * K * sizeof(float);
     auto kern = k_ffn_gemv<FMT, PHASE, RWP, U, NTMAX>;
     // one-time set-up per device and shared-memory size (kept out of stream

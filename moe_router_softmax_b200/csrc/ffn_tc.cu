@@ -185,6 +185,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         }
     }
 }
+// Bounded wait that ignores the abort flag (for the drain after an abort).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, long long cycles) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > cycles) return false;
+    return true;
+}
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -382,12 +389,22 @@ template <int FMT>
 __host__ __device__ constexpr int kRawBytes() { return FMT == MOE_W_BF16 ? 0 : kRawRowBytes * kBlockM; }
 
 // warps: 0 A/raw producer, 1 MMA, 2..5 epilogue, 6 B producer, 7.. dequant
+// (kDeqGroups groups of kDeqWarps), then one gate warp per dequant group
 constexpr int kWarpB = 2 + kEpiWarps;
 constexpr int kWarpDeq0 = kWarpB + 1;
 
 template <int FMT, int CFG>
 __host__ __device__ constexpr int tc_threads() {
-    return 32 * (kWarpDeq0 + (FMT == MOE_W_BF16 ? 0 : TcCfg<FMT, CFG>::kDeqGroups * kDeqWarps));
+    return 32 * (kWarpDeq0 + (FMT == MOE_W_BF16 ? 0 : TcCfg<FMT, CFG>::kDeqGroups * (kDeqWarps + 1)));
+}
+
+// Named hardware barriers between a dequant group's gate warp and its eight
+// warps (id 0 is __syncthreads): one per (group, A slot).
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 template <int FMT, int PHASE, int CFG>
@@ -439,7 +456,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SA; ++i) {
-            mbar_init(&a_full[i], kDeq ? kDeqWarps : 1);
+            mbar_init(&a_full[i], kDeq ? kDeqWarps + 1 : 1);  // int: eight dequant warps and the gate
             mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < kMaxBSlots; ++i) {
@@ -707,6 +724,51 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             if (lane == 0) mbar_arrive(&tempty[acc]);
             if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1; }
         }
+    } else if (kDeq && warp >= kWarpDeq0 + C::kDeqGroups * kDeqWarps) {
+        // ---------------------------------------------------- gate warps
+        // One per dequant group: for each of the group's stages it waits until
+        // the codes have landed and the MMAs are done with the A slot, releases
+        // the group's eight warps through a named barrier, then waits for the
+        // stage's B slot and arrives on a_full with them.  Every mbarrier wait
+        // costs a warp ~130 cycles even when the phase has completed; taking all
+        // of them here leaves the dequant warps one hardware barrier per stage.
+        // The gate never skips a release (after an abort it releases without
+        // waiting), so the dequant warps cannot block on a stage that is never
+        // released.
+        const int group = warp - (kWarpDeq0 + C::kDeqGroups * kDeqWarps);
+        int stage = 0, rstage = 0, bstage = 0;
+        uint32_t phase = 0, rphase = 0, bphase = 0;
+        uint32_t step = 0;
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            for (int kk = 0; kk < nk; ++kk, ++step) {
+                const int sub = kk % SUB;
+                const bool raw_last = sub == SUB - 1 || kk == nk - 1;
+                if ((int)(step % C::kDeqGroups) == group) {
+                    bool ok = !s_abort;
+                    // a single group takes both halves of an int4 raw stage and
+                    // waits for its codes once; two groups each wait for their half
+                    if (ok && (sub == 0 || C::kDeqGroups > 1)) ok = mbar_wait(&r_full[rstage], rphase, &s_abort);
+                    if (ok) ok = mbar_wait(&a_empty[stage], phase ^ 1, &s_abort);
+                    // after an abort the slot's waits are skipped, so make sure the
+                    // group has left this slot's previous release (its warps and
+                    // this gate arrive on a_full after every release) before
+                    // releasing it again: a named barrier must never collect two
+                    // releases at once
+                    if (!ok) mbar_wait_for(&a_full[stage], phase ^ 1, kWaitCycles / 4);
+                    __syncwarp();
+                    named_arrive(1 + group * SA + stage, 32 * (kDeqWarps + 1));
+                    // while the group expands the stage, wait for its B slot; the
+                    // gate's own arrival on a_full then tells the MMA issuer that A
+                    // and B are both ready
+                    if (ok) mbar_wait(&b_full[bstage], bphase, &s_abort);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&a_full[stage]);
+                }
+                if (++stage == SA) { stage = 0; phase ^= 1; }
+                if (++bstage == b_slots) { bstage = 0; bphase ^= 1; }
+                if (raw_last && ++rstage == SR) { rstage = 0; rphase ^= 1; }
+            }
+        }
     } else if (kDeq) {
         // ---------------------------------------------------- dequantisation
         // two threads per tile row, each expanding one 64-wide atom of the
@@ -714,51 +776,54 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         // columns 32 hf .. 32 hf + 31 of the A stage.  A warp may only reach
         // TMEM lanes 32 (warp % 4) .. +31, so the row is taken from the warp's
         // lane quadrant; the eight warps of a group cover each quadrant twice
-        // (both atoms of its rows).  The first warp of the group also waits for
-        // the stage's B slot, so a completed a_full means A and B are both ready.
+        // (both atoms of its rows).  A stage starts when the group's gate warp
+        // releases it (codes, A slot and B slot all ready), so a completed
+        // a_full means A and B are both ready for the MMAs.
         const int dw = warp - kWarpDeq0;              // 0 .. C::kDeqGroups*kDeqWarps-1
         const int group = dw / kDeqWarps;
         const int quad = warp & 3;
         const int r = quad * 32 + lane, hf = (dw % kDeqWarps) / 4;
-        const bool b_waiter = (dw % kDeqWarps) == 0;
-        int stage = 0, rstage = 0, bstage = 0;
-        uint32_t phase = 0, rphase = 0, bphase = 0;
+        int stage = 0, rstage = 0;
         uint32_t step = 0;                              // stages seen, across items
-        for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
             const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
             const uint8_t *blob = scale_blob(p, it.e);
             const int wrow = PHASE == 1 ? (r < 64 ? it.m0 * 64 + r : p.L.I + it.m0 * 64 + r - 64)
                                         : min(it.m0 * kBlockM + r, p.n_units - 1);
             const uint16_t *srow = reinterpret_cast<const uint16_t *>(blob + (PHASE == 1 ? p.L.off.s13 : p.L.off.s2)) +
                                    (size_t)wrow * (p.K / 64);
-            bool ok = true;
+            // int4: the group scale of this thread's atom is loaded one of the
+            // group's stages ahead (the scales are read from global memory, where
+            // a miss costs a few hundred cycles that the current stage then hides)
+            auto scale_at = [&](int kq) -> uint16_t {
+                return (kq < nk && hf < atoms_at(kq)) ? __ldg(srow + kq * ATOMS + hf) : (uint16_t)0;
+            };
+            uint16_t s_next = 0;
+            if (FMT == MOE_W_INT4) {
+                const int k0 = (int)((group - (int)(step % C::kDeqGroups) + C::kDeqGroups) % C::kDeqGroups);
+                s_next = scale_at(k0);
+            }
             for (int kk = 0; kk < nk; ++kk, ++step) {
                 const int sub = kk % SUB;
                 const bool raw_last = sub == SUB - 1 || kk == nk - 1;  // last stage of this raw stage
                 if ((int)(step % C::kDeqGroups) != group) {   // the other group's stage
-                    if (++stage == SA) { stage = 0; phase ^= 1; }
-                    if (++bstage == b_slots) { bstage = 0; bphase ^= 1; }
+                    if (++stage == SA) stage = 0;
                     if (raw_last) {
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&r_empty[rstage]);
-                        if (++rstage == SR) { rstage = 0; rphase ^= 1; }
+                        if (++rstage == SR) rstage = 0;
                     }
                     continue;
                 }
                 const bool mine = hf < atoms_at(kk);  // this thread's atom lies inside K
                 __nv_bfloat162 s2 = __floats2bfloat162_rn(0.0f, 0.0f);
-                if (FMT == MOE_W_INT4 && mine)
-                    s2 = __bfloat162bfloat162(__ushort_as_bfloat16(__ldg(srow + kk * ATOMS + hf)));
-                // the codes have landed, and the MMAs are done with this A slot (a
-                // single group takes both halves of an int4 raw stage, so it waits
-                // for the codes once; two groups each wait for their own half)
-                if ((sub == 0 || C::kDeqGroups > 1) && !mbar_wait(&r_full[rstage], rphase, &s_abort)) {
-                    ok = false;
-                    break;
+                if (FMT == MOE_W_INT4) {
+                    s2 = __bfloat162bfloat162(__ushort_as_bfloat16(s_next));
+                    s_next = scale_at(kk + C::kDeqGroups);
                 }
-                if (!mbar_wait(&a_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
+                named_sync(1 + group * SA + stage, 32 * (kDeqWarps + 1));
                 tc_fence_after();
-                if (mine) {
+                if (mine && !s_abort) {
                     // the raw tile landed 128-byte swizzled (16-byte chunk j of row r
                     // at chunk j ^ (r % 8)), so the 32 rows a warp reads at once
                     // spread over all banks
@@ -822,18 +887,15 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     tmem_st16(ta + 16, o + 16);
                     tmem_st_wait();
                 }
-                if (b_waiter && !mbar_wait(&b_full[bstage], bphase, &s_abort)) { ok = false; break; }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&a_full[stage]);
                     if (raw_last) mbar_arrive(&r_empty[rstage]);
                 }
-                if (++stage == SA) { stage = 0; phase ^= 1; }
-                if (++bstage == b_slots) { bstage = 0; bphase ^= 1; }
-                if (raw_last && ++rstage == SR) { rstage = 0; rphase ^= 1; }
+                if (++stage == SA) stage = 0;
+                if (raw_last && ++rstage == SR) rstage = 0;
             }
-            if (!ok) break;
         }
     }
 

@@ -159,7 +159,7 @@ class MoeLayer:
                  slot_table: torch.Tensor | None = None, expert_bytes: int | None = None,
                  pool_slots: int | None = None):
         self.fmt, self.E, self.H, self.I = int(fmt), int(E), int(H), int(I)
-        self.expert_bytes = int(expert_bytes or moe_expert_bytes(fmt, H, I))
+        self.expert_bytes = int(expert_bytes or (moe_expert_bytes(fmt, H, I) + 255) // 256 * 256)
         self.home, self.pool, self.slot_table = home, pool, slot_table
         if pool_slots is None:
             pool_slots = 0 if pool is None else pool.numel() // self.expert_bytes
@@ -463,7 +463,7 @@ def make_layer(fmt: int, w13: torch.Tensor, w2: torch.Tensor, stream=None) -> Mo
     formats, then packed by moe_pack_expert)."""
     E, I2, H = w13.shape
     I = I2 // 2
-    eb = moe_expert_bytes(fmt, H, I)
+    eb = (moe_expert_bytes(fmt, H, I) + 255) // 256 * 256   # blob stride: a multiple of 256 bytes
     home = torch.empty(E * eb, dtype=torch.uint8, device=w13.device)
     for e in range(E):
         blob = home[e * eb:(e + 1) * eb]

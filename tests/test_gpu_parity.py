@@ -550,3 +550,25 @@ def test_one_token_with_repeated_ids(fmt):
     got = rows.cpu().numpy()[rp.cpu().numpy().ravel()[valid]]
     assert rel_err(got, orows[valid]) <= FFN_TOL
     assert rel_err(bf16_dev_to_f64(y), oracle.combine(orows, ids, w, E)) <= FFN_TOL
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("E,H,I,k", [(8, 256, 128, 2), (6, 1024, 320, 4), (16, 512, 192, 8), (12, 2816, 704, 8),
+                                     (4, 64, 64, 1)])
+def test_one_token_every_element(fmt, E, H, I, k):
+    """One-token batches through the GEMV kernels (the one-token kernels spread
+    the rows of every routed expert over all lane groups; phase 1 writes the gate
+    and up projections, phase 2 forms h while staging it): every row against the
+    oracle, at shapes whose rows split unevenly over the lane groups."""
+    w13, w2 = syn.expert_weights(E, H, I, seed=E * 7 + I)
+    x = syn.activations(1, H, seed=H)
+    lg = syn.router_logits(1, E, "normal", seed=k)
+    L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    ids, w, counts, offsets, sr, rp, rows, y = _run_layer(L, torch.from_numpy(lg).to(DEV), xd, k,
+                                                          path=moe.MOE_FFN_GEMV)
+    oi, ow, orows, oy = oracle.moe_layer(oracle_layer_for(fmt, w13, w2), lg, x, k)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    assert rel_err(rows.cpu().numpy()[rp.cpu().numpy()], orows) <= FFN_TOL
+    assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
+    assert moe.moe_take_device_errors() == (0, 0)

@@ -259,7 +259,7 @@ class Runner:
         R = self.T * self.k
         auto_tc = R >= TC_MIN_ROUTES[self.layers[0].fmt]
         tc = self.path == self.moe.MOE_FFN_TC or (self.path == self.moe.MOE_FFN_AUTO and auto_tc)
-        return 4 + (3 if tc else 2)
+        return 3 + (3 if tc else 2)
 
     def distinct_experts(self):
         """Distinct routed experts of each batch (read back from our own routing)."""
@@ -1191,7 +1191,7 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
                       "routes_on_resident_slots": round(sum(share) / len(share), 4) if share else None},
         "sweep": sweep,
         "hbm_peak_gbs": hbm_peak,
-        "gpu_launches": steps_done * L * (4 + (3 if (path == moe.MOE_FFN_TC or
+        "gpu_launches": steps_done * L * (3 + (3 if (path == moe.MOE_FFN_TC or
                                                       (path == moe.MOE_FFN_AUTO and T * k >= TC_MIN_ROUTES[s4.fmt]))
                                                      else 2))
                         + (steps_done // 8) * L * (2 if device_refresh else 0),

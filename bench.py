@@ -44,13 +44,33 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, summed
-# over the grouped-FFN launches of one call) from one-pass ncu captures of the
-# kernels as they stand, keyed by (workload, --path): (bytes, what was captured).
-# A workload without an entry reports null.
+# over the gather and grouped-FFN launches of one layer call) from one-pass ncu
+# captures of the kernels as they stand, keyed by (workload, --path):
+# (bytes, algorithmic bytes of the captured call, what was captured).  The
+# captured call is the first graph-replayed step of
+#   bench.py --quick --headline-only --steps 10 --warmup 3 --layers 2
+#            --no-cpu-baseline [--config C] [--tokens T]
+# (batch 3 of seed 0; ncu -s skips the 8 distinct-expert probes and the 3 warm-up
+# calls), whose distinct experts differ from the bench's 8-batch average, so the
+# traffic is compared with that call's own algorithmic bytes.  A workload
+# without an entry reports null.
+_CAPTURE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+            "--clock-control none -k regex:'k_ffn|k_gather_rows', one layer call of bench.py --quick "
+            "--headline-only --layers 2")
 NCU_TRAFFIC_BYTES = {
-    ("moe-layer-bf16-decode-T64", "auto"): (1.5134e9, "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum "
-                                                      "--clock-control none: gather + both tcgen05 launches, "
-                                                      "bench.py --config decode-bf16 --quick --layers 2"),
+    ("moe-layer-bf16-decode-T64", "auto"): (1508265472, 1499103232, _CAPTURE + " (gather + 2 tcgen05 launches)"),
+    ("moe-layer-bf16-decode-T8", "auto"): (584258304, 582889472, _CAPTURE + " --tokens 8 (gather + 2 tcgen05 launches)"),
+    ("moe-layer-bf16-decode-T1", "auto"): (95552000, 95163904, _CAPTURE + " --tokens 1 (2 GEMV launches)"),
+    ("moe-layer-int8-decode-T64", "auto"): (309138176, 304539136,
+                                            _CAPTURE + " --config decode-int8 (gather + 2 tcgen05 launches)"),
+    ("moe-layer-int8-decode-T8", "auto"): (143885056, 143187968,
+                                           _CAPTURE + " --config decode-int8 --tokens 8 (gather + 2 tcgen05 launches)"),
+    ("moe-layer-int8-decode-T1", "auto"): (47808512, 47719936,
+                                           _CAPTURE + " --config decode-int8 --tokens 1 (2 GEMV launches)"),
+    ("moe-layer-int4-decode-T64", "auto"): (404842496, 398464000,
+                                            _CAPTURE + " --config int4-decode (gather + 2 tcgen05 launches)"),
+    ("moe-layer-int4-prefill-T1024", "auto"): (524295936, 410189824,
+                                               _CAPTURE + " --config int4-prefill (gather + 2 tcgen05 launches)"),
 }
 
 # routes from which the library's AUTO path takes the tensor-core FFN (bf16, int8,
@@ -239,6 +259,7 @@ class Runner:
         self.ws = torch.empty(max(moe.moe_grouped_ffn_workspace(layers[0], T, k), 16), dtype=torch.uint8, device=dev)
         self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
         self.ev = None
+        self.side = None
 
     def step(self, i, ffn_events=None):
         moe = self.moe
@@ -248,11 +269,27 @@ class Runner:
         moe.moe_route_topk(lg, self.k, self.ids, self.w)
         counts, offsets, sr, rp = moe.moe_permute(self.ids, L.E, hits=self.hits[li], out=self.perm)
         if ffn_events is not None:
-            ffn_events[0].record()
+            self._mark(ffn_events[0])
         moe.moe_grouped_ffn(L, x, self.k, counts, offsets, sr, rows=self.rows, ws=self.ws, path=self.path)
         if ffn_events is not None:
-            ffn_events[1].record()
+            self._mark(ffn_events[1])
         moe.moe_combine(self.rows, rp, self.w, self.y)
+
+    def _mark(self, ev):
+        """Record a timing event on a side stream forked from the current one:
+        inside a graph capture the event node then hangs off the last kernel
+        (it fires when that kernel completes) without sitting between two
+        kernels, so the programmatic-launch edges of the main chain stay."""
+        torch = self.torch
+        if self.side is None:
+            self.side = torch.cuda.Stream()
+        self.side.wait_stream(torch.cuda.current_stream())
+        ev.record(self.side)
+
+    def join(self):
+        """Join the side stream back (the end of a capture that used _mark)."""
+        if self.side is not None:
+            self.torch.cuda.current_stream().wait_stream(self.side)
 
     def launches_per_step(self):
         """route, permute, FFN (2 GEMV launches, or gather + 2 tensor-core launches), combine"""
@@ -276,11 +313,11 @@ FFN_SAMPLE_EVERY = 1
 
 def _capture(torch, runner, first, n):
     """One CUDA graph of n consecutive steps, with an external event pair around
-    the grouped-FFN launches of every FFN_SAMPLE_EVERY-th step (event record
-    nodes inside the graph; every step, so a 20-step run gives 20 pairs).  An
-    event node between two kernels also cuts their programmatic-launch edge: the
-    permute -> FFN and FFN -> combine hand-offs of a sampled step wait for the
-    previous kernel to finish (the FFN's own launches keep theirs)."""
+    the grouped-FFN launches of every FFN_SAMPLE_EVERY-th step (every step, so a
+    20-step run gives 20 pairs).  The event nodes sit on a side stream: the first
+    fires when the permute kernel completes, the second when the FFN's last
+    launch does, and neither cuts the programmatic-launch edges of the kernel
+    chain (an event node between two kernels would)."""
     g = torch.cuda.CUDAGraph()
     sampled = [j for j in range(n) if j % FFN_SAMPLE_EVERY == FFN_SAMPLE_EVERY // 2] or [0]
     evs = {j: (torch.cuda.Event(enable_timing=True, external=True),
@@ -288,13 +325,15 @@ def _capture(torch, runner, first, n):
     with torch.cuda.graph(g):
         for j in range(n):
             runner.step(first + j, evs.get(j))
+        runner.join()
     return g, list(evs.values())
 
 
 def time_steps(torch, runner, steps, warmup, dist):
     """Exactly `steps` steps between two events, replayed from CUDA graphs of one
     rotation over the layers (so Python launch overhead is out of the timed
-    region).  Returns (total ms, per-step FFN ms from the last replay of each graph)."""
+    region; each graph is launched once before it, untimed).  Returns (total ms,
+    per-step FFN ms from the last replay of each graph)."""
     G = len(runner.layers)
     for i in range(warmup):
         runner.step(i)
@@ -305,6 +344,8 @@ def time_steps(torch, runner, steps, warmup, dist):
         graphs.append(_capture(torch, runner, warmup, G))
     if rem:
         graphs.append(_capture(torch, runner, warmup, rem))
+    for g, _ in graphs:  # a graph's first launch also uploads it: keep that out of the timed region
+        g.replay()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -564,18 +605,19 @@ def ffn_roofline(T, k, H, I, eb, distinct, ffn_ms, peaks, traffic):
     gbs = alg_bytes / (ffn_ms / 1e3) / 1e9
     flops = 2.0 * T * k * 3 * H * I
     tflops = flops / (ffn_ms / 1e3) / 1e12
-    tr = None if traffic is None else traffic[0]
-    tr_src = None if traffic is None else traffic[1]
+    tr, tr_alg, tr_src = (None, None, None) if traffic is None else traffic
     if T > 64:
         return {"bound": "tensor", "achieved": round(tflops, 1), "peak": tf_sust, "unit": "TFLOP/s",
-                "frac": round(tflops / tf_sust, 4), "traffic": tr, "traffic_capture": tr_src,
+                "frac": round(tflops / tf_sust, 4), "traffic": tr, "traffic_alg_bytes": tr_alg,
+                "traffic_capture": tr_src,
                 "peak_source": f"{src} sustained bf16 (bf16_tflops_sustained)",
                 "alg_flops_per_launch": flops,
                 "hbm": {"achieved_gbs": round(gbs, 1), "peak": hbm_peak, "frac": round(gbs / hbm_peak, 4),
                         "alg_bytes_per_launch": int(alg_bytes)},
                 "avg_launch_us": round(ffn_ms * 1e3, 2)}
     return {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(gbs / hbm_peak, 4), "traffic": tr, "traffic_capture": tr_src,
+            "frac": round(gbs / hbm_peak, 4), "traffic": tr, "traffic_alg_bytes": tr_alg,
+            "traffic_capture": tr_src,
             "peak_source": f"{src} (hbm_gbs)", "alg_bytes_per_launch": int(alg_bytes),
             "avg_launch_us": round(ffn_ms * 1e3, 2)}
 

@@ -329,7 +329,8 @@ MOE_API moe_status moe_copy_to_slots(const void *home, void *pool, uint64_t expe
                              const int32_t *slots, int32_t n, moe_stream_t stream);
 
 /* Diagnostics: synchronise the device, then read and clear the first problem
- * the tensor-core kernels recorded since the last call.  *code = 0 and MOE_OK
+ * the FFN kernels recorded since the last call (the tensor-core kernels' record
+ * first, then the GEMV kernels': a slot past the pool).  *code = 0 and MOE_OK
  * if none; MOE_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the
  * kernel then drained out without finishing its work); MOE_ERR_CUDA if an
  * index check failed (the access was skipped; *info holds the value). */

@@ -367,7 +367,8 @@ moe_status moe_take_device_errors(uint32_t *code, uint32_t *info) {
     *code = c;
     *info = i;
     if (c >= 0x1000u && c < 0x2000u)
-        return set_error(MOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (warp %u)", c & 0xFFFu);
+        return set_error(MOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (warp %u, barrier word %#x)",
+                         c & 0xFFFu, i);
     if (c == 0x2005u || c == 0x2006u)
         return set_error(MOE_ERR_CUDA, "slot %u of the slot table is past the pool; that expert's routes were skipped",
                          i);

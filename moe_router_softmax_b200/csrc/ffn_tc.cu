@@ -36,7 +36,9 @@
 // programmatic dependent launches: only the B producer waits for the previous
 // kernel.  Every mbarrier wait is bounded (and suspends in hardware while it
 // waits); on timeout the kernel records an error word and every role drains
-// out.
+// out.  The weight loads carry an evict-first L2 policy (each weight is read
+// once) and the route-tile loads an evict-last one (every M tile of an expert
+// re-reads them), so the weight stream does not push xs and h out of L2.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -195,19 +197,34 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, lo
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+// L2 policies: the weight stream is read once (evict first); the route tiles
+// are re-read by every M tile of an expert (evict last).
+__device__ __forceinline__ uint64_t l2_policy_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
+                                            uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;"
+        ::"r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
         : "memory");
 }
 // 3-D box {x, y, z} of a weight map: x along the row, y the row of the matrix,
 // z the blob (expert or pool slot).  Coordinates past an extent read zeros.
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
-                                            int z) {
+                                            int z, uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
-        ::"r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+        ::"r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(pol)
         : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -502,6 +519,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     if (warp == 0) {
         // ------------------------------------- A producer: weights or raw codes
         if (lane == 0) {
+            const uint64_t pol = l2_policy_first();
             int stage = 0;
             uint32_t phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
@@ -523,8 +541,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                         if (!mbar_wait(&r_empty[stage], phase ^ 1, &s_abort)) { ok = false; break; }
                         mbar_arrive_expect_tx(&r_full[stage], (uint32_t)RAW);
                         uint8_t *dst = sRaw + stage * RAW;
-                        tma_load_3d(dst, ma, &r_full[stage], rs * kRawRowBytes, ya0, za);
-                        tma_load_3d(dst + 64 * kRawRowBytes, ma, &r_full[stage], rs * kRawRowBytes, ya1, za);
+                        tma_load_3d(dst, ma, &r_full[stage], rs * kRawRowBytes, ya0, za, pol);
+                        tma_load_3d(dst + 64 * kRawRowBytes, ma, &r_full[stage], rs * kRawRowBytes, ya1, za, pol);
                         if (++stage == SR) { stage = 0; phase ^= 1; }
                     }
                 } else {
@@ -534,9 +552,9 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                         mbar_arrive_expect_tx(&a_full[stage], (uint32_t)na * kATileBytes);
                         for (int a = 0; a < na; ++a) {
                             uint8_t *dst = sA + (stage * ATOMS + a) * kATileBytes;
-                            tma_load_3d(dst, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya0, za);
+                            tma_load_3d(dst, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya0, za, pol);
                             tma_load_3d(dst + kATileBytes / 2, ma, &a_full[stage], (kk * ATOMS + a) * kBlockK, ya1,
-                                        za);
+                                        za, pol);
                         }
                         if (++stage == SA) { stage = 0; phase ^= 1; }
                     }
@@ -551,6 +569,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             // input the previous launch writes: wait for it here, while the
             // other roles already stream weights
             pdl_wait();
+            const uint64_t pol = l2_policy_last();
             int stage = 0;
             uint32_t phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
@@ -569,7 +588,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                     for (int a = 0; a < na; ++a)
                         for (int j = 0; j < rows_ld; j += big ? 64 : 16)
                             tma_load_2d(db + a * b_atom_bytes + j * 128, big ? &map_b64 : &map_b, &b_full[stage],
-                                        (kk * ATOMS + a) * kBlockK, it.row0 + j);
+                                        (kk * ATOMS + a) * kBlockK, it.row0 + j, pol);
                     if (++stage == b_slots) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;

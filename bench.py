@@ -266,8 +266,8 @@ class Runner:
         li = i % len(self.layers)
         L = self.layers[li]
         _, _, lg, x = self.batches[i % len(self.batches)]
-        moe.moe_route_topk(lg, self.k, self.ids, self.w)
-        counts, offsets, sr, rp = moe.moe_permute(self.ids, L.E, hits=self.hits[li], out=self.perm)
+        _, _, counts, offsets, sr, rp = moe.moe_route_permute(lg, self.k, hits=self.hits[li], ids_w=(self.ids, self.w),
+                                                              out=self.perm)
         if ffn_events is not None:
             self._mark(ffn_events[0])
         moe.moe_grouped_ffn(L, x, self.k, counts, offsets, sr, rows=self.rows, ws=self.ws, path=self.path)
@@ -292,11 +292,9 @@ class Runner:
             self.torch.cuda.current_stream().wait_stream(self.side)
 
     def launches_per_step(self):
-        """route, permute, FFN (2 GEMV launches, or gather + 2 tensor-core launches), combine"""
-        R = self.T * self.k
-        auto_tc = R >= TC_MIN_ROUTES[self.layers[0].fmt]
-        tc = self.path == self.moe.MOE_FFN_TC or (self.path == self.moe.MOE_FFN_AUTO and auto_tc)
-        return 3 + (3 if tc else 2)
+        """route + permute (one launch up to FUSED_MAX_R routes, else two), FFN (2 GEMV
+        launches, or gather + 2 tensor-core launches), combine"""
+        return launches_per_layer(self.moe, self.T * self.k, self.layers[0].fmt, self.path)
 
     def distinct_experts(self):
         """Distinct routed experts of each batch (read back from our own routing)."""
@@ -309,6 +307,15 @@ class Runner:
 
 
 FFN_SAMPLE_EVERY = 1
+
+# routes up to which moe_route_permute is one launch
+FUSED_MAX_R = 256
+
+
+def launches_per_layer(moe, R, fmt, path):
+    auto_tc = R >= TC_MIN_ROUTES[fmt]
+    tc = path == moe.MOE_FFN_TC or (path == moe.MOE_FFN_AUTO and auto_tc)
+    return (1 if R <= FUSED_MAX_R else 2) + (3 if tc else 2) + 1
 
 
 def _capture(torch, runner, first, n):
@@ -486,6 +493,8 @@ def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
     perm = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
             torch.empty(T * k, dtype=torch.int32, device=dev), torch.empty(T * k, dtype=torch.int32, device=dev))
     moe.moe_permute(ids, E, out=perm)
+    perm1 = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
+             torch.empty(k, dtype=torch.int32, device=dev), torch.empty(k, dtype=torch.int32, device=dev))
     rows = torch.randn((T * k, H), generator=g, device=dev, dtype=torch.float32)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     hits = torch.zeros(E, dtype=torch.int32, device=dev)
@@ -509,6 +518,8 @@ def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
         ("route_topk", lambda: moe.moe_route_topk(lg, k, ids=ids, w=w), T * E * 4 + R * 8),
         ("route_min_weight (0.6)", lambda: moe.moe_route_min_weight(ids2, w2, E, 0.6, slot_table=table), R * 16 + E * 4),
         ("permute + hits", lambda: moe.moe_permute(ids, E, hits=hits, out=perm), R * 4 + R * 8 + E * 12),
+        ("route_permute (T=1, one launch)", lambda: moe.moe_route_permute(lg[:1], k, hits=hits, ids_w=(ids[:1], w[:1]),
+                                                                          out=perm1), E * 4 + k * 8 + k * 16 + E * 12),
         ("combine", lambda: moe.moe_combine(rows, perm[3], w, y), R * H * 4 + R * 8 + T * H * 2),
         ("quantize_int8 (one w13)", lambda: moe.moe_quantize_int8(wq, q8, s8), 2 * I * H * 3 + 2 * I * 4),
         ("quantize_int4 (one w13)", lambda: moe.moe_quantize_int4(wq, q4, s4), 2 * I * H * 2 + I * H + 2 * I * (H // 64) * 2),
@@ -1010,8 +1021,7 @@ def stack_steps(torch, moe, stack, T, k, steps, warmup, seed, refresh_every=8, p
         x = x_stage[j]
         for l in range(L):
             lay = stack.layers[l]
-            moe.moe_route_topk(lg_stage[j, l], k, ids, w)
-            moe.moe_permute(ids, E, hits=hits[l] if with_hits else None, out=perm)
+            moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if with_hits else None, ids_w=(ids, w), out=perm)
             moe.moe_grouped_ffn(lay, x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
             y = ybuf[l & 1]
             moe.moe_combine(rows, perm[3], w, y)
@@ -1110,8 +1120,7 @@ def stack_steps_device(torch, moe, stack, T, k, steps, warmup, seed, refresh_eve
     side = torch.cuda.Stream(dev)
 
     def layer(j, l, x):
-        moe.moe_route_topk(lg_stage[j, l], k, ids, w)
-        moe.moe_permute(ids, E, hits=hits[l] if j == 0 else None, out=perm)
+        moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if j == 0 else None, ids_w=(ids, w), out=perm)
         moe.moe_grouped_ffn(stack.layers[l], x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
         y = ybuf[l & 1]
         moe.moe_combine(rows, perm[3], w, y)
@@ -1233,9 +1242,7 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
                       "routes_on_resident_slots": round(sum(share) / len(share), 4) if share else None},
         "sweep": sweep,
         "hbm_peak_gbs": hbm_peak,
-        "gpu_launches": steps_done * L * (3 + (3 if (path == moe.MOE_FFN_TC or
-                                                      (path == moe.MOE_FFN_AUTO and T * k >= TC_MIN_ROUTES[s4.fmt]))
-                                                     else 2))
+        "gpu_launches": steps_done * L * launches_per_layer(moe, T * k, s4.fmt, path)
                         + (steps_done // 8) * L * (2 if device_refresh else 0),
         "clocks": clk,
     }

@@ -186,6 +186,18 @@ MOE_API moe_status moe_permute(const int32_t *ids, int32_t T, int32_t k, int32_t
                        int32_t *offsets, int32_t *sorted_route, int32_t *route_pos, uint32_t *hits,
                        moe_stream_t stream);
 
+/*
+ * moe_route_topk followed by moe_permute, with the same arguments and the
+ * same results bit for bit (ids, w, counts, offsets, sorted_route, route_pos,
+ * hits), in one launch when T*k <= 256: one CTA routes the batch's tokens into
+ * shared memory and groups the routes there (a one-token decode step then
+ * launches one kernel before the FFN instead of two).  Larger batches run the
+ * two kernels.  T == 0 behaves as moe_permute's empty grouping.
+ */
+MOE_API moe_status moe_route_permute(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *ids, float *w,
+                                     int32_t *counts, int32_t *offsets, int32_t *sorted_route, int32_t *route_pos,
+                                     uint32_t *hits, moe_stream_t stream);
+
 /* hits[e] += number of the n ids equal to e; ids outside [0,E) are ignored
  * (expert_pool.rs, count_hits). */
 MOE_API moe_status moe_expert_hits(const int32_t *ids, int64_t n, int32_t E, uint32_t *hits, moe_stream_t stream);

@@ -20,6 +20,9 @@ cudaError_t launch_route_min_weight(int32_t *, float *, const int32_t *, int, in
 cudaError_t launch_permute(const int32_t *, int, int, int32_t *, int32_t *, int32_t *, int32_t *, uint32_t *,
                            cudaStream_t);
 cudaError_t launch_expert_hits(const int32_t *, int64_t, int, uint32_t *, cudaStream_t);
+bool route_permute_fused(int T, int k);
+cudaError_t launch_route_permute(const float *, int, int, int, int32_t *, float *, int32_t *, int32_t *, int32_t *,
+                                 int32_t *, uint32_t *, cudaStream_t);
 cudaError_t launch_combine(const float *, const int32_t *, const float *, int, int, int, uint16_t *, cudaStream_t);
 cudaError_t launch_quantize_int8(const uint16_t *, int, int, int8_t *, float *, cudaStream_t);
 cudaError_t launch_quantize_int4(const uint16_t *, int, int, uint8_t *, uint16_t *, cudaStream_t);
@@ -195,6 +198,25 @@ moe_status moe_permute(const int32_t *ids, int32_t T, int32_t k, int32_t E, int3
                        "moe_permute launch");
 }
 
+moe_status moe_route_permute(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *ids, float *w,
+                             int32_t *counts, int32_t *offsets, int32_t *sorted_route, int32_t *route_pos,
+                             uint32_t *hits, moe_stream_t stream) {
+    moe_status st = check_shape(E, k, 64, 64);
+    if (st != MOE_OK) return st;
+    if ((st = check_tk(T, k)) != MOE_OK) return st;
+    if (T == 0) return moe_permute(nullptr, 0, k, E, counts, offsets, sorted_route, route_pos, hits, stream);
+    CHECK_ARG(logits && ids && w && counts && offsets && sorted_route && route_pos, "moe_route_permute: NULL pointer");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (route_permute_fused(T, k))
+        return cuda_status(launch_route_permute(logits, T, E, k, ids, w, counts, offsets, sorted_route, route_pos,
+                                                hits, s),
+                           "moe_route_permute launch");
+    if ((st = cuda_status(launch_route_topk(logits, T, E, k, ids, w, s), "moe_route_permute: route")) != MOE_OK)
+        return st;
+    return cuda_status(launch_permute(ids, T * k, E, counts, offsets, sorted_route, route_pos, hits, s),
+                       "moe_route_permute: permute");
+}
+
 moe_status moe_expert_hits(const int32_t *ids, int64_t n, int32_t E, uint32_t *hits, moe_stream_t stream) {
     CHECK_ARG(E >= 1 && E <= kMaxE, "E=%d outside [1, %d]", E, kMaxE);
     CHECK_ARG(n >= 0, "n=%lld is negative", (long long)n);
@@ -312,8 +334,8 @@ moe_status moe_layer_forward(const moe_layer *layer, const float *logits, const 
     int32_t *sorted = reinterpret_cast<int32_t *>(base + f.sorted);
     int32_t *pos = reinterpret_cast<int32_t *>(base + f.pos);
     float *rows = reinterpret_cast<float *>(base + f.rows);
-    if ((st = moe_route_topk(logits, T, v.E, k, ids, w, stream)) != MOE_OK) return st;
-    if ((st = moe_permute(ids, T, k, v.E, counts, offsets, sorted, pos, hits, stream)) != MOE_OK) return st;
+    if ((st = moe_route_permute(logits, T, v.E, k, ids, w, counts, offsets, sorted, pos, hits, stream)) != MOE_OK)
+        return st;
     if ((st = moe_grouped_ffn(layer, x, T, k, counts, offsets, sorted, rows, base + f.ffn, ws_bytes - f.ffn, stream)) !=
         MOE_OK)
         return st;

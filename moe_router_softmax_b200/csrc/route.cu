@@ -153,6 +153,109 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
     route_token_warp<VPL>([l](int e) { return __ldg(l + e); }, E, k, ids + (size_t)t * k, w + (size_t)t * k);
 }
 
+// ------------------------------------- routing and grouping in one launch
+// For a small batch (R = T*k <= kFusedMaxR) the top-k above and the stable
+// grouping of moe_permute in one CTA: warp w routes tokens w, w + 16, ... into
+// shared memory; the routes are counted per expert (shared-memory atomics: a
+// count does not depend on the order of its increments), an exclusive scan over
+// the experts gives each group's base, and route r lands at its expert's base
+// plus the number of routes r' < r of the same expert, i.e. ascending r inside
+// a group.  The outputs are those of moe_route_topk followed by moe_permute, bit
+// for bit, from one launch instead of two.
+constexpr int kFusedMaxR = 256;
+constexpr int kFusedThreads = 512;
+
+template <int VPL>
+__global__ void __launch_bounds__(kFusedThreads) k_route_permute(const float *__restrict__ logits, int T, int E, int k,
+                                                                 int32_t *__restrict__ ids, float *__restrict__ w,
+                                                                 int32_t *__restrict__ counts,
+                                                                 int32_t *__restrict__ offsets,
+                                                                 int32_t *__restrict__ sorted_route,
+                                                                 int32_t *__restrict__ route_pos,
+                                                                 uint32_t *__restrict__ hits) {
+    constexpr int NW = kFusedThreads / 32, PER = kMaxE / kFusedThreads;
+    __shared__ int32_t s_ids[kFusedMaxR];
+    __shared__ float s_w[kFusedMaxR];
+    __shared__ int s_cnt[kMaxE];
+    __shared__ int s_base[kMaxE];
+    __shared__ int s_warp[NW];
+    __shared__ int s_total;
+    // programmatic dependent launch: wait for the logits, then let the next
+    // kernel be scheduled
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int R = T * k;
+    for (int t = warp; t < T; t += NW) {
+        const float *l = logits + (size_t)t * E;
+        route_token_warp<VPL>([l](int e) { return __ldg(l + e); }, E, k, s_ids + t * k, s_w + t * k);
+    }
+    for (int e = tid; e < E; e += kFusedThreads) s_cnt[e] = 0;
+    __syncthreads();
+    for (int r = tid; r < R; r += kFusedThreads) {
+        const int e = s_ids[r];
+        ids[r] = e;
+        w[r] = s_w[r];
+        if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
+    }
+    __syncthreads();
+    // exclusive scan of the counts; thread tid holds experts PER*tid .. PER*tid + PER-1
+    int loc[PER], sum = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = tid * PER + i;
+        loc[i] = e < E ? s_cnt[e] : 0;
+        sum += loc[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < NW ? s_warp[lane] : 0;
+        int x = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += u;
+        }
+        if (lane < NW) s_warp[lane] = x - v;
+        if (lane == 31) s_total = x;
+    }
+    __syncthreads();
+    int run = s_warp[warp] + incl - sum;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = tid * PER + i;
+        if (e < E) {
+            s_base[e] = run;
+            counts[e] = loc[i];
+            offsets[e] = run;
+            if (hits) hits[e] += (uint32_t)loc[i];
+        }
+        run += loc[i];
+    }
+    if (tid == 0) offsets[E] = s_total;
+    __syncthreads();
+    for (int r = tid; r < R; r += kFusedThreads) {
+        const int e = s_ids[r];
+        if (e >= 0 && e < E) {
+            int rank = 0;
+            for (int q = 0; q < r; ++q) rank += s_ids[q] == e;
+            const int pos = s_base[e] + rank;
+            sorted_route[pos] = r;
+            route_pos[r] = pos;
+        } else {
+            route_pos[r] = -1;
+        }
+    }
+    for (int i = s_total + tid; i < R; i += kFusedThreads) sorted_route[i] = -1;
+}
+
 // ------------------------------------------------ router projection + top-k
 // The step before the routing: logits[t][e] = sum_h x[t][h] * w_router[e][h]
 // (x bf16, router weights fp32, fp32 fused multiply-adds), then the top-k
@@ -384,6 +487,25 @@ cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t 
     if (vpl <= 8) return launch_pdl(k_route_topk<8>, grid, block, 0, s, logits, T, E, k, ids, w);
     if (vpl <= 16) return launch_pdl(k_route_topk<16>, grid, block, 0, s, logits, T, E, k, ids, w);
     return launch_pdl(k_route_topk<32>, grid, block, 0, s, logits, T, E, k, ids, w);
+}
+
+bool route_permute_fused(int T, int k) { return (int64_t)T * k <= kFusedMaxR; }
+
+cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32_t *ids, float *w,
+                                 int32_t *counts, int32_t *offsets, int32_t *sorted_route, int32_t *route_pos,
+                                 uint32_t *hits, cudaStream_t s) {
+    const int vpl = (E + 31) / 32;
+    dim3 block(kFusedThreads), grid(1);
+    auto go = [&](auto kern) {
+        return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, ids, w, counts, offsets, sorted_route, route_pos,
+                          hits);
+    };
+    if (vpl <= 1) return go(k_route_permute<1>);
+    if (vpl <= 2) return go(k_route_permute<2>);
+    if (vpl <= 4) return go(k_route_permute<4>);
+    if (vpl <= 8) return go(k_route_permute<8>);
+    if (vpl <= 16) return go(k_route_permute<16>);
+    return go(k_route_permute<32>);
 }
 
 }  // namespace moe

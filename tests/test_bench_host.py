@@ -43,3 +43,18 @@ def test_traffic_entries_name_their_capture():
         # decode traffic is within a few percent of the algorithmic bytes; prefill
         # adds its fp32 rows and activation re-reads
         assert 1.0 <= val[0] / val[1] <= (1.4 if "prefill" in key[0] else 1.05)
+
+
+class _FakeMoe:
+    MOE_FFN_AUTO, MOE_FFN_GEMV, MOE_FFN_TC = 0, 1, 2
+
+
+def test_launch_count_per_layer_step():
+    m = _FakeMoe()
+    # one token: fused route + permute, two GEMV launches, combine
+    assert bench.launches_per_layer(m, 8, 0, m.MOE_FFN_AUTO) == 1 + 2 + 1
+    # 64 tokens: route and permute apart, gather + two tensor-core launches, combine
+    assert bench.launches_per_layer(m, 512, 0, m.MOE_FFN_AUTO) == 2 + 3 + 1
+    # the boundary of the one-launch routing, and a forced path
+    assert bench.launches_per_layer(m, bench.FUSED_MAX_R, 2, m.MOE_FFN_GEMV) == 1 + 2 + 1
+    assert bench.launches_per_layer(m, bench.FUSED_MAX_R + 1, 2, m.MOE_FFN_TC) == 2 + 3 + 1

@@ -76,6 +76,52 @@ def test_permute_and_hits_bit_exact(T, k, E):
     assert np.array_equal(hits.cpu().numpy().view(np.uint32), oracle.hits(ids, E, hits0))
 
 
+# moe_route_permute: one launch for T*k <= 256 (the first six cases, including
+# the boundary R = 256 and E = 1024), the two kernels beyond it (the last two)
+@pytest.mark.parametrize("T,E,k,kind", [(1, 128, 8, "normal"), (8, 128, 8, "biased"), (32, 128, 8, "normal"),
+                                        (1, 1024, 32, "normal"), (3, 11, 5, "normal"), (64, 8, 4, "biased"),
+                                        (33, 128, 8, "normal"), (1024, 128, 8, "biased")])
+def test_route_permute_matches_the_oracle_and_the_two_calls(T, E, k, kind):
+    lg = syn.router_logits(T, E, kind, seed=7 * T + E)
+    rng = np.random.default_rng(T + k)
+    hits0 = rng.integers(0, 50, size=E).astype(np.uint32)
+    h_one = torch.from_numpy(hits0.view(np.int32)).to(DEV)
+    h_two = torch.from_numpy(hits0.view(np.int32)).to(DEV)
+    d_lg = torch.from_numpy(lg).to(DEV)
+    one = moe.moe_route_permute(d_lg, k, hits=h_one)
+    ids, w = moe.moe_route_topk(d_lg, k)
+    two = (ids, w) + tuple(moe.moe_permute(ids, E, hits=h_two))
+    for a, b in zip(one, two):
+        assert np.array_equal(a.cpu().numpy().view(np.uint32), b.cpu().numpy().view(np.uint32))
+    assert np.array_equal(h_one.cpu().numpy(), h_two.cpu().numpy())
+    oi, ow = oracle.route_topk(lg, k)
+    assert np.array_equal(one[0].cpu().numpy(), oi)
+    assert bits_equal(one[1].cpu().numpy(), ow)
+    for g, r in zip(one[2:], oracle.permute(oi, E)):
+        assert np.array_equal(g.cpu().numpy(), r)
+    assert np.array_equal(h_one.cpu().numpy().view(np.uint32), oracle.hits(oi, E, hits0))
+
+
+def test_route_permute_ties_nan_inf():
+    rng = np.random.default_rng(4)
+    lg = rng.integers(-2, 3, size=(30, 40)).astype(np.float32)
+    lg[0, :] = 0.0
+    lg[1, 5] = np.nan
+    lg[2, [1, 7]] = np.inf
+    lg[3, :] = -np.inf
+    lg[3, 9] = 1.0
+    lg[4, ::3] = -0.0
+    ids, w, counts, offsets, sr, rp = moe.moe_route_permute(torch.from_numpy(lg).to(DEV), 6)
+    oi, ow = oracle.route_topk(lg, 6)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    g = w.cpu().numpy()
+    assert np.array_equal(np.isnan(g), np.isnan(ow))
+    fin = ~np.isnan(ow)
+    assert bits_equal(np.where(fin, g, 0), np.where(fin, ow, 0))
+    for a, r in zip((counts, offsets, sr, rp), oracle.permute(oi, 40)):
+        assert np.array_equal(a.cpu().numpy(), r)
+
+
 @pytest.mark.parametrize("n,E", [(1, 4), (5, 4), (100000, 128), (33333, 1024)])
 def test_expert_hits_bit_exact(n, E):
     rng = np.random.default_rng(n)

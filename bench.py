@@ -292,9 +292,9 @@ class Runner:
             self.torch.cuda.current_stream().wait_stream(self.side)
 
     def launches_per_step(self):
-        """route + permute (one launch up to FUSED_MAX_R routes, else two), FFN (2 GEMV
+        """route + permute (one launch up to FUSED_MAX_T tokens, else two), FFN (2 GEMV
         launches, or gather + 2 tensor-core launches), combine"""
-        return launches_per_layer(self.moe, self.T * self.k, self.layers[0].fmt, self.path)
+        return launches_per_layer(self.moe, self.T, self.k, self.layers[0].fmt, self.path)
 
     def distinct_experts(self):
         """Distinct routed experts of each batch (read back from our own routing)."""
@@ -308,14 +308,14 @@ class Runner:
 
 FFN_SAMPLE_EVERY = 1
 
-# routes up to which moe_route_permute is one launch
-FUSED_MAX_R = 256
+# tokens up to which moe_route_permute is one launch
+FUSED_MAX_T = 16
 
 
-def launches_per_layer(moe, R, fmt, path):
-    auto_tc = R >= TC_MIN_ROUTES[fmt]
+def launches_per_layer(moe, T, k, fmt, path):
+    auto_tc = T * k >= TC_MIN_ROUTES[fmt]
     tc = path == moe.MOE_FFN_TC or (path == moe.MOE_FFN_AUTO and auto_tc)
-    return (1 if R <= FUSED_MAX_R else 2) + (3 if tc else 2) + 1
+    return (1 if T <= FUSED_MAX_T else 2) + (3 if tc else 2) + 1
 
 
 def _capture(torch, runner, first, n):
@@ -495,6 +495,8 @@ def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
     moe.moe_permute(ids, E, out=perm)
     perm1 = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
              torch.empty(k, dtype=torch.int32, device=dev), torch.empty(k, dtype=torch.int32, device=dev))
+    perm8 = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
+             torch.empty(8 * k, dtype=torch.int32, device=dev), torch.empty(8 * k, dtype=torch.int32, device=dev))
     rows = torch.randn((T * k, H), generator=g, device=dev, dtype=torch.float32)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     hits = torch.zeros(E, dtype=torch.int32, device=dev)
@@ -518,6 +520,9 @@ def time_kernels(torch, moe, layer, T, E, H, I, k, dev, n=100):
         ("route_topk", lambda: moe.moe_route_topk(lg, k, ids=ids, w=w), T * E * 4 + R * 8),
         ("route_min_weight (0.6)", lambda: moe.moe_route_min_weight(ids2, w2, E, 0.6, slot_table=table), R * 16 + E * 4),
         ("permute + hits", lambda: moe.moe_permute(ids, E, hits=hits, out=perm), R * 4 + R * 8 + E * 12),
+        ("route_permute (T=8, one launch)", lambda: moe.moe_route_permute(lg[:8], k, hits=hits,
+                                                                          ids_w=(ids[:8], w[:8]), out=perm8),
+         8 * E * 4 + 8 * k * 8 + 8 * k * 16 + E * 12),
         ("route_permute (T=1, one launch)", lambda: moe.moe_route_permute(lg[:1], k, hits=hits, ids_w=(ids[:1], w[:1]),
                                                                           out=perm1), E * 4 + k * 8 + k * 16 + E * 12),
         ("combine", lambda: moe.moe_combine(rows, perm[3], w, y), R * H * 4 + R * 8 + T * H * 2),
@@ -1242,7 +1247,7 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
                       "routes_on_resident_slots": round(sum(share) / len(share), 4) if share else None},
         "sweep": sweep,
         "hbm_peak_gbs": hbm_peak,
-        "gpu_launches": steps_done * L * launches_per_layer(moe, T * k, s4.fmt, path)
+        "gpu_launches": steps_done * L * launches_per_layer(moe, T, k, s4.fmt, path)
                         + (steps_done // 8) * L * (2 if device_refresh else 0),
         "clocks": clk,
     }

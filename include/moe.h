@@ -189,10 +189,11 @@ MOE_API moe_status moe_permute(const int32_t *ids, int32_t T, int32_t k, int32_t
 /*
  * moe_route_topk followed by moe_permute, with the same arguments and the
  * same results bit for bit (ids, w, counts, offsets, sorted_route, route_pos,
- * hits), in one launch when T*k <= 256: one CTA routes the batch's tokens into
- * shared memory and groups the routes there (a one-token decode step then
- * launches one kernel before the FFN instead of two).  Larger batches run the
- * two kernels.  T == 0 behaves as moe_permute's empty grouping.
+ * hits), in one launch when T <= 16: one CTA routes the batch's tokens (one
+ * warp each) into shared memory and groups the routes there (a small decode
+ * step then launches one kernel before the FFN instead of two; up to 64 KiB of
+ * shared memory).  Larger batches run the two kernels.  T == 0 behaves as moe_permute's empty
+ * grouping.
  */
 MOE_API moe_status moe_route_permute(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *ids, float *w,
                                      int32_t *counts, int32_t *offsets, int32_t *sorted_route, int32_t *route_pos,

@@ -154,16 +154,20 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
 }
 
 // ------------------------------------- routing and grouping in one launch
-// For a small batch (R = T*k <= kFusedMaxR) the top-k above and the stable
-// grouping of moe_permute in one CTA: warp w routes tokens w, w + 16, ... into
-// shared memory; the routes are counted per expert (shared-memory atomics: a
-// count does not depend on the order of its increments), an exclusive scan over
-// the experts gives each group's base, and route r lands at its expert's base
-// plus the number of routes r' < r of the same expert, i.e. ascending r inside
-// a group.  The outputs are those of moe_route_topk followed by moe_permute, bit
-// for bit, from one launch instead of two.
-constexpr int kFusedMaxR = 256;
+// For a decode batch (T <= 16 tokens, one per warp; R = T*k <= kFusedMaxR) the
+// top-k above and the stable grouping of moe_permute in one CTA of 16 warps.
+// Warp w routes token w into shared memory (a token's top-k is a chain of k
+// warp reductions, so one CTA routing more tokens than it has warps would be
+// slower than the many-CTA routing kernel); then the grouping takes moe_permute's steps
+// over the routes held there: warp w owns a contiguous segment of routes and
+// counts them per expert with __match_any_sync (no atomics), a scan in (expert,
+// warp) order gives every warp its base row per expert, and a second walk of
+// the segment places each route at that base plus its rank among the equal ids
+// before it.  The outputs are those of moe_route_topk followed by moe_permute,
+// bit for bit, from one launch instead of two.
+constexpr int kFusedMaxR = 1024;
 constexpr int kFusedThreads = 512;
+constexpr int kFusedWarps = kFusedThreads / 32;
 
 template <int VPL>
 __global__ void __launch_bounds__(kFusedThreads) k_route_permute(const float *__restrict__ logits, int T, int E, int k,
@@ -173,11 +177,10 @@ __global__ void __launch_bounds__(kFusedThreads) k_route_permute(const float *__
                                                                  int32_t *__restrict__ sorted_route,
                                                                  int32_t *__restrict__ route_pos,
                                                                  uint32_t *__restrict__ hits) {
-    constexpr int NW = kFusedThreads / 32, PER = kMaxE / kFusedThreads;
+    constexpr int NW = kFusedWarps, PER = kMaxE / kFusedThreads;
+    extern __shared__ int s_cw[];  // [NW][E] per-warp counts, then bases
     __shared__ int32_t s_ids[kFusedMaxR];
-    __shared__ float s_w[kFusedMaxR];
-    __shared__ int s_cnt[kMaxE];
-    __shared__ int s_base[kMaxE];
+    __shared__ float s_wt[kFusedMaxR];
     __shared__ int s_warp[NW];
     __shared__ int s_total;
     // programmatic dependent launch: wait for the logits, then let the next
@@ -188,24 +191,37 @@ __global__ void __launch_bounds__(kFusedThreads) k_route_permute(const float *__
     const int R = T * k;
     for (int t = warp; t < T; t += NW) {
         const float *l = logits + (size_t)t * E;
-        route_token_warp<VPL>([l](int e) { return __ldg(l + e); }, E, k, s_ids + t * k, s_w + t * k);
+        route_token_warp<VPL>([l](int e) { return __ldg(l + e); }, E, k, s_ids + t * k, s_wt + t * k);
     }
-    for (int e = tid; e < E; e += kFusedThreads) s_cnt[e] = 0;
+    for (int i = tid; i < NW * E; i += kFusedThreads) s_cw[i] = 0;
     __syncthreads();
     for (int r = tid; r < R; r += kFusedThreads) {
-        const int e = s_ids[r];
-        ids[r] = e;
-        w[r] = s_w[r];
-        if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
+        ids[r] = s_ids[r];
+        w[r] = s_wt[r];
+    }
+    const int seg = (R + NW - 1) / NW;
+    const int r_begin = warp * seg, r_end = min(R, r_begin + seg);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    // pass 1: per-warp counts
+    for (int base = r_begin; base < r_end; base += 32) {
+        const int r = base + lane;
+        int e = r < r_end ? s_ids[r] : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (peers & lt_mask) == 0) s_cw[warp * E + e] += __popc(peers);
     }
     __syncthreads();
-    // exclusive scan of the counts; thread tid holds experts PER*tid .. PER*tid + PER-1
+    // totals per expert and their exclusive scan; thread tid holds experts
+    // PER*tid .. PER*tid + PER-1
     int loc[PER], sum = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
         const int e = tid * PER + i;
-        loc[i] = e < E ? s_cnt[e] : 0;
-        sum += loc[i];
+        int c = 0;
+        if (e < E)
+            for (int v = 0; v < NW; ++v) c += s_cw[v * E + e];
+        loc[i] = c;
+        sum += c;
     }
     int incl = sum;
 #pragma unroll
@@ -232,26 +248,38 @@ __global__ void __launch_bounds__(kFusedThreads) k_route_permute(const float *__
     for (int i = 0; i < PER; ++i) {
         const int e = tid * PER + i;
         if (e < E) {
-            s_base[e] = run;
             counts[e] = loc[i];
             offsets[e] = run;
             if (hits) hits[e] += (uint32_t)loc[i];
+            int b = run;
+            for (int v = 0; v < NW; ++v) {  // per-warp bases, in warp (= route) order
+                const int c = s_cw[v * E + e];
+                s_cw[v * E + e] = b;
+                b += c;
+            }
         }
         run += loc[i];
     }
     if (tid == 0) offsets[E] = s_total;
     __syncthreads();
-    for (int r = tid; r < R; r += kFusedThreads) {
-        const int e = s_ids[r];
-        if (e >= 0 && e < E) {
-            int rank = 0;
-            for (int q = 0; q < r; ++q) rank += s_ids[q] == e;
-            const int pos = s_base[e] + rank;
-            sorted_route[pos] = r;
-            route_pos[r] = pos;
-        } else {
-            route_pos[r] = -1;
+    // pass 2: stable placement
+    for (int base = r_begin; base < r_end; base += 32) {
+        const int r = base + lane;
+        int e = r < r_end ? s_ids[r] : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (r < r_end) {
+            if (e >= 0) {
+                const int pos = s_cw[warp * E + e] + __popc(peers & lt_mask);
+                sorted_route[pos] = r;
+                route_pos[r] = pos;
+            } else {
+                route_pos[r] = -1;
+            }
         }
+        __syncwarp();
+        if (e >= 0 && (peers & lt_mask) == 0) s_cw[warp * E + e] += __popc(peers);
+        __syncwarp();
     }
     for (int i = s_total + tid; i < R; i += kFusedThreads) sorted_route[i] = -1;
 }
@@ -489,16 +517,28 @@ cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t 
     return launch_pdl(k_route_topk<32>, grid, block, 0, s, logits, T, E, k, ids, w);
 }
 
-bool route_permute_fused(int T, int k) { return (int64_t)T * k <= kFusedMaxR; }
+bool route_permute_fused(int T, int k) { return T <= kFusedWarps && T * k <= kFusedMaxR; }
 
 cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32_t *ids, float *w,
                                  int32_t *counts, int32_t *offsets, int32_t *sorted_route, int32_t *route_pos,
                                  uint32_t *hits, cudaStream_t s) {
     const int vpl = (E + 31) / 32;
+    const size_t smem = (size_t)kFusedWarps * E * sizeof(int);  // <= 64 KiB (E <= 1024)
     dim3 block(kFusedThreads), grid(1);
     auto go = [&](auto kern) {
-        return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, ids, w, counts, offsets, sorted_route, route_pos,
-                          hits);
+        // one-time attribute per device and instantiation (kept out of stream capture)
+        static size_t cached[kMaxDevices] = {};
+        int dev = 0;
+        cudaError_t err = cudaGetDevice(&dev);
+        if (err != cudaSuccess) return err;
+        if (dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (cached[dev] < smem) {
+            err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (err != cudaSuccess) return err;
+            cached[dev] = smem;
+        }
+        return launch_pdl(kern, grid, block, smem, s, logits, T, E, k, ids, w, counts, offsets, sorted_route,
+                          route_pos, hits);
     };
     if (vpl <= 1) return go(k_route_permute<1>);
     if (vpl <= 2) return go(k_route_permute<2>);

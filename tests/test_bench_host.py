@@ -52,9 +52,11 @@ class _FakeMoe:
 def test_launch_count_per_layer_step():
     m = _FakeMoe()
     # one token: fused route + permute, two GEMV launches, combine
-    assert bench.launches_per_layer(m, 8, 0, m.MOE_FFN_AUTO) == 1 + 2 + 1
-    # 64 tokens: route and permute apart, gather + two tensor-core launches, combine
-    assert bench.launches_per_layer(m, 512, 0, m.MOE_FFN_AUTO) == 2 + 3 + 1
-    # the boundary of the one-launch routing, and a forced path
-    assert bench.launches_per_layer(m, bench.FUSED_MAX_R, 2, m.MOE_FFN_GEMV) == 1 + 2 + 1
-    assert bench.launches_per_layer(m, bench.FUSED_MAX_R + 1, 2, m.MOE_FFN_TC) == 2 + 3 + 1
+    assert bench.launches_per_layer(m, 1, 8, 0, m.MOE_FFN_AUTO) == 1 + 2 + 1
+    # 8 tokens: fused route + permute, gather + two tensor-core launches, combine
+    assert bench.launches_per_layer(m, 8, 8, 0, m.MOE_FFN_AUTO) == 1 + 3 + 1
+    # 64 tokens: route and permute apart
+    assert bench.launches_per_layer(m, 64, 8, 0, m.MOE_FFN_AUTO) == 2 + 3 + 1
+    # the boundary of the one-launch routing, and forced paths
+    assert bench.launches_per_layer(m, bench.FUSED_MAX_T, 8, 2, m.MOE_FFN_GEMV) == 1 + 2 + 1
+    assert bench.launches_per_layer(m, bench.FUSED_MAX_T + 1, 1, 2, m.MOE_FFN_TC) == 2 + 3 + 1

@@ -76,11 +76,12 @@ def test_permute_and_hits_bit_exact(T, k, E):
     assert np.array_equal(hits.cpu().numpy().view(np.uint32), oracle.hits(ids, E, hits0))
 
 
-# moe_route_permute: one launch for T*k <= 256 (the first six cases, including
-# the boundary R = 256 and E = 1024), the two kernels beyond it (the last two)
-@pytest.mark.parametrize("T,E,k,kind", [(1, 128, 8, "normal"), (8, 128, 8, "biased"), (32, 128, 8, "normal"),
-                                        (1, 1024, 32, "normal"), (3, 11, 5, "normal"), (64, 8, 4, "biased"),
-                                        (33, 128, 8, "normal"), (1024, 128, 8, "biased")])
+# moe_route_permute: one launch for T <= 16 (the first seven cases, including
+# the boundary T = 16, E = 1024 and T*k = 512), the two kernels beyond it
+@pytest.mark.parametrize("T,E,k,kind", [(1, 128, 8, "normal"), (8, 128, 8, "biased"), (16, 128, 8, "normal"),
+                                        (1, 1024, 32, "normal"), (3, 11, 5, "normal"), (16, 8, 4, "biased"),
+                                        (16, 1024, 32, "normal"), (17, 128, 8, "normal"), (64, 128, 8, "biased"),
+                                        (1024, 128, 8, "biased")])
 def test_route_permute_matches_the_oracle_and_the_two_calls(T, E, k, kind):
     lg = syn.router_logits(T, E, kind, seed=7 * T + E)
     rng = np.random.default_rng(T + k)

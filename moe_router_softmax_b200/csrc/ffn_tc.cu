@@ -883,19 +883,24 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                             }
                         }
                     } else {
+                        // a code c (two's complement) as bf16, exactly: 0x43 over the low
+                        // seven bits is 128 + (c & 127); minus 128 (0x4300) when c >= 0,
+                        // minus 256 (0x4380, the sign bit as the low byte) when c < 0.
+                        // Two masks per word, then per pair of codes two byte permutes and
+                        // one subtraction, in the codes' order (the same selectors as int4).
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {  // 16 codes per chunk -> 8 bf16 pairs (codes exact in bf16)
                             const uint4 u = *reinterpret_cast<const uint4 *>(src + (((cj0 + c) ^ (r & 7)) << 4));
-                            const uint32_t words[4] = {u.x ^ 0x80808080u, u.y ^ 0x80808080u, u.z ^ 0x80808080u,
-                                                       u.w ^ 0x80808080u};
+                            const uint32_t words[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
+                                const uint32_t lo = words[i] & 0x7F7F7F7Fu, sg = words[i] & 0x80808080u;
 #pragma unroll
                                 for (int j = 0; j < 2; ++j) {
-                                    const uint32_t sel0 = 0x7540u | (uint32_t)(2 * j), sel1 = sel0 + 1;
-                                    const float f0 = __uint_as_float(__byte_perm(words[i], 0x4B000000u, sel0)) - 8388736.0f;
-                                    const float f1 = __uint_as_float(__byte_perm(words[i], 0x4B000000u, sel1)) - 8388736.0f;
-                                    __nv_bfloat162 q = __floats2bfloat162_rn(f0, f1);
+                                    const uint32_t sel = j ? 0x4342u : 0x4140u;
+                                    uint32_t v = __byte_perm(lo, 0x43434343u, sel), b = __byte_perm(sg, 0x43434343u, sel);
+                                    __nv_bfloat162 q = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&v),
+                                                               *reinterpret_cast<__nv_bfloat162 *>(&b));
                                     o[8 * c + 2 * i + j] = *reinterpret_cast<uint32_t *>(&q);
                                 }
                             }

@@ -154,20 +154,20 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
 }
 
 // ------------------------------------- routing and grouping in one launch
-// For a decode batch (T <= 16 tokens, one per warp; R = T*k <= kFusedMaxR) the
-// top-k above and the stable grouping of moe_permute in one CTA of 16 warps.
-// Warp w routes token w into shared memory (a token's top-k is a chain of k
-// warp reductions, so one CTA routing more tokens than it has warps would be
-// slower than the many-CTA routing kernel); then the grouping takes moe_permute's steps
-// over the routes held there: warp w owns a contiguous segment of routes and
-// counts them per expert with __match_any_sync (no atomics), a scan in (expert,
-// warp) order gives every warp its base row per expert, and a second walk of
-// the segment places each route at that base plus its rank among the equal ids
-// before it.  The outputs are those of moe_route_topk followed by moe_permute,
-// bit for bit, from one launch instead of two.
-constexpr int kFusedMaxR = 1024;
+// For a decode batch of T <= 16 tokens the top-k above and the stable grouping
+// of moe_permute in one CTA of 16 warps.  Warp w routes token w into shared
+// memory (a token's top-k is a chain of k warp reductions, so one CTA routing
+// more tokens than it has warps would be slower than the many-CTA routing
+// kernel); then the grouping takes moe_permute's steps over the routes held
+// there: warp w owns a contiguous segment of routes and counts them per expert
+// with __match_any_sync (no atomics), a scan in (expert, warp) order gives every
+// warp its base row per expert, and a second walk of the segment places each
+// route at that base plus its rank among the equal ids before it.  The outputs
+// are those of moe_route_topk followed by moe_permute, bit for bit, from one
+// launch instead of two.
 constexpr int kFusedThreads = 512;
 constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kFusedMaxR = kFusedWarps * kMaxK;  // routes of 16 tokens at k <= 32
 
 template <int VPL>
 __global__ void __launch_bounds__(kFusedThreads) k_route_permute(const float *__restrict__ logits, int T, int E, int k,
@@ -517,7 +517,7 @@ cudaError_t launch_route_topk(const float *logits, int T, int E, int k, int32_t 
     return launch_pdl(k_route_topk<32>, grid, block, 0, s, logits, T, E, k, ids, w);
 }
 
-bool route_permute_fused(int T, int k) { return T <= kFusedWarps && T * k <= kFusedMaxR; }
+bool route_permute_fused(int T, int k) { return T <= kFusedWarps && k <= kMaxK; }
 
 cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32_t *ids, float *w,
                                  int32_t *counts, int32_t *offsets, int32_t *sorted_route, int32_t *route_pos,

@@ -330,6 +330,8 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(NT)
 
     // this CTA's slice of the router weights (rows e_lo .. e_hi-1, contiguous)
     // is requested into L2 first, so its DRAM latency overlaps the staging below
+    // (and, under programmatic dependent launch, the previous kernel's tail: the
+    // weights do not depend on it; x does, so the staging waits for it)
     const int e_lo = rank * EB, e_hi = min(E, e_lo + EB);
     if (e_hi > e_lo) {
         const char *slice = reinterpret_cast<const char *>(wr + (size_t)e_lo * H);
@@ -337,6 +339,8 @@ __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(NT)
         for (size_t off = (size_t)threadIdx.x * 128; off < bytes; off += (size_t)NT * 128)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(slice + off));
     }
+    pdl_wait();
+    pdl_launch_dependents();
 
     // the group's activation rows (zero past the last token)
     const int h4 = H / 4;
@@ -442,8 +446,9 @@ cudaError_t launch_router(const uint16_t *x, const float *wr, int T, int H, int 
         attr[dev] = true;
     }
     dim3 grid(kRouterCluster, (unsigned)((T + TOK - 1) / TOK));
-    kern<<<grid, NT, router_smem(TOK, H, E), s>>>(x, wr, T, H, E, k, logits, ids, w);
-    return cudaGetLastError();
+    // programmatic dependent launch (the cluster shape comes from the kernel's
+    // __cluster_dims__)
+    return launch_pdl(kern, grid, dim3(NT), router_smem(TOK, H, E), s, x, wr, T, H, E, k, logits, ids, w);
 }
 
 template <int VPL>

@@ -804,6 +804,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         const int r = quad * 32 + lane, hf = (dw % kDeqWarps) / 4;
         int stage = 0, rstage = 0;
         uint32_t step = 0;                              // stages seen, across items
+        int a_cur = 0;                                  // active expert of the current item
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
             // int4: the group scale of this thread's atom is loaded one of the
             // group's stages ahead (the scales are read from global memory, where
@@ -812,10 +813,19 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
             // its warps skip decoding the item: that alone is 4% at decode.
             const uint16_t *srow = nullptr;
             if (FMT == MOE_W_INT4) {
-                const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
-                const int wrow = PHASE == 1 ? (r < 64 ? it.m0 * 64 + r : p.L.I + it.m0 * 64 + r - 64)
-                                            : min(it.m0 * kBlockM + r, p.n_units - 1);
-                srow = reinterpret_cast<const uint16_t *>(scale_blob(p, it.e) + (PHASE == 1 ? p.L.off.s13 : p.L.off.s2)) +
+                // the item's active expert: items come in increasing order, so the
+                // search starts at the previous item's (and, unlike decode_item, it
+                // reads no route counts or offsets from global memory)
+                int hi = n_act - 1;
+                while (a_cur < hi) {
+                    const int mid = (a_cur + hi + 1) >> 1;
+                    if (s_base[mid] <= item) a_cur = mid; else hi = mid - 1;
+                }
+                const int mt = (item - s_base[a_cur]) % m_tiles;
+                const int wrow = PHASE == 1 ? (r < 64 ? mt * 64 + r : p.L.I + mt * 64 + r - 64)
+                                            : min(mt * kBlockM + r, p.n_units - 1);
+                srow = reinterpret_cast<const uint16_t *>(scale_blob(p, s_act[a_cur]) +
+                                                          (PHASE == 1 ? p.L.off.s13 : p.L.off.s2)) +
                        (size_t)wrow * (p.K / 64);
             }
             auto scale_at = [&](int kq) -> uint16_t {

@@ -11,7 +11,12 @@
 // RemoteExperts::begin).  An expert is reached through the slot table
 // (expert_blob()).
 //
-// Work decomposition.  A work item is (active expert, chunk of <= 8 of its
+// One token (T = 1) has kernels of its own (k_ffn_gemv_tok, below): the k
+// routes' rows are split evenly over all warps, each warp streams its rows
+// without pausing between them, and the set-up before the first weight load is
+// a single round of loads.
+//
+// Work decomposition (T > 1).  A work item is (active expert, chunk of <= 8 of its
 // routes, tile of output rows).  Each CTA (8 warps) takes a contiguous range
 // of items, so consecutive items share an expert and the routes' activations
 // stay in shared memory (fp32, bank-conflict-free "sub-plane" layout).  Inside
@@ -22,6 +27,8 @@
 // L1-bypassing loads, U chunks per row in flight; the partial dot products
 // are reduced across the group with xor shuffles.  LG is chosen so that each
 // lane streams about 11 chunks of each row (K = 2816 or 704).
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -36,13 +43,16 @@ struct FfnParams {
     uint16_t *h;                  // [R][I] bf16 (phase 1 out / phase 2 in)
     float *rows;                  // [R][H] fp32
     int lg;                       // lanes per row group (power of two, <= 32)
+    int xs_floats;                // one-token kernels: activation floats shared memory holds
 };
 
 namespace {
 
-// First slot fault a GEMV kernel recorded (0 = none): 0x2005 for an expert
-// whose slot is past the pool (info = the slot id); the expert's routes are
-// skipped.  Read and cleared by moe_take_device_errors().
+// First fault a GEMV kernel recorded (0 = none): 0x2005 for an expert whose
+// slot is past the pool (info = the slot id; the expert's routes are skipped),
+// 0x2007 for a one-token CTA whose activations would not fit the shared memory
+// it was launched with (info = routes; the CTA does nothing; the host's sizing
+// rules it out).  Read and cleared by moe_take_device_errors().
 __device__ unsigned int g_gemv_error;
 __device__ unsigned int g_gemv_error_info;
 __device__ __forceinline__ void record_gemv_error(unsigned code, unsigned info) {
@@ -52,6 +62,7 @@ __device__ __forceinline__ void record_gemv_error(unsigned code, unsigned info) 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kNTM = 8;  // routes per work item
+constexpr size_t kTokSmemMax = 96 * 1024;  // one-token kernels: activation bytes per CTA
 
 template <int FMT> struct Fmt;
 template <> struct Fmt<MOE_W_BF16> { static constexpr int kElems = 8; };   // per 16-byte chunk
@@ -120,6 +131,22 @@ __device__ void load_acts(const FfnParams &p, float *xs, int row0, int nt, int K
         const int c = e0 / EC, sp = (e0 % EC) / 4;
         float4 *d0 = reinterpret_cast<float4 *>(xs + ((size_t)(t * SP + sp) * nchunks + c) * 4);
         float4 *d1 = reinterpret_cast<float4 *>(xs + ((size_t)(t * SP + sp + 1) * nchunks + c) * 4);
+        *d0 = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+        *d1 = make_float4(bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w));
+    }
+}
+
+// The single token's activations (T = 1: token 0) into shared memory, in
+// load_acts's layout.
+template <int FMT>
+__device__ void load_x0(const FfnParams &p, float *xs, int K, int nchunks) {
+    constexpr int EC = Fmt<FMT>::kElems;
+    for (int piece = threadIdx.x; piece < K / 8; piece += kThreads) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(p.x + (size_t)piece * 8);
+        const int e0 = piece * 8;
+        const int c = e0 / EC, sp = (e0 % EC) / 4;
+        float4 *d0 = reinterpret_cast<float4 *>(xs + ((size_t)sp * nchunks + c) * 4);
+        float4 *d1 = reinterpret_cast<float4 *>(xs + ((size_t)(sp + 1) * nchunks + c) * 4);
         *d0 = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
         *d1 = make_float4(bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w));
     }
@@ -267,12 +294,7 @@ __device__ __forceinline__ void run_item(const FfnParams &p, const float *xs, co
     }
 }
 
-// NTMAX = 1: the one-token kernel (every expert has one route): only the
-// single-route item code is instantiated, which leaves registers for more
-// chunks of each row in flight (bf16: U = 11, a lane's whole share of a row at
-// H = 2816 / I = 704); an expert with more routes is still handled, one route
-// at a time.
-template <int FMT, int PHASE, int RWP, int U, int NTMAX>
+template <int FMT, int PHASE, int RWP, int U>
 __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
     constexpr int UPG = PHASE == 1 ? RWP / 2 : RWP;
     constexpr int EC = Fmt<FMT>::kElems;
@@ -304,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
             const int n = (e < E) ? __ldg(p.counts + e) : 0;
             const bool act = n > 0;
             const unsigned m = __ballot_sync(0xffffffffu, act);
-            const int items = act ? tiles * ((n + NTMAX - 1) / NTMAX) : 0;
+            const int items = act ? tiles * ((n + kNTM - 1) / kNTM) : 0;
             int inc = items;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -368,8 +390,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
         const int chunk = rem / tiles, tile = rem - chunk * tiles;
         const int e = s_act[a];
         const int n_e = __ldg(p.counts + e);
-        const int row0 = __ldg(p.offsets + e) + chunk * NTMAX;
-        const int nt = min(NTMAX, n_e - chunk * NTMAX);
+        const int row0 = __ldg(p.offsets + e) + chunk * kNTM;
+        const int nt = min(kNTM, n_e - chunk * kNTM);
         const uint8_t *blob = expert_blob(p.L, e);
         if (blob == nullptr) {
             // the expert's slot is past the pool: nothing of this item is read or
@@ -385,16 +407,184 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
             cur_key = key;
         }
         const int u0 = tile * upi + gi * UPG;
-        if (NTMAX == 1) {
-            // route t0's activations are sub-planes t0*SP .. of xs
-            constexpr int SP = Fmt<FMT>::kElems / 4;
-            for (int t0 = 0; t0 < nt; ++t0)
-                run_item<FMT, PHASE, RWP, U, 1>(p, xs + (size_t)t0 * SP * nchunks * 4, blob, u0, row0 + t0, 1, K,
-                                                 nchunks, li, lg);
-        } else if (nt > 4) run_item<FMT, PHASE, RWP, U, 8>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
+        if (nt > 4) run_item<FMT, PHASE, RWP, U, 8>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
         else if (nt > 2) run_item<FMT, PHASE, RWP, U, 4>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
         else if (nt > 1) run_item<FMT, PHASE, RWP, U, 2>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
         else run_item<FMT, PHASE, RWP, U, 1>(p, xs, blob, u0, row0, nt, K, nchunks, li, lg);
+    }
+}
+
+// One token (T = 1: k routes of token 0, sorted by expert).  A unit is one
+// gate/up row pair (phase 1) or two consecutive output rows (phase 2) of one
+// route; the k x units are split evenly over the warps of the grid, and inside
+// a warp its 32/lg lane groups take consecutive units.  A unit is read in P
+// passes of C 16-byte chunks per lane and row; while a lane consumes chunk j of
+// one pass it already loads chunk j of its next pass (of the same unit or of its
+// next one), so a warp's weight stream does not stop between units.  The set-up
+// before the first weight load is one round of loads (the offsets), and phase 2
+// issues its first weight loads before it waits for phase 1 (they do not
+// depend on it).
+template <int FMT, int PHASE, int C>
+__global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
+    constexpr int EC = Fmt<FMT>::kElems, SP = EC / 4;
+    extern __shared__ __align__(16) float xs[];
+    __shared__ int s_exp[kMaxK];
+    __shared__ int s_nroutes;
+    const int H = p.L.H, I = p.L.I;
+    const int K = PHASE == 1 ? H : I;
+    const int nchunks = K / EC;
+    const int n_units = PHASE == 1 ? I : (H + 1) / 2;
+    const int lg = p.lg, gpw = 32 / lg;
+    const int P = (nchunks + lg * C - 1) / (lg * C);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int li = lane & (lg - 1), gi = lane / lg;
+    // phase 1 waits for the permutation before anything else; phase 2 may be
+    // scheduled as soon as phase 1 has started and waits for h further down
+    if (PHASE == 1) pdl_wait();
+    pdl_launch_dependents();
+    // expert of every sorted route (sorted position sr lies in [offsets[e],
+    // offsets[e+1])), and the number of routes: offsets[E], which is below k
+    // when the permutation dropped invalid ids
+    if (threadIdx.x == 0) s_nroutes = min(__ldg(p.offsets + p.L.E), p.k);
+    for (int e = threadIdx.x; e < p.L.E; e += kThreads) {
+        const int lo = __ldg(p.offsets + e), hi = min(__ldg(p.offsets + e + 1), p.k);
+        for (int sr = lo; sr < hi; ++sr) s_exp[sr] = e;
+    }
+    __syncthreads();
+    const int R = s_nroutes;
+    const long long N = (long long)R * n_units;
+    const long long W = (long long)gridDim.x * kWarps;
+    const long long wg = (long long)blockIdx.x * kWarps + warp;
+    const int w_u0 = (int)(N * wg / W), w_u1 = (int)(N * (wg + 1) / W);
+    const int steps = (w_u1 - w_u0 + gpw - 1) / gpw * P;
+    // the routes whose activations this CTA reads (its warps' units are contiguous)
+    const int c_u0 = (int)(N * ((long long)blockIdx.x * kWarps) / W);
+    const int c_u1 = (int)(N * ((long long)(blockIdx.x + 1) * kWarps) / W);
+    const int s_lo = c_u0 / n_units;
+    const int s_hi = c_u1 > c_u0 ? (c_u1 - 1) / n_units : s_lo;
+    if ((PHASE == 1 ? 1 : s_hi - s_lo + 1) * K > p.xs_floats) {
+        // cannot happen with the host's sizing (same for every thread of the CTA)
+        if (threadIdx.x == 0) record_gemv_error(0x2007u, (unsigned)(s_hi - s_lo + 1));
+        return;
+    }
+    const uint64_t qoff = PHASE == 1 ? p.L.off.q13 : p.L.off.q2;
+    const uint64_t soff = PHASE == 1 ? p.L.off.s13 : p.L.off.s2;
+    const size_t row_bytes = (size_t)nchunks * 16;
+
+    // a lane's view of step st: route, first row, where its chunks start;
+    // w0 == nullptr: nothing to load (past the warp's units, or a slot fault)
+    struct Step { const uint8_t *w0; const uint16_t *s0; int sr, r0, c0; bool live, v1; };
+    const size_t dw = PHASE == 1 ? (size_t)I * row_bytes : row_bytes;  // second row - first row
+    const int ds = PHASE == 1 ? I * (K / 64) : K / 64;                  // the same for int4 scales
+    auto step_info = [&](int st, Step &x) {
+        const int trip = st / P, pass = st - trip * P;
+        const int u = w_u0 + trip * gpw + gi;
+        x.live = st < steps && u < w_u1;
+        x.c0 = pass * lg * C + li;
+        x.sr = 0; x.r0 = 0; x.v1 = false; x.w0 = nullptr; x.s0 = nullptr;
+        if (!x.live) return;
+        x.sr = u / n_units;
+        const int i = u - x.sr * n_units;
+        x.r0 = PHASE == 1 ? i : 2 * i;
+        x.v1 = PHASE == 1 || 2 * i + 1 < H;
+        const uint8_t *blob = expert_blob(p.L, s_exp[x.sr]);
+        if (blob == nullptr) return;
+        x.w0 = blob + qoff + (size_t)x.r0 * row_bytes;
+        if (FMT == MOE_W_INT4) x.s0 = reinterpret_cast<const uint16_t *>(blob + soff) + (size_t)x.r0 * (K / 64);
+    };
+
+    uint4 wq[C][2];
+    float sc[C][2];
+    Step cur;
+    step_info(0, cur);
+    {
+        const size_t d1 = cur.v1 ? dw : 0;
+        const int e1 = cur.v1 ? ds : 0;
+#pragma unroll
+        for (int j = 0; j < C; ++j) {
+            const int c = cur.c0 + j * lg;
+            const bool ok = cur.w0 != nullptr && c < nchunks;
+            wq[j][0] = ok ? ld_stream_v4(cur.w0 + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+            wq[j][1] = ok ? ld_stream_v4(cur.w0 + d1 + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+            if (FMT == MOE_W_INT4) {
+                sc[j][0] = ok ? bf16_to_f32(__ldg(cur.s0 + (c >> 1))) : 0.0f;
+                sc[j][1] = ok ? bf16_to_f32(__ldg(cur.s0 + e1 + (c >> 1))) : 0.0f;
+            }
+        }
+    }
+    if (PHASE == 2) pdl_wait();
+    if (PHASE == 1) load_x0<FMT>(p, xs, K, nchunks);
+    else load_acts<FMT, 2>(p, xs, s_lo, s_hi - s_lo + 1, K, nchunks);
+    __syncthreads();
+
+    float a0 = 0.0f, a1 = 0.0f;
+    for (int st = 0; st < steps; ++st) {
+        Step nx;
+        step_info(st + 1, nx);
+        // a lane group past its warp's units computes nothing (its loads were
+        // skipped too) and stays on the first route's activations
+        const int tx = (PHASE == 1 || !cur.live) ? 0 : cur.sr - s_lo;
+        const float *xt = xs + (size_t)tx * SP * nchunks * 4;
+#pragma unroll
+        for (int j = 0; j < C; ++j) {
+            const int c = cur.c0 + j * lg;
+            const uint4 q0 = wq[j][0], q1 = wq[j][1];
+            const float s0 = FMT == MOE_W_INT4 ? sc[j][0] : 1.0f, s1 = FMT == MOE_W_INT4 ? sc[j][1] : 1.0f;
+            {   // chunk j of the next step
+                const int cn = nx.c0 + j * lg;
+                const bool ok = nx.w0 != nullptr && cn < nchunks;
+                const size_t d1 = nx.v1 ? dw : 0;
+                wq[j][0] = ok ? ld_stream_v4(nx.w0 + (size_t)cn * 16) : make_uint4(0, 0, 0, 0);
+                wq[j][1] = ok ? ld_stream_v4(nx.w0 + d1 + (size_t)cn * 16) : make_uint4(0, 0, 0, 0);
+                if (FMT == MOE_W_INT4) {
+                    const int e1 = nx.v1 ? ds : 0;
+                    sc[j][0] = ok ? bf16_to_f32(__ldg(nx.s0 + (cn >> 1))) : 0.0f;
+                    sc[j][1] = ok ? bf16_to_f32(__ldg(nx.s0 + e1 + (cn >> 1))) : 0.0f;
+                }
+            }
+            if (cur.live && c < nchunks) {
+                float p0 = 0.0f, p1 = 0.0f;
+#pragma unroll
+                for (int spi = 0; spi < SP; ++spi) {
+                    float w0[4], w1[4];
+                    decode4<FMT>(q0, spi, w0);
+                    decode4<FMT>(q1, spi, w1);
+                    const float4 xv = *reinterpret_cast<const float4 *>(xt + ((size_t)spi * nchunks + c) * 4);
+                    p0 = fmaf(w0[0], xv.x, p0); p0 = fmaf(w0[1], xv.y, p0);
+                    p0 = fmaf(w0[2], xv.z, p0); p0 = fmaf(w0[3], xv.w, p0);
+                    p1 = fmaf(w1[0], xv.x, p1); p1 = fmaf(w1[1], xv.y, p1);
+                    p1 = fmaf(w1[2], xv.z, p1); p1 = fmaf(w1[3], xv.w, p1);
+                }
+                if (FMT == MOE_W_INT4) { a0 = fmaf(s0, p0, a0); a1 = fmaf(s1, p1, a1); }
+                else { a0 += p0; a1 += p1; }
+            }
+        }
+        if ((st + 1) % P == 0) {  // the unit's last pass: reduce over the group, write
+            for (int off = lg >> 1; off > 0; off >>= 1) {
+                a0 += __shfl_xor_sync(0xffffffffu, a0, off);
+                a1 += __shfl_xor_sync(0xffffffffu, a1, off);
+            }
+            if (cur.live && li == 0) {
+                if (cur.w0 == nullptr) {
+                    record_gemv_error(0x2005u, (unsigned)__ldg(p.L.slot_table + s_exp[cur.sr]));
+                } else {
+                    const int r1 = PHASE == 1 ? I + cur.r0 : cur.r0 + 1;
+                    if (FMT == MOE_W_INT8) {
+                        const float *sp = reinterpret_cast<const float *>(cur.w0 - qoff - (size_t)cur.r0 * row_bytes + soff);
+                        a0 *= __ldg(sp + cur.r0);
+                        if (cur.v1) a1 *= __ldg(sp + r1);
+                    }
+                    if (PHASE == 1) {
+                        p.h[(size_t)cur.sr * I + cur.r0] = f32_to_bf16_rne(gelu_tanh(a0) * a1);
+                    } else {
+                        p.rows[(size_t)cur.sr * H + cur.r0] = a0;
+                        if (cur.v1) p.rows[(size_t)cur.sr * H + r1] = a1;
+                    }
+                }
+            }
+            a0 = 0.0f; a1 = 0.0f;
+        }
+        cur = nx;
     }
 }
 
@@ -406,14 +596,14 @@ int pick_lg(int nchunks, int per_lane) {
     return lg;
 }
 
-template <int FMT, int PHASE, int RWP, int U, int NTMAX>
+template <int FMT, int PHASE, int RWP, int U>
 cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
     FfnParams p = p0;
     const int K = PHASE == 1 ? p.L.H : p.L.I;
     const int nchunks = K / Fmt<FMT>::kElems;
     p.lg = pick_lg(nchunks, 8);
-    const size_t smem = (size_t)NTMAX * K * sizeof(float);
-    auto kern = k_ffn_gemv<FMT, PHASE, RWP, U, NTMAX>;
+    const size_t smem = (size_t)kNTM * K * sizeof(float);
+    auto kern = k_ffn_gemv<FMT, PHASE, RWP, U>;
     // one-time set-up per device and shared-memory size (kept out of stream
     // capture: after the first call a launch is the only API call made here)
     static int cached_smem[kMaxDevices] = {}, cached_per_sm[kMaxDevices] = {};
@@ -435,23 +625,66 @@ cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
     return launch_pdl(kern, dim3((unsigned)(n_sm * per_sm)), dim3(kThreads), smem, s, p);
 }
 
+
+// Shared-memory floats a one-token kernel needs for a CTA's activations
+// (phase 1: the token; phase 2: the h rows of the routes its units touch),
+// with a grid of at least n_sm CTAs.
+size_t tok_xs_floats(const FfnParams &p, int phase, int n_sm) {
+    if (phase == 1) return (size_t)p.L.H;
+    const long long n_units = (p.L.H + 1) / 2, N = (long long)p.k * n_units;
+    const long long per_cta = (N + n_sm - 1) / n_sm;
+    const long long span = std::min<long long>(p.k, (per_cta - 1) / n_units + 2);
+    return (size_t)span * p.L.I;
+}
+
+template <int FMT, int PHASE, int C>
+cudaError_t launch_tok(const FfnParams &p0, int n_sm, cudaStream_t s) {
+    FfnParams p = p0;
+    const int nchunks = (PHASE == 1 ? p.L.H : p.L.I) / Fmt<FMT>::kElems;
+    int lg = 1;  // the narrowest group that covers a row in one pass, at most a warp
+    while (lg < 32 && lg * C < nchunks) lg <<= 1;
+    p.lg = lg;
+    p.xs_floats = (int)tok_xs_floats(p, PHASE, n_sm);
+    const size_t smem = (size_t)p.xs_floats * sizeof(float);
+    auto kern = k_ffn_gemv_tok<FMT, PHASE, C>;
+    static size_t cached_smem[kMaxDevices] = {};
+    static int cached_per_sm[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (cached_smem[dev] < smem) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        int per_sm = 0;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+        if (err != cudaSuccess) return err;
+        cached_per_sm[dev] = per_sm < 1 ? 1 : per_sm;
+        cached_smem[dev] = smem;
+    }
+    return launch_pdl(kern, dim3((unsigned)(n_sm * cached_per_sm[dev])), dim3(kThreads), smem, s, p);
+}
+
 template <int FMT>
 cudaError_t launch_fmt(const FfnParams &p, int n_sm, cudaStream_t s) {
     // rows per lane group: 2 (one gate/up pair in phase 1); U chunks
     // of each row in flight, so a lane keeps 8 x 16 bytes of weights in flight
     constexpr int RWP = 2;
     constexpr int U = 8 / RWP;
-    if (p.T == 1) {  // one token: at most one route per expert (unless ids repeat)
-        // chunks per row in flight: all 11 of a lane's share for bf16; 6 for the
-        // int formats, whose expansion needs the registers
-        constexpr int U1 = FMT == MOE_W_BF16 ? 11 : 6;
-        cudaError_t err = launch_phase<FMT, 1, RWP, U1, 1>(p, n_sm, s);
+    // one token: the streaming kernels above, while a CTA's activations fit in
+    // shared memory beside a second CTA (at H = 2816, I = 704: 11 KiB in phase 1,
+    // 5.5 KiB in phase 2); chunks per lane and row in each pass: 6 (4 for int4,
+    // whose scales take registers too)
+    if (p.T == 1 && p.k <= kMaxK && tok_xs_floats(p, 1, n_sm) * 4 <= kTokSmemMax &&
+        tok_xs_floats(p, 2, n_sm) * 4 <= kTokSmemMax) {
+        constexpr int C = FMT == MOE_W_INT4 ? 4 : 6;
+        cudaError_t err = launch_tok<FMT, 1, C>(p, n_sm, s);
         if (err != cudaSuccess) return err;
-        return launch_phase<FMT, 2, RWP, U1, 1>(p, n_sm, s);
+        return launch_tok<FMT, 2, C>(p, n_sm, s);
     }
-    cudaError_t err = launch_phase<FMT, 1, RWP, U, kNTM>(p, n_sm, s);
+    cudaError_t err = launch_phase<FMT, 1, RWP, U>(p, n_sm, s);
     if (err != cudaSuccess) return err;
-    return launch_phase<FMT, 2, RWP, U, kNTM>(p, n_sm, s);
+    return launch_phase<FMT, 2, RWP, U>(p, n_sm, s);
 }
 
 }  // namespace

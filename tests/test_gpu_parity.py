@@ -578,9 +578,9 @@ def test_layer_with_min_weight_matches_oracle():
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
 def test_one_token_with_repeated_ids(fmt):
-    """The one-token GEMV kernel assumes one route per expert but must still be
-    right when a caller's ids repeat an expert within the token (here experts 2
-    and 5 twice each, and one dropped id)."""
+    """One-token GEMV calls must be right when a caller's ids repeat an expert
+    within the token (here experts 2 and 5 twice each) and when the permutation
+    dropped an id (so fewer than k routes have an expert)."""
     E, H, I, k = 8, 256, 128, 6
     w13, w2 = syn.expert_weights(E, H, I, seed=12)
     L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
@@ -603,10 +603,11 @@ def test_one_token_with_repeated_ids(fmt):
 @pytest.mark.parametrize("E,H,I,k", [(8, 256, 128, 2), (6, 1024, 320, 4), (16, 512, 192, 8), (12, 2816, 704, 8),
                                      (4, 64, 64, 1)])
 def test_one_token_every_element(fmt, E, H, I, k):
-    """One-token batches through the GEMV kernels (the one-token kernels spread
-    the rows of every routed expert over all lane groups; phase 1 writes the gate
-    and up projections, phase 2 forms h while staging it): every row against the
-    oracle, at shapes whose rows split unevenly over the lane groups."""
+    """One-token batches through the GEMV path's one-token kernels (the k routes'
+    rows split evenly over all warps of the grid, each read in passes of a few
+    chunks per lane): every row against the oracle, at shapes whose rows split
+    unevenly over the warps and lane groups, and rows that take one pass or
+    several."""
     w13, w2 = syn.expert_weights(E, H, I, seed=E * 7 + I)
     x = syn.activations(1, H, seed=H)
     lg = syn.router_logits(1, E, "normal", seed=k)

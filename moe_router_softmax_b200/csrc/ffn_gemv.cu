@@ -43,7 +43,13 @@ struct FfnParams {
     uint16_t *h;                  // [R][I] bf16 (phase 1 out / phase 2 in)
     float *rows;                  // [R][H] fp32
     int lg;                       // lanes per row group (power of two, <= 32)
-    int xs_floats;                // one-token kernels: activation floats shared memory holds
+    // one-token kernels: activation floats shared memory holds; passes per unit;
+    // the N = k * units split over the W warps of the grid (warp w starts at
+    // floor(w * N / W)) and 1 / W; 1 / units per route (division-free indices)
+    int xs_floats, passes;
+    unsigned n_all, n_warps;
+    double inv_warps;
+    float inv_units;
 };
 
 namespace {
@@ -424,6 +430,23 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnParams p) {
 // before the first weight load is one round of loads (the offsets), and phase 2
 // issues its first weight loads before it waits for phase 1 (they do not
 // depend on it).
+// a / b for 0 <= a < 2^24 and b >= 1, from inv_b = 1/b rounded to float: the
+// float quotient is within 1/16 of a/b there, so one correction step is exact.
+__device__ __forceinline__ int div_small(int a, int b, float inv_b) {
+    int q = (int)((float)a * inv_b);
+    if (q * b > a) --q;
+    else if ((q + 1) * b <= a) ++q;
+    return q;
+}
+// floor(a / b) for a < 2^32, 1 <= b < 2^31, from inv_b = 1/b rounded to double
+// (quotient within 2^-20 of a/b; one correction step).
+__device__ __forceinline__ unsigned div_u32(unsigned a, unsigned b, double inv_b) {
+    unsigned q = (unsigned)((double)a * inv_b);
+    if ((unsigned long long)q * b > a) --q;
+    else if ((unsigned long long)(q + 1) * b <= a) ++q;
+    return q;
+}
+
 template <int FMT, int PHASE, int C>
 __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     constexpr int EC = Fmt<FMT>::kElems, SP = EC / 4;
@@ -434,12 +457,31 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     const int K = PHASE == 1 ? H : I;
     const int nchunks = K / EC;
     const int n_units = PHASE == 1 ? I : (H + 1) / 2;
-    const int lg = p.lg, gpw = 32 / lg;
-    const int P = (nchunks + lg * C - 1) / (lg * C);
+    const int lg = p.lg, gpw = 32 / lg, P = p.passes;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int li = lane & (lg - 1), gi = lane / lg;
-    // phase 1 waits for the permutation before anything else; phase 2 may be
-    // scheduled as soon as phase 1 has started and waits for h further down
+    // the warp's units (all k routes' units split evenly over the grid's warps;
+    // units of routes the permutation left empty are skipped below) and the
+    // routes whose activations the CTA reads: no device data needed yet
+    auto warp_start = [&](unsigned w) { return (int)div_u32(w * p.n_all, p.n_warps, p.inv_warps); };
+    const int w_u0 = warp_start(blockIdx.x * kWarps + warp), w_u1 = warp_start(blockIdx.x * kWarps + warp + 1);
+    const int trips = (w_u1 - w_u0 + gpw - 1) / gpw;
+    const int c_u0 = warp_start(blockIdx.x * kWarps), c_u1 = warp_start((blockIdx.x + 1) * kWarps);
+    if (c_u1 == c_u0) return;  // no units (fewer units than warps); exiting also releases dependents
+    const int s_lo = div_small(c_u0, n_units, p.inv_units);
+    const int s_hi = div_small(c_u1 - 1, n_units, p.inv_units);
+    if ((PHASE == 1 ? 1 : s_hi - s_lo + 1) * K > p.xs_floats) {
+        // cannot happen with the host's sizing (same for every thread of the CTA)
+        if (threadIdx.x == 0) record_gemv_error(0x2007u, (unsigned)(s_hi - s_lo + 1));
+        return;
+    }
+    // the lane group's first unit: route and unit within the route
+    int nx_u = w_u0 + gi;
+    int nx_sr = div_small(nx_u, n_units, p.inv_units);
+    int nx_i = nx_u - nx_sr * n_units;
+    int nx_trip = 0, nx_pass = 0;
+    // phase 1 waits for the permutation here; phase 2 may be scheduled as soon
+    // as phase 1 has started and waits for h further down
     if (PHASE == 1) pdl_wait();
     pdl_launch_dependents();
     // expert of every sorted route (sorted position sr lies in [offsets[e],
@@ -452,51 +494,44 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     }
     __syncthreads();
     const int R = s_nroutes;
-    const long long N = (long long)R * n_units;
-    const long long W = (long long)gridDim.x * kWarps;
-    const long long wg = (long long)blockIdx.x * kWarps + warp;
-    const int w_u0 = (int)(N * wg / W), w_u1 = (int)(N * (wg + 1) / W);
-    const int steps = (w_u1 - w_u0 + gpw - 1) / gpw * P;
-    // the routes whose activations this CTA reads (its warps' units are contiguous)
-    const int c_u0 = (int)(N * ((long long)blockIdx.x * kWarps) / W);
-    const int c_u1 = (int)(N * ((long long)(blockIdx.x + 1) * kWarps) / W);
-    const int s_lo = c_u0 / n_units;
-    const int s_hi = c_u1 > c_u0 ? (c_u1 - 1) / n_units : s_lo;
-    if ((PHASE == 1 ? 1 : s_hi - s_lo + 1) * K > p.xs_floats) {
-        // cannot happen with the host's sizing (same for every thread of the CTA)
-        if (threadIdx.x == 0) record_gemv_error(0x2007u, (unsigned)(s_hi - s_lo + 1));
-        return;
-    }
     const uint64_t qoff = PHASE == 1 ? p.L.off.q13 : p.L.off.q2;
     const uint64_t soff = PHASE == 1 ? p.L.off.s13 : p.L.off.s2;
     const size_t row_bytes = (size_t)nchunks * 16;
 
-    // a lane's view of step st: route, first row, where its chunks start;
-    // w0 == nullptr: nothing to load (past the warp's units, or a slot fault)
+    // a lane's view of a step (one pass over one unit): route, first row, where
+    // its chunks start; w0 == nullptr: nothing to load (past the warp's units, a
+    // route the permutation left empty, or a slot fault).  next_step() takes the
+    // step after the previous one, walking (trip, pass) and (route, unit).
     struct Step { const uint8_t *w0; const uint16_t *s0; int sr, r0, c0; bool live, v1; };
     const size_t dw = PHASE == 1 ? (size_t)I * row_bytes : row_bytes;  // second row - first row
     const int ds = PHASE == 1 ? I * (K / 64) : K / 64;                  // the same for int4 scales
-    auto step_info = [&](int st, Step &x) {
-        const int trip = st / P, pass = st - trip * P;
-        const int u = w_u0 + trip * gpw + gi;
-        x.live = st < steps && u < w_u1;
-        x.c0 = pass * lg * C + li;
-        x.sr = 0; x.r0 = 0; x.v1 = false; x.w0 = nullptr; x.s0 = nullptr;
-        if (!x.live) return;
-        x.sr = u / n_units;
-        const int i = u - x.sr * n_units;
-        x.r0 = PHASE == 1 ? i : 2 * i;
-        x.v1 = PHASE == 1 || 2 * i + 1 < H;
-        const uint8_t *blob = expert_blob(p.L, s_exp[x.sr]);
-        if (blob == nullptr) return;
-        x.w0 = blob + qoff + (size_t)x.r0 * row_bytes;
-        if (FMT == MOE_W_INT4) x.s0 = reinterpret_cast<const uint16_t *>(blob + soff) + (size_t)x.r0 * (K / 64);
+    auto next_step = [&](Step &x) {
+        x.live = nx_trip < trips && nx_u < w_u1 && nx_sr < R;
+        x.c0 = nx_pass * lg * C + li;
+        x.sr = nx_sr;
+        x.r0 = PHASE == 1 ? nx_i : 2 * nx_i;
+        x.v1 = PHASE == 1 || 2 * nx_i + 1 < H;
+        x.w0 = nullptr; x.s0 = nullptr;
+        if (x.live) {
+            const uint8_t *blob = expert_blob(p.L, s_exp[x.sr]);
+            if (blob != nullptr) {
+                x.w0 = blob + qoff + (size_t)x.r0 * row_bytes;
+                if (FMT == MOE_W_INT4) x.s0 = reinterpret_cast<const uint16_t *>(blob + soff) + (size_t)x.r0 * (K / 64);
+            }
+        }
+        if (++nx_pass == P) {
+            nx_pass = 0;
+            ++nx_trip;
+            nx_u += gpw;
+            nx_i += gpw;
+            while (nx_i >= n_units) { nx_i -= n_units; ++nx_sr; }
+        }
     };
 
     uint4 wq[C][2];
     float sc[C][2];
     Step cur;
-    step_info(0, cur);
+    next_step(cur);
     {
         const size_t d1 = cur.v1 ? dw : 0;
         const int e1 = cur.v1 ? ds : 0;
@@ -518,9 +553,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     __syncthreads();
 
     float a0 = 0.0f, a1 = 0.0f;
+    const int steps = trips * P;
     for (int st = 0; st < steps; ++st) {
         Step nx;
-        step_info(st + 1, nx);
+        next_step(nx);
         // a lane group past its warp's units computes nothing (its loads were
         // skipped too) and stays on the first route's activations
         const int tx = (PHASE == 1 || !cur.live) ? 0 : cur.sr - s_lo;
@@ -628,11 +664,12 @@ cudaError_t launch_phase(const FfnParams &p0, int n_sm, cudaStream_t s) {
 
 // Shared-memory floats a one-token kernel needs for a CTA's activations
 // (phase 1: the token; phase 2: the h rows of the routes its units touch),
-// with a grid of at least n_sm CTAs.
+// with a grid of at least n_sm CTAs: a CTA takes at most N / n_sm + 1 of the
+// N units, consecutive ones.
 size_t tok_xs_floats(const FfnParams &p, int phase, int n_sm) {
     if (phase == 1) return (size_t)p.L.H;
     const long long n_units = (p.L.H + 1) / 2, N = (long long)p.k * n_units;
-    const long long per_cta = (N + n_sm - 1) / n_sm;
+    const long long per_cta = N / n_sm + 1;
     const long long span = std::min<long long>(p.k, (per_cta - 1) / n_units + 2);
     return (size_t)span * p.L.I;
 }
@@ -644,7 +681,10 @@ cudaError_t launch_tok(const FfnParams &p0, int n_sm, cudaStream_t s) {
     int lg = 1;  // the narrowest group that covers a row in one pass, at most a warp
     while (lg < 32 && lg * C < nchunks) lg <<= 1;
     p.lg = lg;
+    p.passes = (nchunks + lg * C - 1) / (lg * C);
     p.xs_floats = (int)tok_xs_floats(p, PHASE, n_sm);
+    const int n_units = PHASE == 1 ? p.L.I : (p.L.H + 1) / 2;
+    p.inv_units = 1.0f / (float)n_units;
     const size_t smem = (size_t)p.xs_floats * sizeof(float);
     auto kern = k_ffn_gemv_tok<FMT, PHASE, C>;
     static size_t cached_smem[kMaxDevices] = {};
@@ -662,7 +702,11 @@ cudaError_t launch_tok(const FfnParams &p0, int n_sm, cudaStream_t s) {
         cached_per_sm[dev] = per_sm < 1 ? 1 : per_sm;
         cached_smem[dev] = smem;
     }
-    return launch_pdl(kern, dim3((unsigned)(n_sm * cached_per_sm[dev])), dim3(kThreads), smem, s, p);
+    const int grid = n_sm * cached_per_sm[dev];
+    p.n_all = (unsigned)(p.k * n_units);
+    p.n_warps = (unsigned)(grid * kWarps);
+    p.inv_warps = 1.0 / (double)p.n_warps;
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), smem, s, p);
 }
 
 template <int FMT>
@@ -675,8 +719,11 @@ cudaError_t launch_fmt(const FfnParams &p, int n_sm, cudaStream_t s) {
     // shared memory beside a second CTA (at H = 2816, I = 704: 11 KiB in phase 1,
     // 5.5 KiB in phase 2); chunks per lane and row in each pass: 6 (4 for int4,
     // whose scales take registers too)
+    // (and while w * N stays below 2^32 for every warp w, at up to 8 CTAs per SM)
+    const unsigned long long max_units = (unsigned long long)p.k * std::max(p.L.I, (p.L.H + 1) / 2);
     if (p.T == 1 && p.k <= kMaxK && tok_xs_floats(p, 1, n_sm) * 4 <= kTokSmemMax &&
-        tok_xs_floats(p, 2, n_sm) * 4 <= kTokSmemMax) {
+        tok_xs_floats(p, 2, n_sm) * 4 <= kTokSmemMax &&
+        max_units * (unsigned long long)(n_sm * 8 * kWarps) < (1ull << 32)) {
         constexpr int C = FMT == MOE_W_INT4 ? 4 : 6;
         cudaError_t err = launch_tok<FMT, 1, C>(p, n_sm, s);
         if (err != cudaSuccess) return err;

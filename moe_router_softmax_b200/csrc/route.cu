@@ -64,67 +64,62 @@ __device__ float exp_p(float x) {
     return __fmul_rn(p, pow2_bits(ni));
 }
 
-// A 32-bit key whose unsigned order is the logit order of ranks_before: NaN
-// below every number (key 0, and every NaN alike), -0 equal to +0, otherwise
-// the IEEE bits made monotone (negative: all bits flipped; positive: sign set).
-// Equal keys are then ordered by expert id separately.
+// The routing order: a larger logit ranks first, equal logits (-0 equal to +0)
+// by the lower expert id, NaN after every number.  rank_key gives a 32-bit key
+// whose unsigned order is that logit order: NaN below every number (key 0, and
+// every NaN alike), -0 equal to +0, otherwise the IEEE bits made monotone
+// (negative: all bits flipped; positive: sign set).  Equal keys are then
+// ordered by expert id separately.
 __device__ __forceinline__ uint32_t rank_key(float v) {
     if (v != v) return 0u;
     const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// (va, ea) ranks before (vb, eb): larger logit, then lower id; NaN last.
-__device__ __forceinline__ bool ranks_before(float va, int ea, float vb, int eb) {
-    bool na = va != va, nb = vb != vb;
-    if (na != nb) return nb;
-    if (!na && va != vb) return va > vb;
-    return ea < eb;
-}
-
 // Top-k and weights of one token, by one warp.  load(e) returns logit e for
 // e < E; lane l holds experts l, l+32, ...; the k winners are taken one at a
 // time by a warp arg-best, then the softmax over them (max logit first).
+// Each logit's rank key is formed once (plus one, so that 0 marks a taken or
+// absent slot below every NaN's key of 1); a lane's best slot is its largest key
+// (the first slot on ties: the lower id), the warp's winner the largest key,
+// then the lowest id holding it -- the routing order above.
 template <int VPL, class Load>
 __device__ __forceinline__ void route_token_warp(Load load, int E, int k, int32_t *ids_row, float *w_row) {
     const int lane = threadIdx.x & 31;
     float v[VPL];
-    uint32_t avail = 0;
+    uint32_t key[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
         int e = lane + 32 * i;
         v[i] = 0.0f;
+        key[i] = 0u;
         if (e < E) {
             v[i] = load(e);
-            avail |= 1u << i;
+            key[i] = rank_key(v[i]) + 1u;
         }
     }
     float my_v = 0.0f;
     int my_e = 0;
     for (int j = 0; j < k; ++j) {
-        // best available value held by this lane (ties to the lower id: i ascending)
-        bool has = false;
-        float bv = 0.0f;
-        int be = 0;
+        uint32_t bk = key[0];
+        float bv = v[0];
+        int bi = 0;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            if ((avail >> i) & 1u) {
-                int e = lane + 32 * i;
-                if (!has || ranks_before(v[i], e, bv, be)) {
-                    has = true;
-                    bv = v[i];
-                    be = e;
-                }
+        for (int i = 1; i < VPL; ++i)
+            if (key[i] > bk) {
+                bk = key[i];
+                bv = v[i];
+                bi = i;
             }
-        }
-        // warp arg-best in two reductions: the largest rank key, then the lowest
-        // expert id among the lanes holding it
-        const uint32_t key = has ? rank_key(bv) : 0u;
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-        const int cand = (has && key == kmax) ? be : 0x7fffffff;
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+        const int cand = (bk != 0u && bk == kmax) ? lane + 32 * bi : 0x7fffffff;
         const int win = __reduce_min_sync(0xffffffffu, cand);
         const float wv = __shfl_sync(0xffffffffu, bv, win & 31);
-        if (lane == (win & 31)) avail &= ~(1u << (win >> 5));
+        if (lane == (win & 31)) {
+#pragma unroll
+            for (int i = 0; i < VPL; ++i)
+                if (i == (win >> 5)) key[i] = 0u;
+        }
         if (lane == j) {
             my_v = wv;
             my_e = win;
@@ -282,6 +277,86 @@ __global__ void __launch_bounds__(kFusedThreads) k_route_permute(const float *__
         __syncwarp();
     }
     for (int i = s_total + tid; i < R; i += kFusedThreads) sorted_route[i] = -1;
+}
+
+// The same outputs for one token (T = 1, so k <= 32 routes) from a single
+// warp: lane r holds route r; the counts of the experts a lane owns (a
+// contiguous block of VPL ids) come from one pass over the routes by shuffles,
+// their exclusive scan in id order gives the offsets, and route r goes to
+// offsets[e_r] + (routes before r with the same expert) -- the stable order of
+// moe_permute.  No block barrier, and the hit counters are read before the
+// logits arrive.
+template <int VPL>
+__global__ void __launch_bounds__(32) k_route_permute_warp(const float *__restrict__ logits, int T, int E, int k,
+                                                           int32_t *__restrict__ ids, float *__restrict__ w,
+                                                           int32_t *__restrict__ counts,
+                                                           int32_t *__restrict__ offsets,
+                                                           int32_t *__restrict__ sorted_route,
+                                                           int32_t *__restrict__ route_pos,
+                                                           uint32_t *__restrict__ hits) {
+    __shared__ int32_t s_ids[32];
+    __shared__ float s_wt[32];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x;
+    const int R = T * k;
+    const int e0 = lane * VPL;  // this lane's experts: e0 .. e0 + VPL - 1
+    uint32_t hv[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) hv[i] = (hits != nullptr && e0 + i < E) ? hits[e0 + i] : 0u;
+    for (int t = 0; t < T; ++t) {
+        const float *l = logits + (size_t)t * E;
+        route_token_warp<VPL>([l](int e) { return __ldg(l + e); }, E, k, s_ids + t * k, s_wt + t * k);
+    }
+    __syncwarp();
+    const int raw = lane < R ? s_ids[lane] : -1;
+    const int er = (raw >= 0 && raw < E) ? raw : -1;
+    if (lane < R) {
+        ids[lane] = raw;
+        w[lane] = s_wt[lane];
+    }
+    // one pass over the routes: counts of this lane's experts, and for route
+    // `lane` the valid routes of lower experts and of its expert before it
+    int c[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) c[i] = 0;
+    int lower = 0, same_before = 0;
+    for (int r = 0; r < R; ++r) {
+        const int e = __shfl_sync(0xffffffffu, er, r);
+        const int d = e - e0;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) c[i] += (d == i);
+        lower += (e >= 0 && e < er);
+        same_before += (r < lane && e == er);
+    }
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) sum += c[i];
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int e = e0 + i;
+        if (e < E) {
+            counts[e] = c[i];
+            offsets[e] = run;
+            if (hits) hits[e] = hv[i] + (uint32_t)c[i];
+        }
+        run += c[i];
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0) offsets[E] = total;
+    if (lane < R) {
+        const int pos = er >= 0 ? lower + same_before : -1;
+        route_pos[lane] = pos;
+        if (pos >= 0) sorted_route[pos] = lane;
+        if (lane >= total) sorted_route[lane] = -1;
+    }
 }
 
 // ------------------------------------------------ router projection + top-k
@@ -545,6 +620,18 @@ cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32
         return launch_pdl(kern, grid, block, smem, s, logits, T, E, k, ids, w, counts, offsets, sorted_route,
                           route_pos, hits);
     };
+    if (T == 1) {  // one warp (no shared-memory attribute needed)
+        auto one = [&](auto kern) {
+            return launch_pdl(kern, dim3(1), dim3(32), 0, s, logits, T, E, k, ids, w, counts, offsets, sorted_route,
+                              route_pos, hits);
+        };
+        if (vpl <= 1) return one(k_route_permute_warp<1>);
+        if (vpl <= 2) return one(k_route_permute_warp<2>);
+        if (vpl <= 4) return one(k_route_permute_warp<4>);
+        if (vpl <= 8) return one(k_route_permute_warp<8>);
+        if (vpl <= 16) return one(k_route_permute_warp<16>);
+        return one(k_route_permute_warp<32>);
+    }
     if (vpl <= 1) return go(k_route_permute<1>);
     if (vpl <= 2) return go(k_route_permute<2>);
     if (vpl <= 4) return go(k_route_permute<4>);

@@ -76,12 +76,14 @@ def test_permute_and_hits_bit_exact(T, k, E):
     assert np.array_equal(hits.cpu().numpy().view(np.uint32), oracle.hits(ids, E, hits0))
 
 
-# moe_route_permute: one launch for T <= 16 (the first seven cases, including
-# the boundary T = 16, E = 1024 and T*k = 512), the two kernels beyond it
+# moe_route_permute: one warp for T*k <= 32 (the one-token cases, (3, 11, 5) and
+# the boundary cases with 30 or 32 routes), one CTA for T <= 16 (including
+# T*k = 33 and the boundary T = 16, E = 1024, T*k = 512), the two kernels beyond
 @pytest.mark.parametrize("T,E,k,kind", [(1, 128, 8, "normal"), (8, 128, 8, "biased"), (16, 128, 8, "normal"),
                                         (1, 1024, 32, "normal"), (3, 11, 5, "normal"), (16, 8, 4, "biased"),
                                         (16, 1024, 32, "normal"), (17, 128, 8, "normal"), (64, 128, 8, "biased"),
-                                        (1024, 128, 8, "biased")])
+                                        (1024, 128, 8, "biased"), (4, 128, 8, "biased"), (2, 40, 16, "normal"),
+                                        (5, 1000, 6, "normal"), (1, 1, 1, "normal"), (3, 64, 11, "normal")])
 def test_route_permute_matches_the_oracle_and_the_two_calls(T, E, k, kind):
     lg = syn.router_logits(T, E, kind, seed=7 * T + E)
     rng = np.random.default_rng(T + k)
@@ -103,7 +105,8 @@ def test_route_permute_matches_the_oracle_and_the_two_calls(T, E, k, kind):
     assert np.array_equal(h_one.cpu().numpy().view(np.uint32), oracle.hits(oi, E, hits0))
 
 
-def test_route_permute_ties_nan_inf():
+@pytest.mark.parametrize("T", [30, 5])  # 5 tokens x 6 = 30 routes: the one-warp kernel
+def test_route_permute_ties_nan_inf(T):
     rng = np.random.default_rng(4)
     lg = rng.integers(-2, 3, size=(30, 40)).astype(np.float32)
     lg[0, :] = 0.0
@@ -112,6 +115,7 @@ def test_route_permute_ties_nan_inf():
     lg[3, :] = -np.inf
     lg[3, 9] = 1.0
     lg[4, ::3] = -0.0
+    lg = np.ascontiguousarray(lg[:T])
     ids, w, counts, offsets, sr, rp = moe.moe_route_permute(torch.from_numpy(lg).to(DEV), 6)
     oi, ow = oracle.route_topk(lg, 6)
     assert np.array_equal(ids.cpu().numpy(), oi)

@@ -60,13 +60,13 @@ _CAPTURE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_
 NCU_TRAFFIC_BYTES = {
     ("moe-layer-bf16-decode-T64", "auto"): (1506798080, 1499103232, _CAPTURE + " (gather + 2 tcgen05 launches)"),
     ("moe-layer-bf16-decode-T8", "auto"): (584320256, 582889472, _CAPTURE + " --tokens 8 (gather + 2 tcgen05 launches)"),
-    ("moe-layer-bf16-decode-T1", "auto"): (95552000, 95163904, _CAPTURE + " --tokens 1 (2 GEMV launches)"),
+    ("moe-layer-bf16-decode-T1", "auto"): (95452928, 95163904, _CAPTURE + " --tokens 1 (2 one-token GEMV launches)"),
     ("moe-layer-int8-decode-T64", "auto"): (309052672, 304539136,
                                             _CAPTURE + " --config decode-int8 (gather + 2 tcgen05 launches)"),
     ("moe-layer-int8-decode-T8", "auto"): (143898624, 143187968,
                                            _CAPTURE + " --config decode-int8 --tokens 8 (gather + 2 tcgen05 launches)"),
-    ("moe-layer-int8-decode-T1", "auto"): (47808512, 47719936,
-                                           _CAPTURE + " --config decode-int8 --tokens 1 (2 GEMV launches)"),
+    ("moe-layer-int8-decode-T1", "auto"): (47799040, 47719936,
+                                           _CAPTURE + " --config decode-int8 --tokens 1 (2 one-token GEMV launches)"),
     ("moe-layer-int4-decode-T64", "auto"): (404323840, 398464000,
                                             _CAPTURE + " --config int4-decode (gather + 2 tcgen05 launches)"),
     ("moe-layer-int4-prefill-T1024", "auto"): (520957184, 410189824,

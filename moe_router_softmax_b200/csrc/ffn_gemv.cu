@@ -452,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     constexpr int EC = Fmt<FMT>::kElems, SP = EC / 4;
     extern __shared__ __align__(16) float xs[];
     __shared__ int s_exp[kMaxK];
+    __shared__ const uint8_t *s_blob[kMaxK];
     __shared__ int s_nroutes;
     const int H = p.L.H, I = p.L.I;
     const int K = PHASE == 1 ? H : I;
@@ -484,13 +485,18 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     // as phase 1 has started and waits for h further down
     if (PHASE == 1) pdl_wait();
     pdl_launch_dependents();
-    // expert of every sorted route (sorted position sr lies in [offsets[e],
-    // offsets[e+1])), and the number of routes: offsets[E], which is below k
-    // when the permutation dropped invalid ids
+    // expert and blob of every sorted route (sorted position sr lies in
+    // [offsets[e], offsets[e+1]); the slot-table entry is read in the same round
+    // of loads as the offsets), and the number of routes: offsets[E], which is
+    // below k when the permutation dropped invalid ids
     if (threadIdx.x == 0) s_nroutes = min(__ldg(p.offsets + p.L.E), p.k);
     for (int e = threadIdx.x; e < p.L.E; e += kThreads) {
         const int lo = __ldg(p.offsets + e), hi = min(__ldg(p.offsets + e + 1), p.k);
-        for (int sr = lo; sr < hi; ++sr) s_exp[sr] = e;
+        const uint8_t *blob = expert_blob(p.L, e);
+        for (int sr = lo; sr < hi; ++sr) {
+            s_exp[sr] = e;
+            s_blob[sr] = blob;
+        }
     }
     __syncthreads();
     const int R = s_nroutes;
@@ -513,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
         x.v1 = PHASE == 1 || 2 * nx_i + 1 < H;
         x.w0 = nullptr; x.s0 = nullptr;
         if (x.live) {
-            const uint8_t *blob = expert_blob(p.L, s_exp[x.sr]);
+            const uint8_t *blob = s_blob[x.sr];
             if (blob != nullptr) {
                 x.w0 = blob + qoff + (size_t)x.r0 * row_bytes;
                 if (FMT == MOE_W_INT4) x.s0 = reinterpret_cast<const uint16_t *>(blob + soff) + (size_t)x.r0 * (K / 64);

@@ -483,37 +483,43 @@ def _pool_layers(fmt, E, H, I, w13, w2, slot_of, n_slots):
     return Ld, OL
 
 
+@pytest.mark.parametrize("T", [45, 1])
 @pytest.mark.parametrize("fmt", [0, 1, 2])
 @pytest.mark.parametrize("path", [moe.MOE_FFN_GEMV, moe.MOE_FFN_TC])
-def test_pool_with_more_slots_than_experts_matches_the_oracle(fmt, path):
+def test_pool_with_more_slots_than_experts_matches_the_oracle(fmt, path, T):
     """A pool holds more slots than the layer has experts (prain's 540 cache
     slots are shared by the layers; remote_experts.cpp reads a cached expert from
     its device slot): 8 experts, 24 slots, slot ids up to 23.  Both kernel paths
-    against the oracle on the same slot table, every row and output element."""
-    E, H, I, k, T = 8, 512, 192, 3, 45
+    (at one token the GEMV path's one-token kernels) against the oracle on the
+    same slot table, every row and output element."""
+    E, H, I, k = 8, 512, 192, 3
     w13, w2 = syn.expert_weights(E, H, I, seed=77)
     slot_of = np.array([23, -1, 17, 5, -1, 20, 0, 11], np.int32)
     Ld, OL = _pool_layers(fmt, E, H, I, w13, w2, slot_of, 24)
     x = syn.activations(T, H, seed=78)
     lg = syn.router_logits(T, E, "normal", seed=79)
+    if T == 1:
+        lg[0, 1] += 4.0                      # the token reads a home expert as well as pooled ones
     xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
     ids, w, counts, offsets, sr, rp, rows, y = _run_layer(Ld, torch.from_numpy(lg).to(DEV), xd, k, path=path)
     assert moe.moe_take_device_errors() == (0, 0)
     oi, ow, orows, oy = oracle.moe_layer(OL, lg, x, k)
+    assert (slot_of[oi] >= 0).any() and (slot_of[oi] < 0).any()
     assert np.array_equal(ids.cpu().numpy(), oi)
     assert rel_err(rows.cpu().numpy()[rp.cpu().numpy()], orows) <= FFN_TOL
     assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
 
 
+@pytest.mark.parametrize("T", [40, 1])
 @pytest.mark.parametrize("path", [moe.MOE_FFN_GEMV, moe.MOE_FFN_TC])
-def test_slot_past_the_pool_is_refused_and_reported(path):
+def test_slot_past_the_pool_is_refused_and_reported(path, T):
     """A slot table entry at or past pool_slots is refused on the device: that
     expert's routes are skipped (their rows keep what the caller put there), the
     kernels record the bad slot for moe_take_device_errors, and every other
     expert's rows still match the oracle.  The kernels resolve such an expert to
     its home blob for any address they form, so nothing outside the buffers is
-    read."""
-    E, H, I, k, T = 8, 256, 128, 2, 40
+    read.  At one token the GEMV path runs its one-token kernels."""
+    E, H, I, k = 8, 256, 128, 2
     w13, w2 = syn.expert_weights(E, H, I, seed=81)
     slot_of = np.array([2, -1, 0, -1, 1, -1, -1, -1], np.int32)
     Ld, OL = _pool_layers(2, E, H, I, w13, w2, slot_of, 3)
@@ -522,6 +528,8 @@ def test_slot_past_the_pool_is_refused_and_reported(path):
     Ld.slot_table.copy_(torch.from_numpy(bad))
     x = syn.activations(T, H, seed=82)
     lg = syn.router_logits(T, E, "normal", seed=83)
+    if T == 1:
+        lg[0, 4] += 6.0                      # the token routes to the bad slot's expert
     xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
     moe.moe_take_device_errors()             # start from a clear word
     ids, w = moe.moe_route_topk(torch.from_numpy(lg).to(DEV), k)

@@ -115,6 +115,35 @@ __device__ __forceinline__ void decode4(const uint4 &q, int sp, float w[4]) {
     }
 }
 
+// decode4 as two pairs (w[0], w[1]) and (w[2], w[3]); the int formats' bias is
+// taken off both weights of a pair in one packed subtraction (exact: integers
+// below 2^24), so the values equal decode4's.
+template <int FMT>
+__device__ __forceinline__ void decode4_pairs(const uint4 &q, int sp, float2 &lo, float2 &hi) {
+    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+    if (FMT == MOE_W_BF16) {
+        const uint32_t a = words[2 * sp], b = words[2 * sp + 1];
+        lo = make_float2(bf16_lo(a), bf16_hi(a));
+        hi = make_float2(bf16_lo(b), bf16_hi(b));
+    } else if (FMT == MOE_W_INT8) {
+        const uint32_t a = words[sp] ^ 0x80808080u;
+        const float2 bias = make_float2(-8388736.0f, -8388736.0f);
+        lo = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(a, 0x4B000000u, 0x7540)),
+                                    __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7541))), bias);
+        hi = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(a, 0x4B000000u, 0x7542)),
+                                    __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7543))), bias);
+    } else {
+        const uint32_t word = words[sp >> 1];
+        const uint32_t l4 = word & 0x0F0F0F0Fu, h4 = (word >> 4) & 0x0F0F0F0Fu;
+        const uint32_t s0 = (sp & 1) ? 0x7542u : 0x7540u, s1 = (sp & 1) ? 0x7543u : 0x7541u;
+        const float2 bias = make_float2(-8388616.0f, -8388616.0f);
+        lo = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(l4, 0x4B000000u, s0)),
+                                    __uint_as_float(__byte_perm(h4, 0x4B000000u, s0))), bias);
+        hi = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(l4, 0x4B000000u, s1)),
+                                    __uint_as_float(__byte_perm(h4, 0x4B000000u, s1))), bias);
+    }
+}
+
 // Load the activations of the item's routes into shared memory as fp32.
 // Layout: xs[((t * SP + sp) * nchunks + c) * 4 + i] = x_t[c * kElems + 4 sp + i]
 // so that lanes reading consecutive chunks of one sub-plane hit consecutive
@@ -585,20 +614,22 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
                 }
             }
             if (cur.live && c < nchunks) {
-                float p0 = 0.0f, p1 = 0.0f;
+                // even and odd weights in two packed partial sums (sm_100 packed
+                // fp32 fma: half the fma instructions)
+                float2 p0 = make_float2(0.0f, 0.0f), p1 = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int spi = 0; spi < SP; ++spi) {
-                    float w0[4], w1[4];
-                    decode4<FMT>(q0, spi, w0);
-                    decode4<FMT>(q1, spi, w1);
+                    float2 w0l, w0h, w1l, w1h;
+                    decode4_pairs<FMT>(q0, spi, w0l, w0h);
+                    decode4_pairs<FMT>(q1, spi, w1l, w1h);
                     const float4 xv = *reinterpret_cast<const float4 *>(xt + ((size_t)spi * nchunks + c) * 4);
-                    p0 = fmaf(w0[0], xv.x, p0); p0 = fmaf(w0[1], xv.y, p0);
-                    p0 = fmaf(w0[2], xv.z, p0); p0 = fmaf(w0[3], xv.w, p0);
-                    p1 = fmaf(w1[0], xv.x, p1); p1 = fmaf(w1[1], xv.y, p1);
-                    p1 = fmaf(w1[2], xv.z, p1); p1 = fmaf(w1[3], xv.w, p1);
+                    const float2 xl = make_float2(xv.x, xv.y), xh = make_float2(xv.z, xv.w);
+                    p0 = __ffma2_rn(w0l, xl, p0); p0 = __ffma2_rn(w0h, xh, p0);
+                    p1 = __ffma2_rn(w1l, xl, p1); p1 = __ffma2_rn(w1h, xh, p1);
                 }
-                if (FMT == MOE_W_INT4) { a0 = fmaf(s0, p0, a0); a1 = fmaf(s1, p1, a1); }
-                else { a0 += p0; a1 += p1; }
+                const float r0 = p0.x + p0.y, r1 = p1.x + p1.y;
+                if (FMT == MOE_W_INT4) { a0 = fmaf(s0, r0, a0); a1 = fmaf(s1, r1, a1); }
+                else { a0 += r0; a1 += r1; }
             }
         }
         if ((st + 1) % P == 0) {  // the unit's last pass: reduce over the group, write

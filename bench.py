@@ -266,8 +266,11 @@ class Runner:
         li = i % len(self.layers)
         L = self.layers[li]
         _, _, lg, x = self.batches[i % len(self.batches)]
-        _, _, counts, offsets, sr, rp = moe.moe_route_permute(lg, self.k, hits=self.hits[li], ids_w=(self.ids, self.w),
-                                                              out=self.perm)
+        # the routing and the FFN as separate calls, so that the FFN's event pair
+        # times the FFN alone (moe_route_ffn, which the stacks use, would run a
+        # one-token step's routing inside the FFN's first launch)
+        _, _, counts, offsets, sr, rp = moe.moe_route_permute(lg, self.k, hits=self.hits[li],
+                                                              ids_w=(self.ids, self.w), out=self.perm)
         if ffn_events is not None:
             self._mark(ffn_events[0])
         moe.moe_grouped_ffn(L, x, self.k, counts, offsets, sr, rows=self.rows, ws=self.ws, path=self.path)
@@ -310,12 +313,22 @@ FFN_SAMPLE_EVERY = 1
 
 # tokens up to which moe_route_permute is one launch
 FUSED_MAX_T = 16
+ROUTE_IN_FFN_MAX_E = 128  # moe_route_ffn routes inside the one-token FFN launches up to this E
 
 
-def launches_per_layer(moe, T, k, fmt, path):
+def routes_in_ffn(moe, T, k, fmt, E, path):
+    """Whether moe_route_ffn runs the routing inside the FFN's launches: one token,
+    E <= ROUTE_IN_FFN_MAX_E, the AUTO path taking the GEMV kernels."""
+    return T == 1 and E <= ROUTE_IN_FFN_MAX_E and path == moe.MOE_FFN_AUTO and T * k < TC_MIN_ROUTES[fmt]
+
+
+def launches_per_layer(moe, T, k, fmt, path, E=None):
+    """Our launches per layer step; E given: the step calls moe_route_ffn, whose
+    one-token steps route inside the FFN's launches (no routing launch)."""
     auto_tc = T * k >= TC_MIN_ROUTES[fmt]
     tc = path == moe.MOE_FFN_TC or (path == moe.MOE_FFN_AUTO and auto_tc)
-    return (1 if T <= FUSED_MAX_T else 2) + (3 if tc else 2) + 1
+    route = 0 if E is not None and routes_in_ffn(moe, T, k, fmt, E, path) else (1 if T <= FUSED_MAX_T else 2)
+    return route + (3 if tc else 2) + 1
 
 
 def _capture(torch, runner, first, n):
@@ -1026,8 +1039,13 @@ def stack_steps(torch, moe, stack, T, k, steps, warmup, seed, refresh_every=8, p
         x = x_stage[j]
         for l in range(L):
             lay = stack.layers[l]
-            moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if with_hits else None, ids_w=(ids, w), out=perm)
-            moe.moe_grouped_ffn(lay, x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
+            if path == moe.MOE_FFN_AUTO:  # for one token the routing runs inside the FFN's launches
+                moe.moe_route_ffn(lay, lg_stage[j, l], x, k, hits=hits[l] if with_hits else None, ids_w=(ids, w),
+                                  out=perm, rows=rows, ws=ws)
+            else:
+                moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if with_hits else None, ids_w=(ids, w),
+                                      out=perm)
+                moe.moe_grouped_ffn(lay, x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
             y = ybuf[l & 1]
             moe.moe_combine(rows, perm[3], w, y)
             x = y
@@ -1125,8 +1143,12 @@ def stack_steps_device(torch, moe, stack, T, k, steps, warmup, seed, refresh_eve
     side = torch.cuda.Stream(dev)
 
     def layer(j, l, x):
-        moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if j == 0 else None, ids_w=(ids, w), out=perm)
-        moe.moe_grouped_ffn(stack.layers[l], x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
+        if path == moe.MOE_FFN_AUTO:  # for one token the routing runs inside the FFN's launches
+            moe.moe_route_ffn(stack.layers[l], lg_stage[j, l], x, k, hits=hits[l] if j == 0 else None,
+                              ids_w=(ids, w), out=perm, rows=rows, ws=ws)
+        else:
+            moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if j == 0 else None, ids_w=(ids, w), out=perm)
+            moe.moe_grouped_ffn(stack.layers[l], x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
         y = ybuf[l & 1]
         moe.moe_combine(rows, perm[3], w, y)
         return y
@@ -1247,7 +1269,7 @@ def stack_main(args, T, E, H, I, k, world, rank, local):
                       "routes_on_resident_slots": round(sum(share) / len(share), 4) if share else None},
         "sweep": sweep,
         "hbm_peak_gbs": hbm_peak,
-        "gpu_launches": steps_done * L * launches_per_layer(moe, T, k, s4.fmt, path)
+        "gpu_launches": steps_done * L * launches_per_layer(moe, T, k, s4.fmt, path, s4.E)
                         + (steps_done // 8) * L * (2 if device_refresh else 0),
         "clocks": clk,
     }

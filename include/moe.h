@@ -238,6 +238,25 @@ MOE_API moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *
                                 int32_t path, moe_stream_t stream);
 
 /*
+ * moe_route_permute followed by moe_grouped_ffn (AUTO path), with the arguments
+ * of both (T, k and E from the layer; ws sized by moe_grouped_ffn_workspace())
+ * and the same results: ids, w, counts, offsets, sorted_route, route_pos and hits
+ * bit for bit, rows bit for bit as moe_grouped_ffn's.  For one token (T == 1,
+ * E <= 128) where AUTO takes the GEMV kernels (k below 24 / 32 / 40 for bf16 /
+ * int8 / int4) the routing runs inside the FFN's two launches
+ * instead of a launch of its own: every CTA takes the token's top-k from the
+ * logits with the routing kernels' code and groups the k routes itself, and
+ * CTA 0 of the first launch writes the routing outputs (one launch fewer per
+ * one-token layer step).  Otherwise the two calls run as they are.  The stages
+ * of the pages' layer (prain README's route -> permute -> FFN; remote_experts.cpp
+ * RemoteExperts::begin) are unchanged; only where they run differs.
+ */
+MOE_API moe_status moe_route_ffn(const moe_layer *layer, const float *logits, const uint16_t *x, int32_t T,
+                                 int32_t k, uint32_t *hits, int32_t *ids, float *w, int32_t *counts,
+                                 int32_t *offsets, int32_t *sorted_route, int32_t *route_pos, float *rows,
+                                 void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Grouped FFN without a caller-provided workspace, for callers that cannot
  * allocate device memory (a plugin or serving runtime that passes the library
  * only its input and output buffers, or a loop that must never call
@@ -274,7 +293,8 @@ MOE_API moe_status moe_combine(const float *rows, const int32_t *route_pos, cons
 
 /*
  * The whole layer in one call: route -> permute (+hits) -> grouped FFN ->
- * combine.  logits fp32 [T][E], x bf16 [T][H] -> y bf16 [T][H].  hits
+ * combine (moe_route_ffn, then moe_combine).  logits fp32 [T][E], x bf16
+ * [T][H] -> y bf16 [T][H].  hits
  * (uint32 [E]), ids_out (int32 [T][k]) and w_out (fp32 [T][k]) are nullable.
  * ws: at least moe_layer_forward_workspace() bytes.
  */

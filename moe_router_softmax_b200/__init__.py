@@ -33,7 +33,7 @@ FMT = {"bf16": MOE_W_BF16, "int8": MOE_W_INT8, "int4": MOE_W_INT4}
 # every symbol include/moe.h declares
 EXPORTS = [
     "moe_version", "moe_last_error", "moe_expert_bytes", "moe_blob_offsets", "moe_route_topk", "moe_permute",
-    "moe_route_permute",
+    "moe_route_permute", "moe_route_ffn",
     "moe_expert_hits", "moe_grouped_ffn_workspace", "moe_grouped_ffn", "moe_grouped_ffn_path", "moe_combine",
     "moe_layer_forward_workspace", "moe_layer_forward", "moe_quantize_int8", "moe_quantize_int4",
     "moe_pack_expert", "moe_copy_to_slots", "moe_refresh_target", "moe_apply_placement",
@@ -67,6 +67,7 @@ _SIG = {
     "moe_route_topk": (i32, [P, i32, i32, i32, P, P, P]),
     "moe_permute": (i32, [P, i32, i32, i32, P, P, P, P, P, P]),
     "moe_route_permute": (i32, [P, i32, i32, i32, P, P, P, P, P, P, P, P]),
+    "moe_route_ffn": (i32, [LP, P, P, i32, i32, P, P, P, P, P, P, P, P, P, sz, P]),
     "moe_expert_hits": (i32, [P, i64, i32, P, P]),
     "moe_grouped_ffn_workspace": (sz, [LP, i32, i32]),
     "moe_grouped_ffn": (i32, [LP, P, i32, i32, P, P, P, P, P, sz, P]),
@@ -243,7 +244,7 @@ def moe_permute(ids: torch.Tensor, E: int, hits: torch.Tensor | None = None, out
 
 def moe_route_permute(logits: torch.Tensor, k: int, hits: torch.Tensor | None = None, ids_w=None, out=None,
                       stream=None):
-    """moe_route_topk then moe_permute in one call (one launch for T*k <= 256).
+    """moe_route_topk then moe_permute in one call (one launch for T <= 16).
     Returns (ids, w, counts, offsets, sorted_route, route_pos)."""
     T, E = logits.shape
     R = T * k
@@ -288,6 +289,36 @@ def moe_grouped_ffn(layer: MoeLayer, x: torch.Tensor, k: int, counts, offsets, s
                                      _dev(sorted_route, torch.int32, "sorted_route"), _dev(rows, torch.float32, "rows"),
                                      _dev(ws, torch.uint8, "ws"), ws.numel(), int(path), _stream(stream)))
     return rows
+
+
+def moe_route_ffn(layer: MoeLayer, logits: torch.Tensor, x: torch.Tensor, k: int, hits: torch.Tensor | None = None,
+                  ids_w=None, out=None, rows: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                  stream=None):
+    """moe_route_permute then moe_grouped_ffn in one call (for one token the
+    routing runs inside the FFN's launches).  Returns (ids, w, counts, offsets,
+    sorted_route, route_pos, rows)."""
+    T, E = logits.shape
+    R = T * k
+    dev = logits.device
+    ids, w = ids_w if ids_w is not None else (torch.empty((T, k), dtype=torch.int32, device=dev),
+                                              torch.empty((T, k), dtype=torch.float32, device=dev))
+    if out is None:
+        out = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int32, device=dev),
+               torch.empty(max(R, 1), dtype=torch.int32, device=dev)[:R],
+               torch.empty(max(R, 1), dtype=torch.int32, device=dev)[:R])
+    counts, offsets, sorted_route, route_pos = out
+    if rows is None:
+        rows = torch.empty((max(R, 1), layer.H), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty(max(moe_grouped_ffn_workspace(layer, T, k), 16), dtype=torch.uint8, device=dev)
+    _check(_lib.moe_route_ffn(layer.ref(), _dev(logits, torch.float32, "logits"), _dev(x, BF16, "x"), T, k,
+                              None if hits is None else _dev(hits, (torch.int32, torch.uint32), "hits"),
+                              _dev(ids, torch.int32, "ids"), _dev(w, torch.float32, "w"),
+                              _dev(counts, torch.int32, "counts"), _dev(offsets, torch.int32, "offsets"),
+                              _dev(sorted_route, torch.int32, "sorted_route"),
+                              _dev(route_pos, torch.int32, "route_pos"), _dev(rows, torch.float32, "rows"),
+                              _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+    return ids, w, counts, offsets, sorted_route, route_pos, rows
 
 
 def moe_combine(rows: torch.Tensor, route_pos: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None,

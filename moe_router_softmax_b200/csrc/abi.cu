@@ -27,6 +27,10 @@ cudaError_t launch_combine(const float *, const int32_t *, const float *, int, i
 cudaError_t launch_quantize_int8(const uint16_t *, int, int, int8_t *, float *, cudaStream_t);
 cudaError_t launch_quantize_int4(const uint16_t *, int, int, uint8_t *, uint16_t *, cudaStream_t);
 size_t ffn_gemv_workspace(int T, int k, int I);
+bool ffn_gemv_can_route(const LayerView &L, int T, int k);
+cudaError_t launch_ffn_gemv_routed(const LayerView &L, const uint16_t *x, const float *logits, int k,
+                                   uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
+                                   int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws, cudaStream_t s);
 cudaError_t launch_ffn_gemv(const LayerView &, const uint16_t *, int, int, const int32_t *, const int32_t *,
                             const int32_t *, float *, void *, cudaStream_t);
 size_t ffn_tc_workspace(int T, int k, int E, int H, int I);
@@ -232,6 +236,16 @@ size_t moe_grouped_ffn_workspace(const moe_layer *layer, int32_t T, int32_t k) {
     return align256(a > b ? a : b);
 }
 
+// The kernel path MOE_FFN_AUTO takes.  Measured on B200 (Gemma-shaped layer,
+// top-8, FFN alone): the tensor-core kernels win from 3 tokens for bf16 (56.9 vs
+// 61.9 us; at 2 tokens the GEMV: 44.4 vs 51.0), from 4 for int8 (63.2 vs 67.5)
+// and from about 5 for int4 (6 tokens: 90.8 vs 98.1); one token at top-8 stays
+// on the GEMV.
+static int auto_path(const LayerView &v, int T, int k) {
+    const int min_routes = v.fmt == MOE_W_BF16 ? 24 : (v.fmt == MOE_W_INT8 ? 32 : 40);
+    return (T * k >= min_routes && ffn_tc_supports(v.fmt, v.H, v.I, v.stride)) ? MOE_FFN_TC : MOE_FFN_GEMV;
+}
+
 moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *x, int32_t T, int32_t k,
                                 const int32_t *counts, const int32_t *offsets, const int32_t *sorted_route,
                                 float *rows, void *ws, size_t ws_bytes, int32_t path, moe_stream_t stream) {
@@ -244,16 +258,7 @@ moe_status moe_grouped_ffn_path(const moe_layer *layer, const uint16_t *x, int32
     if (T == 0) return MOE_OK;
     CHECK_ARG(x && counts && offsets && sorted_route && rows && ws, "moe_grouped_ffn: NULL pointer");
     CHECK_ARG(aligned16(x) && aligned16(rows) && aligned16(ws), "x, rows and ws must be 16-byte aligned");
-    const int R = T * k;
-    int use = path;
-    if (use == MOE_FFN_AUTO) {
-        // measured on B200 (Gemma-shaped layer, top-8, FFN alone): the
-        // tensor-core kernels win from 3 tokens for bf16 (56.9 vs 61.9 us; at 2
-        // tokens the GEMV: 44.4 vs 51.0), from 4 for int8 (63.2 vs 67.5) and from
-        // about 5 for int4 (6 tokens: 90.8 vs 98.1); one token stays on the GEMV
-        const int min_routes = v.fmt == MOE_W_BF16 ? 24 : (v.fmt == MOE_W_INT8 ? 32 : 40);
-        use = (R >= min_routes && ffn_tc_supports(v.fmt, v.H, v.I, v.stride)) ? MOE_FFN_TC : MOE_FFN_GEMV;
-    }
+    const int use = path == MOE_FFN_AUTO ? auto_path(v, T, k) : path;
     if (use == MOE_FFN_TC && !ffn_tc_supports(v.fmt, v.H, v.I, v.stride))
         return set_error(MOE_ERR_UNSUPPORTED, "tensor-core path does not handle format %d at H=%d I=%d stride=%llu",
                          v.fmt, v.H, v.I, (unsigned long long)v.stride);
@@ -273,6 +278,32 @@ moe_status moe_grouped_ffn(const moe_layer *layer, const uint16_t *x, int32_t T,
                            size_t ws_bytes, moe_stream_t stream) {
     return moe_grouped_ffn_path(layer, x, T, k, counts, offsets, sorted_route, rows, ws, ws_bytes, MOE_FFN_AUTO,
                                 stream);
+}
+
+moe_status moe_route_ffn(const moe_layer *layer, const float *logits, const uint16_t *x, int32_t T, int32_t k,
+                         uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
+                         int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+    LayerView v;
+    moe_status st = layer_view(layer, &v);
+    if (st != MOE_OK) return st;
+    if ((st = check_shape(v.E, k, v.H, v.I)) != MOE_OK) return st;
+    if ((st = check_tk(T, k)) != MOE_OK) return st;
+    if (T != 1 || auto_path(v, T, k) != MOE_FFN_GEMV || !ffn_gemv_can_route(v, T, k)) {
+        // the two calls (moe_route_permute checks its own arguments)
+        if ((st = moe_route_permute(logits, T, v.E, k, ids, w, counts, offsets, sorted_route, route_pos, hits,
+                                    stream)) != MOE_OK)
+            return st;
+        return moe_grouped_ffn(layer, x, T, k, counts, offsets, sorted_route, rows, ws, ws_bytes, stream);
+    }
+    CHECK_ARG(logits && x && ids && w && counts && offsets && sorted_route && route_pos && rows && ws,
+              "moe_route_ffn: NULL pointer");
+    CHECK_ARG(aligned16(x) && aligned16(rows) && aligned16(ws), "x, rows and ws must be 16-byte aligned");
+    const size_t need = align256(ffn_gemv_workspace(T, k, v.I));
+    CHECK_ARG(ws_bytes >= need, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    return cuda_status(launch_ffn_gemv_routed(v, x, logits, k, hits, ids, w, counts, offsets, sorted_route, route_pos,
+                                              rows, ws, (cudaStream_t)stream),
+                       "moe_route_ffn launch");
 }
 
 moe_status moe_combine(const float *rows, const int32_t *route_pos, const float *w, int32_t T, int32_t k, int32_t H,
@@ -334,10 +365,8 @@ moe_status moe_layer_forward(const moe_layer *layer, const float *logits, const 
     int32_t *sorted = reinterpret_cast<int32_t *>(base + f.sorted);
     int32_t *pos = reinterpret_cast<int32_t *>(base + f.pos);
     float *rows = reinterpret_cast<float *>(base + f.rows);
-    if ((st = moe_route_permute(logits, T, v.E, k, ids, w, counts, offsets, sorted, pos, hits, stream)) != MOE_OK)
-        return st;
-    if ((st = moe_grouped_ffn(layer, x, T, k, counts, offsets, sorted, rows, base + f.ffn, ws_bytes - f.ffn, stream)) !=
-        MOE_OK)
+    if ((st = moe_route_ffn(layer, logits, x, T, k, hits, ids, w, counts, offsets, sorted, pos, rows, base + f.ffn,
+                            ws_bytes - f.ffn, stream)) != MOE_OK)
         return st;
     return moe_combine(rows, pos, w, T, k, v.H, y, stream);
 }

@@ -30,6 +30,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -50,6 +51,14 @@ struct FfnParams {
     unsigned n_all, n_warps;
     double inv_warps;
     float inv_units;
+    // one-token kernels that route the token themselves (logits != nullptr):
+    // its router logits [E], and the routing outputs that CTA 0 of phase 1
+    // writes (those of moe_route_permute; counts, offsets and sorted_route then
+    // point at the caller's buffers, which the kernels do not read)
+    const float *logits;
+    uint32_t *hits;
+    int32_t *ids_out, *counts_out, *offsets_out, *sorted_out, *pos_out;
+    float *w_out;
 };
 
 namespace {
@@ -476,7 +485,88 @@ __device__ __forceinline__ unsigned div_u32(unsigned a, unsigned b, double inv_b
     return q;
 }
 
-template <int FMT, int PHASE, int C>
+// The one token's routing inside a one-token kernel (E <= 128): warp 0 takes
+// the top-k of the logits (topk::route_token_warp, the routing kernels' code)
+// while the other threads read the slot table; then route r, in lane r, goes to
+// sorted position (routes of lower experts) + (routes of its expert before it),
+// the stable grouping of moe_permute, and each sorted position gets its expert's
+// blob.  With `write` (CTA 0 of phase 1) warp 0 also stores the routing outputs
+// and adds the counts to the hit counters (read before the logits arrive).
+__device__ __forceinline__ void tok_route(const FfnParams &p, bool write, int *s_exp, const uint8_t **s_blob) {
+    constexpr int VPL = 4;  // E <= 128
+    __shared__ int32_t s_rid[kMaxK];
+    __shared__ float s_rw[kMaxK];
+    __shared__ int s_slot[128];
+    const int E = p.L.E, k = p.k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t hv[VPL];
+    if (warp == 0) {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = lane * VPL + i;
+            hv[i] = (write && p.hits != nullptr && e < E) ? p.hits[e] : 0u;
+        }
+        const float *l = p.logits;
+        topk::route_token_warp<VPL>([l](int e) { return __ldg(l + e); }, E, k, s_rid, s_rw);
+    } else if (threadIdx.x - 32 < E) {
+        const int e = threadIdx.x - 32;
+        s_slot[e] = p.L.slot_table ? __ldg(p.L.slot_table + e) : -1;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int er = lane < k ? s_rid[lane] : -1;
+        int lower = 0, same_before = 0;
+        int c[VPL];
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) c[i] = 0;
+        for (int r = 0; r < k; ++r) {
+            const int e = __shfl_sync(0xffffffffu, er, r);
+            lower += (e < er);
+            same_before += (r < lane && e == er);
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) c[i] += (e == lane * VPL + i);
+        }
+        if (lane < k) {
+            const int pos = lower + same_before;
+            const int sl = s_slot[er];
+            const bool bad = p.L.slot_table != nullptr && sl >= p.L.pool_slots;
+            s_exp[pos] = er;
+            s_blob[pos] = bad ? nullptr : (sl >= 0 ? p.L.pool + (uint64_t)sl * p.L.stride : p.L.home + (uint64_t)er * p.L.stride);
+            if (write) {
+                p.ids_out[lane] = er;
+                p.w_out[lane] = s_rw[lane];
+                p.pos_out[lane] = pos;
+                p.sorted_out[pos] = lane;
+            }
+        }
+        if (write) {
+            int sum = 0;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) sum += c[i];
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            int run = incl - sum;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int e = lane * VPL + i;
+                if (e < E) {
+                    p.counts_out[e] = c[i];
+                    p.offsets_out[e] = run;
+                    if (p.hits) p.hits[e] = hv[i] + (uint32_t)c[i];
+                }
+                run += c[i];
+            }
+            if (lane == 0) p.offsets_out[E] = k;
+        }
+    }
+    __syncthreads();
+}
+
+template <int FMT, int PHASE, int C, bool ROUTE>
 __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     constexpr int EC = Fmt<FMT>::kElems, SP = EC / 4;
     extern __shared__ __align__(16) float xs[];
@@ -497,9 +587,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     const int w_u0 = warp_start(blockIdx.x * kWarps + warp), w_u1 = warp_start(blockIdx.x * kWarps + warp + 1);
     const int trips = (w_u1 - w_u0 + gpw - 1) / gpw;
     const int c_u0 = warp_start(blockIdx.x * kWarps), c_u1 = warp_start((blockIdx.x + 1) * kWarps);
-    if (c_u1 == c_u0) return;  // no units (fewer units than warps); exiting also releases dependents
-    const int s_lo = div_small(c_u0, n_units, p.inv_units);
-    const int s_hi = div_small(c_u1 - 1, n_units, p.inv_units);
+    // a CTA without units (fewer units than warps) exits at once, which also
+    // releases dependents -- unless it is the CTA that writes the routing
+    const bool writer = ROUTE && PHASE == 1 && blockIdx.x == 0;
+    if (c_u1 == c_u0 && !writer) return;
+    const int s_lo = c_u1 > c_u0 ? div_small(c_u0, n_units, p.inv_units) : 0;
+    const int s_hi = c_u1 > c_u0 ? div_small(c_u1 - 1, n_units, p.inv_units) : 0;
     if ((PHASE == 1 ? 1 : s_hi - s_lo + 1) * K > p.xs_floats) {
         // cannot happen with the host's sizing (same for every thread of the CTA)
         if (threadIdx.x == 0) record_gemv_error(0x2007u, (unsigned)(s_hi - s_lo + 1));
@@ -514,20 +607,28 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     // as phase 1 has started and waits for h further down
     if (PHASE == 1) pdl_wait();
     pdl_launch_dependents();
-    // expert and blob of every sorted route (sorted position sr lies in
-    // [offsets[e], offsets[e+1]); the slot-table entry is read in the same round
-    // of loads as the offsets), and the number of routes: offsets[E], which is
-    // below k when the permutation dropped invalid ids
-    if (threadIdx.x == 0) s_nroutes = min(__ldg(p.offsets + p.L.E), p.k);
-    for (int e = threadIdx.x; e < p.L.E; e += kThreads) {
-        const int lo = __ldg(p.offsets + e), hi = min(__ldg(p.offsets + e + 1), p.k);
-        const uint8_t *blob = expert_blob(p.L, e);
-        for (int sr = lo; sr < hi; ++sr) {
-            s_exp[sr] = e;
-            s_blob[sr] = blob;
+    if (ROUTE) {
+        // the kernel routes the token itself: all k routes are valid
+        tok_route(p, writer, s_exp, s_blob);
+        if (c_u1 == c_u0) return;  // the writer without units of its own
+        if (threadIdx.x == 0) s_nroutes = p.k;
+        __syncthreads();
+    } else {
+        // expert and blob of every sorted route (sorted position sr lies in
+        // [offsets[e], offsets[e+1]); the slot-table entry is read in the same
+        // round of loads as the offsets), and the number of routes: offsets[E],
+        // which is below k when the permutation dropped invalid ids
+        if (threadIdx.x == 0) s_nroutes = min(__ldg(p.offsets + p.L.E), p.k);
+        for (int e = threadIdx.x; e < p.L.E; e += kThreads) {
+            const int lo = __ldg(p.offsets + e), hi = min(__ldg(p.offsets + e + 1), p.k);
+            const uint8_t *blob = expert_blob(p.L, e);
+            for (int sr = lo; sr < hi; ++sr) {
+                s_exp[sr] = e;
+                s_blob[sr] = blob;
+            }
         }
+        __syncthreads();
     }
-    __syncthreads();
     const int R = s_nroutes;
     const uint64_t qoff = PHASE == 1 ? p.L.off.q13 : p.L.off.q2;
     const uint64_t soff = PHASE == 1 ? p.L.off.s13 : p.L.off.s2;
@@ -711,7 +812,17 @@ size_t tok_xs_floats(const FfnParams &p, int phase, int n_sm) {
     return (size_t)span * p.L.I;
 }
 
-template <int FMT, int PHASE, int C>
+// The one-token kernels take the call: T = 1, a CTA's activations fit in shared
+// memory beside a second CTA, and w * N stays below 2^32 for every warp w (at up
+// to 8 CTAs per SM).
+bool tok_fits(const FfnParams &p, int n_sm) {
+    const unsigned long long max_units = (unsigned long long)p.k * std::max(p.L.I, (p.L.H + 1) / 2);
+    return p.T == 1 && p.k <= kMaxK && tok_xs_floats(p, 1, n_sm) * 4 <= kTokSmemMax &&
+           tok_xs_floats(p, 2, n_sm) * 4 <= kTokSmemMax &&
+           max_units * (unsigned long long)(n_sm * 8 * kWarps) < (1ull << 32);
+}
+
+template <int FMT, int PHASE, int C, bool ROUTE>
 cudaError_t launch_tok(const FfnParams &p0, int n_sm, cudaStream_t s) {
     FfnParams p = p0;
     const int nchunks = (PHASE == 1 ? p.L.H : p.L.I) / Fmt<FMT>::kElems;
@@ -723,7 +834,7 @@ cudaError_t launch_tok(const FfnParams &p0, int n_sm, cudaStream_t s) {
     const int n_units = PHASE == 1 ? p.L.I : (p.L.H + 1) / 2;
     p.inv_units = 1.0f / (float)n_units;
     const size_t smem = (size_t)p.xs_floats * sizeof(float);
-    auto kern = k_ffn_gemv_tok<FMT, PHASE, C>;
+    auto kern = k_ffn_gemv_tok<FMT, PHASE, C, ROUTE>;
     static size_t cached_smem[kMaxDevices] = {};
     static int cached_per_sm[kMaxDevices] = {};
     int dev = 0;
@@ -752,19 +863,19 @@ cudaError_t launch_fmt(const FfnParams &p, int n_sm, cudaStream_t s) {
     // of each row in flight, so a lane keeps 8 x 16 bytes of weights in flight
     constexpr int RWP = 2;
     constexpr int U = 8 / RWP;
-    // one token: the streaming kernels above, while a CTA's activations fit in
-    // shared memory beside a second CTA (at H = 2816, I = 704: 11 KiB in phase 1,
-    // 5.5 KiB in phase 2); chunks per lane and row in each pass: 6 (4 for int4,
-    // whose scales take registers too)
-    // (and while w * N stays below 2^32 for every warp w, at up to 8 CTAs per SM)
-    const unsigned long long max_units = (unsigned long long)p.k * std::max(p.L.I, (p.L.H + 1) / 2);
-    if (p.T == 1 && p.k <= kMaxK && tok_xs_floats(p, 1, n_sm) * 4 <= kTokSmemMax &&
-        tok_xs_floats(p, 2, n_sm) * 4 <= kTokSmemMax &&
-        max_units * (unsigned long long)(n_sm * 8 * kWarps) < (1ull << 32)) {
+    // one token: the streaming kernels above when tok_fits (at H = 2816, I = 704
+    // the activations take 11 KiB in phase 1, 5.5 KiB in phase 2); chunks per lane
+    // and row in each pass: 6 (4 for int4, whose scales take registers too)
+    if (tok_fits(p, n_sm)) {
         constexpr int C = FMT == MOE_W_INT4 ? 4 : 6;
-        cudaError_t err = launch_tok<FMT, 1, C>(p, n_sm, s);
+        if (p.logits != nullptr) {
+            cudaError_t err = launch_tok<FMT, 1, C, true>(p, n_sm, s);
+            if (err != cudaSuccess) return err;
+            return launch_tok<FMT, 2, C, true>(p, n_sm, s);
+        }
+        cudaError_t err = launch_tok<FMT, 1, C, false>(p, n_sm, s);
         if (err != cudaSuccess) return err;
-        return launch_tok<FMT, 2, C>(p, n_sm, s);
+        return launch_tok<FMT, 2, C, false>(p, n_sm, s);
     }
     cudaError_t err = launch_phase<FMT, 1, RWP, U>(p, n_sm, s);
     if (err != cudaSuccess) return err;
@@ -782,6 +893,46 @@ cudaError_t gemv_take_error(unsigned *code, unsigned *info) {
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv_error, &zero, sizeof(unsigned));
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv_error_info, &zero, sizeof(unsigned));
     return e;
+}
+
+bool ffn_gemv_can_route(const LayerView &L, int T, int k) {
+    int n_sm = 0;
+    if (sm_count(&n_sm) != cudaSuccess) return false;
+    FfnParams p{};
+    p.L = L;
+    p.T = T;
+    p.k = k;
+    return T == 1 && L.E <= 128 && tok_fits(p, n_sm);
+}
+
+cudaError_t launch_ffn_gemv_routed(const LayerView &L, const uint16_t *x, const float *logits, int k,
+                                   uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
+                                   int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws,
+                                   cudaStream_t s) {
+    int n_sm = 0;
+    cudaError_t err = sm_count(&n_sm);
+    if (err != cudaSuccess) return err;
+    FfnParams p{};
+    p.L = L;
+    p.x = x;
+    p.T = 1;
+    p.k = k;
+    p.counts = counts;
+    p.offsets = offsets;
+    p.sorted_route = sorted_route;
+    p.h = static_cast<uint16_t *>(ws);
+    p.rows = rows;
+    p.logits = logits;
+    p.hits = hits;
+    p.ids_out = ids;
+    p.w_out = w;
+    p.counts_out = counts;
+    p.offsets_out = offsets;
+    p.sorted_out = sorted_route;
+    p.pos_out = route_pos;
+    if (L.fmt == MOE_W_BF16) return launch_fmt<MOE_W_BF16>(p, n_sm, s);
+    if (L.fmt == MOE_W_INT8) return launch_fmt<MOE_W_INT8>(p, n_sm, s);
+    return launch_fmt<MOE_W_INT4>(p, n_sm, s);
 }
 
 cudaError_t launch_ffn_gemv(const LayerView &L, const uint16_t *x, int T, int k, const int32_t *counts,

@@ -105,6 +105,62 @@ def test_route_permute_matches_the_oracle_and_the_two_calls(T, E, k, kind):
     assert np.array_equal(h_one.cpu().numpy().view(np.uint32), oracle.hits(oi, E, hits0))
 
 
+# moe_route_ffn: one token with E <= 128 routes inside the one-token FFN launches
+# (the first six cases, E up to 128, k up to 8); E = 200 and T = 5 take the two calls
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("T,E,H,I,k", [(1, 128, 256, 128, 8), (1, 8, 256, 128, 6), (1, 12, 2816, 704, 8),
+                                       (1, 6, 1024, 320, 4), (1, 4, 64, 64, 1), (1, 33, 512, 192, 32),
+                                       (1, 200, 256, 128, 8), (5, 16, 512, 192, 3)])
+def test_route_ffn_matches_the_two_calls_and_the_oracle(fmt, T, E, H, I, k):
+    w13, w2 = syn.expert_weights(E, H, I, seed=E + H + k)
+    L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
+    x = syn.activations(T, H, seed=H + 1)
+    lg = syn.router_logits(T, E, "normal", seed=E * 3 + k)
+    rng = np.random.default_rng(E + k)
+    hits0 = rng.integers(0, 50, size=E).astype(np.uint32)
+    h_one = torch.from_numpy(hits0.view(np.int32)).to(DEV)
+    h_two = torch.from_numpy(hits0.view(np.int32)).to(DEV)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    d_lg = torch.from_numpy(lg).to(DEV)
+    one = moe.moe_route_ffn(L, d_lg, xd, k, hits=h_one)
+    two = moe.moe_route_permute(d_lg, k, hits=h_two)
+    rows2 = moe.moe_grouped_ffn(L, xd, k, two[2], two[3], two[4])
+    assert moe.moe_take_device_errors() == (0, 0)
+    for a, b in zip(one[:6], two):
+        assert np.array_equal(a.cpu().numpy().view(np.uint32), b.cpu().numpy().view(np.uint32))
+    assert np.array_equal(h_one.cpu().numpy(), h_two.cpu().numpy())
+    R = T * k
+    assert np.array_equal(one[6][:R].cpu().numpy().view(np.uint32), rows2[:R].cpu().numpy().view(np.uint32))
+    oi, ow = oracle.route_topk(lg, k)
+    assert np.array_equal(one[0].cpu().numpy(), oi)
+    assert bits_equal(one[1].cpu().numpy(), ow)
+    for g, r in zip(one[2:6], oracle.permute(oi, E)):
+        assert np.array_equal(g.cpu().numpy(), r)
+    assert np.array_equal(h_one.cpu().numpy().view(np.uint32), oracle.hits(oi, E, hits0))
+    orows = oracle.ffn_routes(oracle_layer_for(fmt, w13, w2), x, oi)
+    assert rel_err(one[6].cpu().numpy()[one[5].cpu().numpy().ravel()], orows) <= FFN_TOL
+
+
+@pytest.mark.parametrize("fmt", [0, 2])
+def test_route_ffn_one_token_on_a_slot_table(fmt):
+    """The one-token kernels that route for themselves resolve experts through
+    the slot table (a pool of 24 slots behind 8 experts) like the other paths."""
+    E, H, I, k = 8, 512, 192, 3
+    w13, w2 = syn.expert_weights(E, H, I, seed=77)
+    slot_of = np.array([23, -1, 17, 5, -1, 20, 0, 11], np.int32)
+    Ld, OL = _pool_layers(fmt, E, H, I, w13, w2, slot_of, 24)
+    x = syn.activations(1, H, seed=78)
+    lg = syn.router_logits(1, E, "normal", seed=91)
+    lg[0, 1] += 4.0                          # a home expert as well as pooled ones
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    ids, w, counts, offsets, sr, rp, rows = moe.moe_route_ffn(Ld, torch.from_numpy(lg).to(DEV), xd, k)
+    assert moe.moe_take_device_errors() == (0, 0)
+    oi, ow, orows, oy = oracle.moe_layer(OL, lg, x, k)
+    assert np.array_equal(ids.cpu().numpy(), oi)
+    assert (slot_of[oi] >= 0).any() and (slot_of[oi] < 0).any()
+    assert rel_err(rows.cpu().numpy()[rp.cpu().numpy().ravel()], orows) <= FFN_TOL
+
+
 @pytest.mark.parametrize("T", [30, 5])  # 5 tokens x 6 = 30 routes: the one-warp kernel
 def test_route_permute_ties_nan_inf(T):
     rng = np.random.default_rng(4)

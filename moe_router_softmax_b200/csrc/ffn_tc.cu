@@ -62,6 +62,7 @@ constexpr uint32_t kATileBytes = kBlockM * kBlockK * 2;   // 16 KB
 constexpr int kMaxBSlots = 32;
 constexpr int kRawRowBytes = 128;     // per raw stage row
 constexpr long long kWaitCycles = 4000000000ll;           // ~2 s at 2 GHz
+constexpr long long kReadySpins = 8000000ll;              // phase 2's wait for an expert's h: > 1 s of 128-ns sleeps
 constexpr int kXPitch = 17;                               // exchange row pitch (floats): no bank conflicts
 
 // Three rings of stages, each with its own full / empty mbarriers, so no
@@ -129,6 +130,10 @@ struct TcParams {
     int n_units;           // output rows of the weight: 2I (phase 1) or H (phase 2)
     uint16_t *h;           // [R][I] bf16: phase-1 output
     float *rows;           // [R][H] fp32: phase-2 output
+    // per expert, h values published by phase 1: each of an item's two gate-row
+    // epilogue warps adds the item's route count once its h entries are written,
+    // so expert e is complete at 2 * (I / 64) * counts[e]; zeroed by the gather
+    unsigned *ready;
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -140,6 +145,11 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
@@ -466,8 +476,11 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     const int m_tiles = PHASE == 1 ? p.L.I / 64 : (p.L.H + kBlockM - 1) / kBlockM;
     // The next launch (phase 2 after phase 1, the combine after phase 2) may
     // take over SMs as this grid's CTAs finish; it waits for this grid's
-    // results itself where it reads them.
-    pdl_launch_dependents();
+    // results itself where it reads them.  Phase 1 releases phase 2 only from its
+    // B producer, once the gather has completed: phase 2 reads the per-expert
+    // counters the gather zeroes.
+    constexpr bool kEarly = FMT == MOE_W_BF16;  // phase 2 starts per expert (see the B producer)
+    if (PHASE == 2 || !kEarly) pdl_launch_dependents();
     const int nk = (p.K + KS - 1) / KS;  // stages; the last may hold fewer atoms (p.K is a multiple of 64)
     auto atoms_at = [&](int kk) { return min(ATOMS, (p.K - kk * KS) / kBlockK); };
 
@@ -565,16 +578,36 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
     } else if (warp == kWarpB) {
         // ------------------------------------------------ B producer: routes
         if (lane == 0) {
-            // the B operand (xs from k_gather_rows, or h from phase 1) is the one
-            // input the previous launch writes: wait for it here, while the
-            // other roles already stream weights
-            pdl_wait();
+            // the B operand is the one input an earlier launch writes.  Phase 1
+            // (xs from k_gather_rows) waits for the gather here, while the other
+            // roles already stream weights.  Phase 2 (h) waits per item only for
+            // the phase-1 items of the item's expert, through the counters, so it
+            // starts while phase 1's last items still run elsewhere.
+            if (PHASE == 1 || !kEarly) pdl_wait();
+            if (PHASE == 1 && kEarly) pdl_launch_dependents();
             const uint64_t pol = l2_policy_last();
             int stage = 0;
             uint32_t phase = 0;
             for (int item = blockIdx.x; item < total && !s_abort; item += gridDim.x) {
                 const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
                 bool ok = true;
+                if (kEarly && PHASE == 2) {
+                    const unsigned target = 2u * (unsigned)(p.L.I / 64) * (unsigned)__ldg(p.counts + it.e);
+                    long long spins = 0;
+                    while (ld_acquire_gpu(p.ready + it.e) < target) {
+                        if (++spins > kReadySpins || s_abort) {
+                            if (!s_abort) record_error(0x1000u | (unsigned)kWarpB, (unsigned)it.e);
+                            s_abort = 1;
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                    if (!ok) break;
+                    // h was written through the generic proxy by other CTAs; the
+                    // route tiles are read by TMA (the async proxy)
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
                 // up to 32 routes: 16-row boxes; more: 64-row boxes (rows past
                 // the block are another expert's or out of range and zero-filled;
                 // the slot holds them, the MMAs read only the first n_mma)
@@ -738,6 +771,12 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                 }
             }
             if (!ok) break;
+            if (kEarly && PHASE == 1 && lrow < 64) {
+                // this warp's h entries of the item are written: publish them
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(p.ready + it.e, (unsigned)it.n);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -951,11 +990,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 // of 8 elements is stored in the order k_order<MOE_W_INT4> gives.
 __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ sorted_route,
                               const int32_t *__restrict__ offsets, int E, int k, int H, int R, int perm,
-                              uint16_t *__restrict__ xs) {
+                              uint16_t *__restrict__ xs, unsigned *__restrict__ ready) {
     // programmatic dependent launch: wait for the previous kernel before
     // touching memory, then let the next one be scheduled
     pdl_wait();
     pdl_launch_dependents();
+    // the per-expert counters of this call's phase 1 (nullable: gather only)
+    if (ready != nullptr && blockIdx.x == 0)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) ready[e] = 0u;
     const int per = H / 8;
     const int n_valid = __ldg(offsets + E);
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)R * per;
@@ -1062,10 +1104,10 @@ cudaError_t launch_one(const CUtensorMap &mh, const CUtensorMap &mp, const CUten
 }  // namespace
 
 size_t ffn_tc_workspace(int T, int k, int E, int H, int I) {
-    (void)E;
     const size_t R = (size_t)T * k;
     const size_t xs = (R * H * 2 + 255) & ~(size_t)255;
-    return xs + R * I * 2;
+    const size_t h = (R * I * 2 + 255) & ~(size_t)255;
+    return xs + h + (size_t)E * 4;  // xs | h | per-expert phase-1 counters
 }
 
 bool ffn_tc_supports(int fmt, int H, int I, uint64_t stride) {
@@ -1087,14 +1129,16 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     const int R = T * k;
     const int H = L.H, I = L.I, fmt = L.fmt;
     uint16_t *xs = static_cast<uint16_t *>(ws);
-    uint16_t *h = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + (((size_t)R * H * 2 + 255) & ~(size_t)255));
+    const size_t xs_bytes = ((size_t)R * H * 2 + 255) & ~(size_t)255, h_bytes = ((size_t)R * I * 2 + 255) & ~(size_t)255;
+    uint16_t *h = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + xs_bytes);
+    unsigned *ready = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + xs_bytes + h_bytes);
 
     // 1. activations into sorted-route order
     {
         const int64_t n = (int64_t)R * (H / 8);
         const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)n_sm * 8);
         err = launch_pdl(k_gather_rows, dim3((unsigned)blocks), dim3(256), 0, s, x, sorted_route, offsets, L.E, k, H, R,
-                         (int)(L.fmt == MOE_W_INT4), xs);
+                         (int)(L.fmt == MOE_W_INT4), xs, ready);
         if (err != cudaSuccess) return err;
     }
     // 2. tensor maps: weights (home and pool, as rows of one matrix), activations
@@ -1143,6 +1187,7 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
     p.n_block = std::min(two ? TcCfg<MOE_W_INT4, 1>::kNMax : kNMax, (std::max(T, 1) + 15) / 16 * 16);
     p.h = h;
     p.rows = rows;
+    p.ready = ready;
     // every pointer the kernels write through must be set (host-side guard)
     if (p.h == nullptr || p.rows == nullptr || p.counts == nullptr || p.offsets == nullptr || xs == nullptr)
         return cudaErrorInvalidValue;

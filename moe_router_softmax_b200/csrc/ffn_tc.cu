@@ -310,19 +310,26 @@ struct Items {
     int n_act, total, m_tiles, n_block, b_rows, b_slots;
 };
 
+// Called by every thread of the CTA (it holds a __syncthreads).  The counts are
+// read in one round of loads by the whole CTA into s_base, which warp 0 then
+// overwrites in place with the item prefix (a write at position pos <= e never
+// reaches a count not yet read: reads run ahead in e).
 __device__ void build_items(const TcParams &p, int m_tiles, int b_region, int atoms, int *s_act, int *s_base,
                             Items *it) {
     const int lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < p.L.E; e += blockDim.x) s_base[e] = __ldg(p.counts + e);
+    __syncthreads();
     if (threadIdx.x < 32) {
         int n_max = 1;
-        for (int e = lane; e < p.L.E; e += 32) n_max = max(n_max, __ldg(p.counts + e));
+        for (int e = lane; e < p.L.E; e += 32) n_max = max(n_max, s_base[e]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) n_max = max(n_max, __shfl_xor_sync(0xffffffffu, n_max, off));
         const int n_block = min(p.n_block, (n_max + 15) & ~15);
         int n_act = 0, run = 0;
         for (int e0 = 0; e0 < p.L.E; e0 += 32) {
             const int e = e0 + lane;
-            const int n = (e < p.L.E) ? __ldg(p.counts + e) : 0;
+            const int n = (e < p.L.E) ? s_base[e] : 0;
+            __syncwarp();  // every lane has read its count before any prefix is written
             const bool act = n > 0;
             const unsigned m = __ballot_sync(0xffffffffu, act);
             const int items = act ? m_tiles * ((n + n_block - 1) / n_block) : 0;

@@ -219,6 +219,18 @@ __device__ __forceinline__ uint64_t l2_policy_last() {
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+// Stores of the intermediates a later launch re-reads (xs by every M tile of
+// phase 1, h by every M tile of phase 2) with the evict-last policy, so they
+// stay in L2 beside the evict-first weight stream instead of going to DRAM
+// and back.
+__device__ __forceinline__ void st_v4_hint(void *dst, uint4 u, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "r"(u.x), "r"(u.y),
+                 "r"(u.z), "r"(u.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_u16_hint(uint16_t *dst, uint16_t v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.u16 [%0], %1, %2;" ::"l"(dst), "h"(v), "l"(pol) : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
                                             uint64_t pol) {
     asm volatile(
@@ -706,6 +718,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
         int acc = 0;
         uint32_t acc_phase = 0;
         uint32_t xcount = 0;  // exchange chunks used so far (buffer = xcount & 1)
+        const uint64_t h_pol = l2_policy_last();
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok && !s_abort; item += gridDim.x) {
             const ItemInfo it = decode_item(p, s_act, s_base, n_act, m_tiles, n_block, item);
@@ -752,8 +765,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
                                     continue;
                                 }
                                 const float g = v[i] * scale, up = xrow[i];
-                                p.h[(size_t)(it.row0 + j) * p.L.I + k_order<FMT>(icol)] =
-                                    f32_to_bf16_rne(gelu_tanh(g) * up);
+                                st_u16_hint(p.h + (size_t)(it.row0 + j) * p.L.I + k_order<FMT>(icol),
+                                            f32_to_bf16_rne(gelu_tanh(g) * up), h_pol);
                             }
                         }
                         __syncwarp();
@@ -1007,6 +1020,7 @@ __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__r
         for (int e = threadIdx.x; e < E; e += blockDim.x) ready[e] = 0u;
     const int per = H / 8;
     const int n_valid = __ldg(offsets + E);
+    const uint64_t pol = l2_policy_last();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)R * per;
          i += (int64_t)gridDim.x * blockDim.x) {
         const int s = (int)(i / per), c = (int)(i % per);
@@ -1025,7 +1039,7 @@ __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__r
             u.z = __byte_perm(v.z, v.w, 0x5410);
             u.w = __byte_perm(v.z, v.w, 0x7632);
         }
-        reinterpret_cast<uint4 *>(xs + (size_t)s * H)[c] = u;
+        st_v4_hint(reinterpret_cast<uint4 *>(xs + (size_t)s * H) + c, u, pol);
     }
 }
 

@@ -242,11 +242,13 @@ def make_batches(torch, kind, T, E, H, n, dev, seed=0):
 
 
 class Runner:
-    """Device buffers for one batch size; step(i) runs the layer on batch i."""
+    """Device buffers for one batch size; step(i) runs the layer on batch i
+    (one_call: as one moe_layer_forward call, with no FFN events)."""
 
-    def __init__(self, moe, torch, layers, batches, T, k, dev, path=0):
+    def __init__(self, moe, torch, layers, batches, T, k, dev, path=0, one_call=False):
         self.moe, self.torch, self.layers, self.batches, self.T, self.k = moe, torch, layers, batches, T, k
         self.path = path
+        self.one_call = one_call
         E, H = layers[0].E, layers[0].H
         R = T * k
         i32 = torch.int32
@@ -258,6 +260,8 @@ class Runner:
         self.rows = torch.empty((R, H), dtype=torch.float32, device=dev)
         self.ws = torch.empty(max(moe.moe_grouped_ffn_workspace(layers[0], T, k), 16), dtype=torch.uint8, device=dev)
         self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.fws = (torch.empty(moe.moe_layer_forward_workspace(layers[0], T, k), dtype=torch.uint8, device=dev)
+                    if one_call else None)
         self.ev = None
         self.side = None
 
@@ -266,6 +270,10 @@ class Runner:
         li = i % len(self.layers)
         L = self.layers[li]
         _, _, lg, x = self.batches[i % len(self.batches)]
+        if self.one_call:
+            moe.moe_layer_forward(L, lg, x, self.k, y=self.y, hits=self.hits[li], ids_out=self.ids, w_out=self.w,
+                                  ws=self.fws)
+            return
         # the routing and the FFN as separate calls, so that the FFN's event pair
         # times the FFN alone (moe_route_ffn, which the stacks use, would run a
         # one-token step's routing inside the FFN's first launch)
@@ -323,12 +331,15 @@ def routes_in_ffn(moe, T, k, fmt, E, path):
 
 
 def launches_per_layer(moe, T, k, fmt, path, E=None):
-    """Our launches per layer step; E given: the step calls moe_route_ffn, whose
-    one-token steps route inside the FFN's launches (no routing launch)."""
+    """Our launches per layer step; E given: the step calls moe_layer_forward,
+    whose one-token steps route inside the FFN's first launch and combine inside
+    its second (no routing and no combine launch; the shared-memory fit of the
+    fused combine holds at the bench's shapes)."""
     auto_tc = T * k >= TC_MIN_ROUTES[fmt]
     tc = path == moe.MOE_FFN_TC or (path == moe.MOE_FFN_AUTO and auto_tc)
-    route = 0 if E is not None and routes_in_ffn(moe, T, k, fmt, E, path) else (1 if T <= FUSED_MAX_T else 2)
-    return route + (3 if tc else 2) + 1
+    in_ffn = E is not None and routes_in_ffn(moe, T, k, fmt, E, path)
+    route = 0 if in_ffn else (1 if T <= FUSED_MAX_T else 2)
+    return route + (3 if tc else 2) + (0 if in_ffn else 1)
 
 
 def _capture(torch, runner, first, n):
@@ -339,7 +350,7 @@ def _capture(torch, runner, first, n):
     launch does, and neither cuts the programmatic-launch edges of the kernel
     chain (an event node between two kernels would)."""
     g = torch.cuda.CUDAGraph()
-    sampled = [j for j in range(n) if j % FFN_SAMPLE_EVERY == FFN_SAMPLE_EVERY // 2] or [0]
+    sampled = [] if runner.one_call else [j for j in range(n) if j % FFN_SAMPLE_EVERY == FFN_SAMPLE_EVERY // 2] or [0]
     evs = {j: (torch.cuda.Event(enable_timing=True, external=True),
                torch.cuda.Event(enable_timing=True, external=True)) for j in sampled}
     with torch.cuda.graph(g):
@@ -679,6 +690,18 @@ def run_layer_config(ctx, layers, kind, T, name, seed=0):
         "roofline": ffn_roofline(T, k, H, I, eb, d_avg, f_avg, ctx["peaks"], traffic),
         "gpu_launches": runner.launches_per_step() * args.steps,
     }
+    if T == 1 and ctx["path"] == moe.MOE_FFN_AUTO:
+        # the same steps as one moe_layer_forward call each (for one token the
+        # routing runs inside the FFN's first launch and the combine inside its
+        # second): what a caller of the one-call entry point gets per layer
+        r1 = Runner(moe, torch, layers, batches, T, k, dev, ctx["path"], one_call=True)
+        ms1, _ = time_steps(torch, r1, args.steps, args.warmup, dist)
+        ms1 = max_over_ranks(dist, ms1, dev)
+        out["one_call"] = {"tokens_per_s": round(world * T * args.steps / (ms1 / 1e3), 1),
+                           "us_per_step": round(ms1 / args.steps * 1e3, 2),
+                           "gpu_launches": launches_per_layer(moe, T, k, L0.fmt, ctx["path"], E) * args.steps,
+                           "call": "moe_layer_forward"}
+        del r1
     return out, runner, ms, batches
 
 
@@ -1035,19 +1058,23 @@ def stack_steps(torch, moe, stack, T, k, steps, warmup, seed, refresh_every=8, p
     ybuf = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     hits = torch.zeros((L, E), dtype=torch.int32, device=dev)
 
+    fws = torch.empty(moe.moe_layer_forward_workspace(stack.layers[0], T, k), dtype=torch.uint8, device=dev)
+
     def one_step(j, with_hits):
         x = x_stage[j]
         for l in range(L):
             lay = stack.layers[l]
-            if path == moe.MOE_FFN_AUTO:  # for one token the routing runs inside the FFN's launches
-                moe.moe_route_ffn(lay, lg_stage[j, l], x, k, hits=hits[l] if with_hits else None, ids_w=(ids, w),
-                                  out=perm, rows=rows, ws=ws)
+            y = ybuf[l & 1]
+            if path == moe.MOE_FFN_AUTO:
+                # the whole layer in one call: for one token the routing runs inside
+                # the FFN's launches and the combine inside its second one
+                moe.moe_layer_forward(lay, lg_stage[j, l], x, k, y=y, hits=hits[l] if with_hits else None,
+                                      ids_out=ids, w_out=w, ws=fws)
             else:
                 moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if with_hits else None, ids_w=(ids, w),
                                       out=perm)
                 moe.moe_grouped_ffn(lay, x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
-            y = ybuf[l & 1]
-            moe.moe_combine(rows, perm[3], w, y)
+                moe.moe_combine(rows, perm[3], w, y)
             x = y
 
     def window_inputs(first):
@@ -1142,15 +1169,19 @@ def stack_steps_device(torch, moe, stack, T, k, steps, warmup, seed, refresh_eve
     acc = torch.zeros(4, dtype=torch.int64, device=dev)  # promotions, demotions, resident routes, routes
     side = torch.cuda.Stream(dev)
 
+    fws = torch.empty(moe.moe_layer_forward_workspace(stack.layers[0], T, k), dtype=torch.uint8, device=dev)
+
     def layer(j, l, x):
-        if path == moe.MOE_FFN_AUTO:  # for one token the routing runs inside the FFN's launches
-            moe.moe_route_ffn(stack.layers[l], lg_stage[j, l], x, k, hits=hits[l] if j == 0 else None,
-                              ids_w=(ids, w), out=perm, rows=rows, ws=ws)
+        y = ybuf[l & 1]
+        if path == moe.MOE_FFN_AUTO:
+            # the whole layer in one call: for one token the routing runs inside
+            # the FFN's launches and the combine inside its second one
+            moe.moe_layer_forward(stack.layers[l], lg_stage[j, l], x, k, y=y, hits=hits[l] if j == 0 else None,
+                                  ids_out=ids, w_out=w, ws=fws)
         else:
             moe.moe_route_permute(lg_stage[j, l], k, hits=hits[l] if j == 0 else None, ids_w=(ids, w), out=perm)
             moe.moe_grouped_ffn(stack.layers[l], x, k, perm[0], perm[1], perm[2], rows=rows, ws=ws, path=path)
-        y = ybuf[l & 1]
-        moe.moe_combine(rows, perm[3], w, y)
+            moe.moe_combine(rows, perm[3], w, y)
         return y
 
     def window():

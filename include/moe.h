@@ -296,7 +296,13 @@ MOE_API moe_status moe_combine(const float *rows, const int32_t *route_pos, cons
  * combine (moe_route_ffn, then moe_combine).  logits fp32 [T][E], x bf16
  * [T][H] -> y bf16 [T][H].  hits
  * (uint32 [E]), ids_out (int32 [T][k]) and w_out (fp32 [T][k]) are nullable.
- * ws: at least moe_layer_forward_workspace() bytes.
+ * ws: at least moe_layer_forward_workspace() bytes.  y must be 16-byte
+ * aligned.  For one token where moe_route_ffn routes inside the FFN's launches
+ * (the GEMV path, E <= 128), the combine also runs inside the FFN's second
+ * launch: each of its CTAs takes whole output rows of all k routes, keeps those
+ * rows in shared memory and sums them into y in route order with the same fp32
+ * fma as moe_combine, so y is bit-identical to the separate calls; the call is
+ * then two launches, and the rows region of ws is left unwritten.
  */
 MOE_API size_t moe_layer_forward_workspace(const moe_layer *layer, int32_t T, int32_t k);
 MOE_API moe_status moe_layer_forward(const moe_layer *layer, const float *logits, const uint16_t *x, int32_t T,

@@ -28,9 +28,11 @@ cudaError_t launch_quantize_int8(const uint16_t *, int, int, int8_t *, float *, 
 cudaError_t launch_quantize_int4(const uint16_t *, int, int, uint8_t *, uint16_t *, cudaStream_t);
 size_t ffn_gemv_workspace(int T, int k, int I);
 bool ffn_gemv_can_route(const LayerView &L, int T, int k);
+bool ffn_gemv_can_combine(const LayerView &L, int T, int k);
 cudaError_t launch_ffn_gemv_routed(const LayerView &L, const uint16_t *x, const float *logits, int k,
                                    uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
-                                   int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws, cudaStream_t s);
+                                   int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws, uint16_t *y,
+                                   cudaStream_t s);
 cudaError_t launch_ffn_gemv(const LayerView &, const uint16_t *, int, int, const int32_t *, const int32_t *,
                             const int32_t *, float *, void *, cudaStream_t);
 size_t ffn_tc_workspace(int T, int k, int E, int H, int I);
@@ -280,10 +282,15 @@ moe_status moe_grouped_ffn(const moe_layer *layer, const uint16_t *x, int32_t T,
                                 stream);
 }
 
-moe_status moe_route_ffn(const moe_layer *layer, const float *logits, const uint16_t *x, int32_t T, int32_t k,
-                         uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
-                         int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws, size_t ws_bytes,
-                         moe_stream_t stream) {
+// moe_route_ffn; with y non-null (moe_layer_forward) a one-token call whose
+// FFN launches route the token also writes y in its second launch (the combine
+// in the same launch, bit-identical to moe_combine), says so in *combined and
+// leaves rows unwritten.
+static moe_status route_ffn(const moe_layer *layer, const float *logits, const uint16_t *x, int32_t T, int32_t k,
+                            uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
+                            int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws, size_t ws_bytes,
+                            uint16_t *y, bool *combined, moe_stream_t stream) {
+    if (combined) *combined = false;
     LayerView v;
     moe_status st = layer_view(layer, &v);
     if (st != MOE_OK) return st;
@@ -301,9 +308,20 @@ moe_status moe_route_ffn(const moe_layer *layer, const float *logits, const uint
     CHECK_ARG(aligned16(x) && aligned16(rows) && aligned16(ws), "x, rows and ws must be 16-byte aligned");
     const size_t need = align256(ffn_gemv_workspace(T, k, v.I));
     CHECK_ARG(ws_bytes >= need, "workspace %zu bytes < %zu needed", ws_bytes, need);
-    return cuda_status(launch_ffn_gemv_routed(v, x, logits, k, hits, ids, w, counts, offsets, sorted_route, route_pos,
-                                              rows, ws, (cudaStream_t)stream),
-                       "moe_route_ffn launch");
+    const bool fuse = y != nullptr && ffn_gemv_can_combine(v, T, k);
+    moe_status st2 = cuda_status(launch_ffn_gemv_routed(v, x, logits, k, hits, ids, w, counts, offsets, sorted_route,
+                                                        route_pos, rows, ws, fuse ? y : nullptr, (cudaStream_t)stream),
+                                 "moe_route_ffn launch");
+    if (st2 == MOE_OK && combined) *combined = fuse;
+    return st2;
+}
+
+moe_status moe_route_ffn(const moe_layer *layer, const float *logits, const uint16_t *x, int32_t T, int32_t k,
+                         uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
+                         int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+    return route_ffn(layer, logits, x, T, k, hits, ids, w, counts, offsets, sorted_route, route_pos, rows, ws,
+                     ws_bytes, nullptr, nullptr, stream);
 }
 
 moe_status moe_combine(const float *rows, const int32_t *route_pos, const float *w, int32_t T, int32_t k, int32_t H,
@@ -365,9 +383,12 @@ moe_status moe_layer_forward(const moe_layer *layer, const float *logits, const 
     int32_t *sorted = reinterpret_cast<int32_t *>(base + f.sorted);
     int32_t *pos = reinterpret_cast<int32_t *>(base + f.pos);
     float *rows = reinterpret_cast<float *>(base + f.rows);
-    if ((st = moe_route_ffn(layer, logits, x, T, k, hits, ids, w, counts, offsets, sorted, pos, rows, base + f.ffn,
-                            ws_bytes - f.ffn, stream)) != MOE_OK)
+    CHECK_ARG(aligned16(y), "y must be 16-byte aligned");
+    bool combined = false;
+    if ((st = route_ffn(layer, logits, x, T, k, hits, ids, w, counts, offsets, sorted, pos, rows, base + f.ffn,
+                        ws_bytes - f.ffn, y, &combined, stream)) != MOE_OK)
         return st;
+    if (combined) return MOE_OK;  // one token: the FFN's second launch wrote y
     return moe_combine(rows, pos, w, T, k, v.H, y, stream);
 }
 

@@ -59,6 +59,8 @@ struct FfnParams {
     uint32_t *hits;
     int32_t *ids_out, *counts_out, *offsets_out, *sorted_out, *pos_out;
     float *w_out;
+    // one-token phase 2 with the combine (nullable): y [1][H] bf16
+    uint16_t *y;
 };
 
 namespace {
@@ -492,7 +494,9 @@ __device__ __forceinline__ unsigned div_u32(unsigned a, unsigned b, double inv_b
 // the stable grouping of moe_permute, and each sorted position gets its expert's
 // blob.  With `write` (CTA 0 of phase 1) warp 0 also stores the routing outputs
 // and adds the counts to the hit counters (read before the logits arrive).
-__device__ __forceinline__ void tok_route(const FfnParams &p, bool write, int *s_exp, const uint8_t **s_blob) {
+// s_posj / s_wj (nullable) get each route's sorted position and weight.
+__device__ __forceinline__ void tok_route(const FfnParams &p, bool write, int *s_exp, const uint8_t **s_blob,
+                                          int *s_posj = nullptr, float *s_wj = nullptr) {
     constexpr int VPL = 4;  // E <= 128
     __shared__ int32_t s_rid[kMaxK];
     __shared__ float s_rw[kMaxK];
@@ -531,6 +535,10 @@ __device__ __forceinline__ void tok_route(const FfnParams &p, bool write, int *s
             const int sl = s_slot[er];
             const bool bad = p.L.slot_table != nullptr && sl >= p.L.pool_slots;
             s_exp[pos] = er;
+            if (s_posj != nullptr) {
+                s_posj[lane] = pos;
+                s_wj[lane] = s_rw[lane];
+            }
             s_blob[pos] = bad ? nullptr : (sl >= 0 ? p.L.pool + (uint64_t)sl * p.L.stride : p.L.home + (uint64_t)er * p.L.stride);
             if (write) {
                 p.ids_out[lane] = er;
@@ -566,13 +574,21 @@ __device__ __forceinline__ void tok_route(const FfnParams &p, bool write, int *s
     __syncthreads();
 }
 
-template <int FMT, int PHASE, int C, bool ROUTE>
+// Y (phase 2 of a routed call only): the combine of the one token in the same
+// launch.  The CTA then takes the row pairs [cp0, cp0 + np) of every route (its
+// warps split those k * np units, route-major), keeps its rows in shared memory
+// instead of writing them out, and writes y for its rows: the k terms in route
+// order with the fp32 fma of moe_combine, so y is bit-identical to the two calls.
+template <int FMT, int PHASE, int C, bool ROUTE, bool Y = false>
 __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
+    static_assert(!Y || (PHASE == 2 && ROUTE), "the fused combine is phase 2 of a routed call");
     constexpr int EC = Fmt<FMT>::kElems, SP = EC / 4;
     extern __shared__ __align__(16) float xs[];
     __shared__ int s_exp[kMaxK];
     __shared__ const uint8_t *s_blob[kMaxK];
     __shared__ int s_nroutes;
+    __shared__ int s_posj[Y ? kMaxK : 1];
+    __shared__ float s_wj[Y ? kMaxK : 1];
     const int H = p.L.H, I = p.L.I;
     const int K = PHASE == 1 ? H : I;
     const int nchunks = K / EC;
@@ -580,10 +596,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     const int lg = p.lg, gpw = 32 / lg, P = p.passes;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int li = lane & (lg - 1), gi = lane / lg;
-    // the warp's units (all k routes' units split evenly over the grid's warps;
-    // units of routes the permutation left empty are skipped below) and the
-    // routes whose activations the CTA reads: no device data needed yet
-    auto warp_start = [&](unsigned w) { return (int)div_u32(w * p.n_all, p.n_warps, p.inv_warps); };
+    // Y: the CTA's row pairs (one integer division per thread, at set-up)
+    const int cp0 = Y ? (int)((long long)blockIdx.x * n_units / gridDim.x) : 0;
+    const int np = Y ? (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x) - cp0 : n_units;
+    // the warp's units (all k routes' units split evenly over the grid's warps,
+    // or for Y the CTA's k * np units over its warps; units of routes the
+    // permutation left empty are skipped below) and the routes whose activations
+    // the CTA reads: no device data needed yet
+    auto warp_start = [&](unsigned w) {
+        return Y ? (int)(((long long)w - (long long)blockIdx.x * kWarps) * p.k * np / kWarps)
+                 : (int)div_u32(w * p.n_all, p.n_warps, p.inv_warps);
+    };
     const int w_u0 = warp_start(blockIdx.x * kWarps + warp), w_u1 = warp_start(blockIdx.x * kWarps + warp + 1);
     const int trips = (w_u1 - w_u0 + gpw - 1) / gpw;
     const int c_u0 = warp_start(blockIdx.x * kWarps), c_u1 = warp_start((blockIdx.x + 1) * kWarps);
@@ -591,17 +614,20 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     // releases dependents -- unless it is the CTA that writes the routing
     const bool writer = ROUTE && PHASE == 1 && blockIdx.x == 0;
     if (c_u1 == c_u0 && !writer) return;
-    const int s_lo = c_u1 > c_u0 ? div_small(c_u0, n_units, p.inv_units) : 0;
-    const int s_hi = c_u1 > c_u0 ? div_small(c_u1 - 1, n_units, p.inv_units) : 0;
-    if ((PHASE == 1 ? 1 : s_hi - s_lo + 1) * K > p.xs_floats) {
+    const int s_lo = Y ? 0 : (c_u1 > c_u0 ? div_small(c_u0, n_units, p.inv_units) : 0);
+    const int s_hi = Y ? p.k - 1 : (c_u1 > c_u0 ? div_small(c_u1 - 1, n_units, p.inv_units) : 0);
+    // Y: the CTA's rows of every route follow the activations, [sorted route][2 np]
+    float *s_rows = xs + (size_t)p.k * K;
+    if ((PHASE == 1 ? 1 : s_hi - s_lo + 1) * K + (Y ? 2 * p.k * np : 0) > p.xs_floats) {
         // cannot happen with the host's sizing (same for every thread of the CTA)
         if (threadIdx.x == 0) record_gemv_error(0x2007u, (unsigned)(s_hi - s_lo + 1));
         return;
     }
-    // the lane group's first unit: route and unit within the route
+    // the lane group's first unit: route and unit within the route (Y: within
+    // the CTA's np pairs)
     int nx_u = w_u0 + gi;
-    int nx_sr = div_small(nx_u, n_units, p.inv_units);
-    int nx_i = nx_u - nx_sr * n_units;
+    int nx_sr = Y ? nx_u / np : div_small(nx_u, n_units, p.inv_units);
+    int nx_i = nx_u - nx_sr * np;
     int nx_trip = 0, nx_pass = 0;
     // phase 1 waits for the permutation here; phase 2 may be scheduled as soon
     // as phase 1 has started and waits for h further down
@@ -609,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
     pdl_launch_dependents();
     if (ROUTE) {
         // the kernel routes the token itself: all k routes are valid
-        tok_route(p, writer, s_exp, s_blob);
+        tok_route(p, writer, s_exp, s_blob, Y ? s_posj : nullptr, Y ? s_wj : nullptr);
         if (c_u1 == c_u0) return;  // the writer without units of its own
         if (threadIdx.x == 0) s_nroutes = p.k;
         __syncthreads();
@@ -645,8 +671,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
         x.live = nx_trip < trips && nx_u < w_u1 && nx_sr < R;
         x.c0 = nx_pass * lg * C + li;
         x.sr = nx_sr;
-        x.r0 = PHASE == 1 ? nx_i : 2 * nx_i;
-        x.v1 = PHASE == 1 || 2 * nx_i + 1 < H;
+        x.r0 = PHASE == 1 ? nx_i : 2 * (cp0 + nx_i);
+        x.v1 = PHASE == 1 || x.r0 + 1 < H;
         x.w0 = nullptr; x.s0 = nullptr;
         if (x.live) {
             const uint8_t *blob = s_blob[x.sr];
@@ -660,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
             ++nx_trip;
             nx_u += gpw;
             nx_i += gpw;
-            while (nx_i >= n_units) { nx_i -= n_units; ++nx_sr; }
+            while (nx_i >= np) { nx_i -= np; ++nx_sr; }
         }
     };
 
@@ -750,6 +776,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
                     }
                     if (PHASE == 1) {
                         p.h[(size_t)cur.sr * I + cur.r0] = f32_to_bf16_rne(gelu_tanh(a0) * a1);
+                    } else if (Y) {
+                        float *yr = s_rows + (size_t)cur.sr * 2 * np + (cur.r0 - 2 * cp0);
+                        yr[0] = a0;
+                        if (cur.v1) yr[1] = a1;
                     } else {
                         p.rows[(size_t)cur.sr * H + cur.r0] = a0;
                         if (cur.v1) p.rows[(size_t)cur.sr * H + r1] = a1;
@@ -759,6 +789,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv_tok(FfnParams p) {
             a0 = 0.0f; a1 = 0.0f;
         }
         cur = nx;
+    }
+    if (Y) {
+        // y for the CTA's rows 2 cp0 .. 2 (cp0 + np) - 1: the routes in route order
+        __syncthreads();
+        const int n_rows = min(2 * np, H - 2 * cp0);
+        for (int lr = threadIdx.x; lr < n_rows; lr += kThreads) {
+            float a = 0.0f;
+            for (int j = 0; j < p.k; ++j) a = __fmaf_rn(s_wj[j], s_rows[(size_t)s_posj[j] * 2 * np + lr], a);
+            p.y[2 * cp0 + lr] = f32_to_bf16_rne(a);
+        }
     }
 }
 
@@ -812,6 +852,13 @@ size_t tok_xs_floats(const FfnParams &p, int phase, int n_sm) {
     return (size_t)span * p.L.I;
 }
 
+// Phase 2 with the combine (Y): the h rows of all k routes, then the CTA's rows
+// of every route (at most ceil(units / n_sm) row pairs each).
+size_t tok_y_floats(const FfnParams &p, int n_sm) {
+    const long long n_units = (p.L.H + 1) / 2;
+    return (size_t)p.k * p.L.I + (size_t)(2 * p.k * ((n_units + n_sm - 1) / n_sm));
+}
+
 // The one-token kernels take the call: T = 1, a CTA's activations fit in shared
 // memory beside a second CTA, and w * N stays below 2^32 for every warp w (at up
 // to 8 CTAs per SM).
@@ -822,7 +869,7 @@ bool tok_fits(const FfnParams &p, int n_sm) {
            max_units * (unsigned long long)(n_sm * 8 * kWarps) < (1ull << 32);
 }
 
-template <int FMT, int PHASE, int C, bool ROUTE>
+template <int FMT, int PHASE, int C, bool ROUTE, bool Y = false>
 cudaError_t launch_tok(const FfnParams &p0, int n_sm, cudaStream_t s) {
     FfnParams p = p0;
     const int nchunks = (PHASE == 1 ? p.L.H : p.L.I) / Fmt<FMT>::kElems;
@@ -830,11 +877,11 @@ cudaError_t launch_tok(const FfnParams &p0, int n_sm, cudaStream_t s) {
     while (lg < 32 && lg * C < nchunks) lg <<= 1;
     p.lg = lg;
     p.passes = (nchunks + lg * C - 1) / (lg * C);
-    p.xs_floats = (int)tok_xs_floats(p, PHASE, n_sm);
+    p.xs_floats = (int)(Y ? tok_y_floats(p, n_sm) : tok_xs_floats(p, PHASE, n_sm));
     const int n_units = PHASE == 1 ? p.L.I : (p.L.H + 1) / 2;
     p.inv_units = 1.0f / (float)n_units;
     const size_t smem = (size_t)p.xs_floats * sizeof(float);
-    auto kern = k_ffn_gemv_tok<FMT, PHASE, C, ROUTE>;
+    auto kern = k_ffn_gemv_tok<FMT, PHASE, C, ROUTE, Y>;
     static size_t cached_smem[kMaxDevices] = {};
     static int cached_per_sm[kMaxDevices] = {};
     int dev = 0;
@@ -871,6 +918,10 @@ cudaError_t launch_fmt(const FfnParams &p, int n_sm, cudaStream_t s) {
         if (p.logits != nullptr) {
             cudaError_t err = launch_tok<FMT, 1, C, true>(p, n_sm, s);
             if (err != cudaSuccess) return err;
+            if (p.y != nullptr) {
+                if (tok_y_floats(p, n_sm) * 4 > kTokSmemMax) return cudaErrorInvalidValue;
+                return launch_tok<FMT, 2, C, true, true>(p, n_sm, s);
+            }
             return launch_tok<FMT, 2, C, true>(p, n_sm, s);
         }
         cudaError_t err = launch_tok<FMT, 1, C, false>(p, n_sm, s);
@@ -905,10 +956,20 @@ bool ffn_gemv_can_route(const LayerView &L, int T, int k) {
     return T == 1 && L.E <= 128 && tok_fits(p, n_sm);
 }
 
+bool ffn_gemv_can_combine(const LayerView &L, int T, int k) {
+    int n_sm = 0;
+    if (!ffn_gemv_can_route(L, T, k) || sm_count(&n_sm) != cudaSuccess) return false;
+    FfnParams p{};
+    p.L = L;
+    p.T = T;
+    p.k = k;
+    return tok_y_floats(p, n_sm) * 4 <= kTokSmemMax;
+}
+
 cudaError_t launch_ffn_gemv_routed(const LayerView &L, const uint16_t *x, const float *logits, int k,
                                    uint32_t *hits, int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
                                    int32_t *sorted_route, int32_t *route_pos, float *rows, void *ws,
-                                   cudaStream_t s) {
+                                   uint16_t *y, cudaStream_t s) {
     int n_sm = 0;
     cudaError_t err = sm_count(&n_sm);
     if (err != cudaSuccess) return err;
@@ -930,6 +991,7 @@ cudaError_t launch_ffn_gemv_routed(const LayerView &L, const uint16_t *x, const 
     p.offsets_out = offsets;
     p.sorted_out = sorted_route;
     p.pos_out = route_pos;
+    p.y = y;
     if (L.fmt == MOE_W_BF16) return launch_fmt<MOE_W_BF16>(p, n_sm, s);
     if (L.fmt == MOE_W_INT8) return launch_fmt<MOE_W_INT8>(p, n_sm, s);
     return launch_fmt<MOE_W_INT4>(p, n_sm, s);

@@ -53,10 +53,10 @@ def test_launch_count_per_layer_step():
     m = _FakeMoe()
     # one token: fused route + permute, two GEMV launches, combine
     assert bench.launches_per_layer(m, 1, 8, 0, m.MOE_FFN_AUTO) == 1 + 2 + 1
-    # one token through moe_route_ffn (the stacks): the routing inside the two
-    # GEMV launches; not past its expert count, on a forced path, or where AUTO
-    # takes the tensor cores
-    assert bench.launches_per_layer(m, 1, 8, 0, m.MOE_FFN_AUTO, E=128) == 0 + 2 + 1
+    # one token through moe_layer_forward (the stacks): the routing inside the
+    # first GEMV launch and the combine inside the second; not past its expert
+    # count, on a forced path, or where AUTO takes the tensor cores
+    assert bench.launches_per_layer(m, 1, 8, 0, m.MOE_FFN_AUTO, E=128) == 0 + 2 + 0
     assert bench.launches_per_layer(m, 1, 8, 0, m.MOE_FFN_AUTO, E=256) == 1 + 2 + 1
     assert bench.launches_per_layer(m, 1, 8, 0, m.MOE_FFN_GEMV, E=128) == 1 + 2 + 1
     assert bench.launches_per_layer(m, 1, 32, 0, m.MOE_FFN_AUTO, E=128) == 1 + 3 + 1

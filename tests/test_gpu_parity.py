@@ -688,3 +688,63 @@ def test_one_token_every_element(fmt, E, H, I, k):
     assert rel_err(rows.cpu().numpy()[rp.cpu().numpy()], orows) <= FFN_TOL
     assert rel_err(bf16_dev_to_f64(y), oy) <= FFN_TOL
     assert moe.moe_take_device_errors() == (0, 0)
+
+
+# moe_layer_forward at one token: where the FFN's launches route the token, the
+# second launch also takes the combine (each CTA sums the k routes of its own
+# output rows), so y must be bit-identical to moe_route_ffn + moe_combine; the
+# cases cover CTAs without rows (H = 64), k = 32 and E = 200 (two calls, then
+# the separate combine)
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("E,H,I,k", [(128, 256, 128, 8), (8, 256, 128, 6), (128, 2816, 704, 8), (6, 1024, 320, 4),
+                                     (4, 64, 64, 1), (33, 512, 192, 32), (200, 256, 128, 8)])
+def test_layer_forward_one_token_combine_in_the_ffn(fmt, E, H, I, k):
+    w13, w2 = syn.expert_weights(E, H, I, seed=E + 7 * k)
+    L = moe.make_layer(fmt, *device_weights_from_host(w13, w2))
+    x = syn.activations(1, H, seed=H + 3)
+    lg = syn.router_logits(1, E, "normal", seed=E * 5 + k)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    d_lg = torch.from_numpy(lg).to(DEV)
+    h1 = torch.zeros(E, dtype=torch.int32, device=DEV)
+    h2 = torch.zeros(E, dtype=torch.int32, device=DEV)
+    ids1 = torch.empty((1, k), dtype=torch.int32, device=DEV)
+    w1 = torch.empty((1, k), dtype=torch.float32, device=DEV)
+    ys = []
+    for _ in range(2):  # twice: the second call finds the previous call's shared memory and y
+        ys.append(moe.moe_layer_forward(L, d_lg, xd, k, hits=h1, ids_out=ids1, w_out=w1))
+    ids, w, counts, offsets, sr, rp, rows = moe.moe_route_ffn(L, d_lg, xd, k, hits=h2)
+    h2 += torch.from_numpy(oracle.hits(oracle.route_topk(lg, k)[0], E).view(np.int32)).to(DEV)
+    y2 = moe.moe_combine(rows, rp, w, torch.empty((1, H), dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert moe.moe_take_device_errors() == (0, 0)
+    for y1 in ys:
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(ids1, ids) and torch.equal(w1.view(torch.int32), w.view(torch.int32))
+    assert torch.equal(h1, h2)
+    oi, ow, orows, oy = oracle.moe_layer(oracle_layer_for(fmt, w13, w2), lg, x, k)
+    assert np.array_equal(ids1.cpu().numpy(), oi)
+    assert rel_err(bf16_dev_to_f64(ys[0]), oy) <= FFN_TOL
+
+
+@pytest.mark.parametrize("fmt", [0, 2])
+def test_layer_forward_one_token_combine_on_a_slot_table(fmt):
+    """The fused one-token combine reads the rows of pooled and home experts
+    alike: y equals the oracle's on a 24-slot pool behind 8 experts."""
+    E, H, I, k = 8, 512, 192, 3
+    w13, w2 = syn.expert_weights(E, H, I, seed=79)
+    slot_of = np.array([23, -1, 17, 5, -1, 20, 0, 11], np.int32)
+    Ld, OL = _pool_layers(fmt, E, H, I, w13, w2, slot_of, 24)
+    x = syn.activations(1, H, seed=80)
+    lg = syn.router_logits(1, E, "normal", seed=93)
+    lg[0, 1] += 4.0
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    d_lg = torch.from_numpy(lg).to(DEV)
+    y1 = moe.moe_layer_forward(Ld, d_lg, xd, k)
+    ids, w, counts, offsets, sr, rp, rows = moe.moe_route_ffn(Ld, d_lg, xd, k)
+    y2 = moe.moe_combine(rows, rp, w, torch.empty((1, H), dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert moe.moe_take_device_errors() == (0, 0)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    oi, ow, orows, oy = oracle.moe_layer(OL, lg, x, k)
+    assert (slot_of[oi] >= 0).any() and (slot_of[oi] < 0).any()
+    assert rel_err(bf16_dev_to_f64(y1), oy) <= FFN_TOL

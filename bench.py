@@ -825,6 +825,7 @@ def main():
         "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": head["gpu_launches"],
+        **({"one_call": head["one_call"]} if "one_call" in head else {}),
         "clocks": clk,
         "cpu_baseline": cpu,
     }

@@ -31,7 +31,7 @@ def _layers(fmt, E, H, I, n):
 
 
 @pytest.mark.parametrize("fmt", ["bf16", "int8", "int4"])
-@pytest.mark.parametrize("T", [3, 40])
+@pytest.mark.parametrize("T", [1, 3, 40])  # 1: the routing and the combine inside the FFN's launches
 def test_graph_replay_equals_eager_and_oracle(fmt, T):
     E, H, I, k, n = 16, 256, 128, 4, 3
     layers = _layers(moe.FMT[fmt], E, H, I, n)

@@ -14,7 +14,9 @@
 // One token (T = 1) has kernels of its own (k_ffn_gemv_tok, below): the k
 // routes' rows are split evenly over all warps, each warp streams its rows
 // without pausing between them, and the set-up before the first weight load is
-// a single round of loads.
+// a single round of loads.  Where they route the token themselves (a
+// moe_layer_forward call), phase 2 can also take the combine: each CTA then
+// computes every route of its own output rows and writes y (see k_ffn_gemv_tok).
 //
 // Work decomposition (T > 1).  A work item is (active expert, chunk of <= 8 of its
 // routes, tile of output rows).  Each CTA (8 warps) takes a contiguous range

@@ -1006,11 +1006,16 @@ k_ffn_tc(const __grid_constant__ CUtensorMap map_home, const __grid_constant__ C
 }
 
 // x rows gathered into sorted-route order: xs[s] = x[sorted_route[s] / k] for
-// s < offsets[E] (16 bytes per thread).  With `perm` (the int4 kernels) each run
-// of 8 elements is stored in the order k_order<MOE_W_INT4> gives.
-__global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ sorted_route,
-                              const int32_t *__restrict__ offsets, int E, int k, int H, int R, int perm,
-                              uint16_t *__restrict__ xs, unsigned *__restrict__ ready) {
+// s < offsets[E].  One warp per row (grid-stride over rows): the route is read
+// once, then each lane loads up to kGatherPer 16-byte pieces of the row before
+// it stores any, so a row takes one round trip.  With `perm` (the int4 kernels)
+// each run of 8 elements is stored in the order k_order<MOE_W_INT4> gives.
+constexpr int kGatherPer = 12;  // pieces per lane in flight (a 2816-wide row: 11)
+__global__ void __launch_bounds__(256) k_gather_rows(const uint16_t *__restrict__ x,
+                                                     const int32_t *__restrict__ sorted_route,
+                                                     const int32_t *__restrict__ offsets, int E, int k, int H, int R,
+                                                     int perm, uint16_t *__restrict__ xs,
+                                                     unsigned *__restrict__ ready) {
     // programmatic dependent launch: wait for the previous kernel before
     // touching memory, then let the next one be scheduled
     pdl_wait();
@@ -1018,28 +1023,40 @@ __global__ void k_gather_rows(const uint16_t *__restrict__ x, const int32_t *__r
     // the per-expert counters of this call's phase 1 (nullable: gather only)
     if (ready != nullptr && blockIdx.x == 0)
         for (int e = threadIdx.x; e < E; e += blockDim.x) ready[e] = 0u;
-    const int per = H / 8;
-    const int n_valid = __ldg(offsets + E);
+    const int per = H / 8;  // 16-byte pieces per row
+    const int n_valid = min(__ldg(offsets + E), R);
     const uint64_t pol = l2_policy_last();
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)R * per;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int s = (int)(i / per), c = (int)(i % per);
-        if (s >= n_valid) continue;
+    const int lane = threadIdx.x & 31;
+    const int n_warps = (int)(gridDim.x * (blockDim.x >> 5));
+    for (int s = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)); s < n_valid; s += n_warps) {
         const int route = __ldg(sorted_route + s);
-        const int tok = route / k;
         if (route < 0 || route >= R) {
-            record_error(0x2004u, (unsigned)s);
+            if (lane == 0) record_error(0x2004u, (unsigned)s);
             continue;
         }
-        uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)tok * H) + c);
-        if (perm) {  // elements (0,1)(2,3)(4,5)(6,7) -> (0,2)(1,3)(4,6)(5,7)
-            const uint4 v = u;
-            u.x = __byte_perm(v.x, v.y, 0x5410);
-            u.y = __byte_perm(v.x, v.y, 0x7632);
-            u.z = __byte_perm(v.z, v.w, 0x5410);
-            u.w = __byte_perm(v.z, v.w, 0x7632);
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(route / k) * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)s * H);
+        for (int c0 = 0; c0 < per; c0 += 32 * kGatherPer) {
+            uint4 u[kGatherPer];
+#pragma unroll
+            for (int j = 0; j < kGatherPer; ++j) {
+                const int c = c0 + 32 * j + lane;
+                if (c < per) u[j] = __ldg(src + c);
+            }
+#pragma unroll
+            for (int j = 0; j < kGatherPer; ++j) {
+                const int c = c0 + 32 * j + lane;
+                if (c >= per) break;
+                uint4 v = u[j];
+                if (perm) {  // elements (0,1)(2,3)(4,5)(6,7) -> (0,2)(1,3)(4,6)(5,7)
+                    v.x = __byte_perm(u[j].x, u[j].y, 0x5410);
+                    v.y = __byte_perm(u[j].x, u[j].y, 0x7632);
+                    v.z = __byte_perm(u[j].z, u[j].w, 0x5410);
+                    v.w = __byte_perm(u[j].z, u[j].w, 0x7632);
+                }
+                st_v4_hint(dst + c, v, pol);
+            }
         }
-        st_v4_hint(reinterpret_cast<uint4 *>(xs + (size_t)s * H) + c, u, pol);
     }
 }
 
@@ -1156,8 +1173,8 @@ cudaError_t launch_ffn_tc(const LayerView &L, const uint16_t *x, int T, int k, c
 
     // 1. activations into sorted-route order
     {
-        const int64_t n = (int64_t)R * (H / 8);
-        const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)n_sm * 8);
+        // one warp per row, eight rows per CTA, at most 8 CTAs per SM
+        const int blocks = (int)std::min<int64_t>(((int64_t)R + 7) / 8, (int64_t)n_sm * 8);
         err = launch_pdl(k_gather_rows, dim3((unsigned)blocks), dim3(256), 0, s, x, sorted_route, offsets, L.E, k, H, R,
                          (int)(L.fmt == MOE_W_INT4), xs, ready);
         if (err != cudaSuccess) return err;

@@ -58,18 +58,18 @@ _CAPTURE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_
             "--clock-control none -k regex:'k_ffn|k_gather_rows', one layer call of bench.py --quick "
             "--headline-only --layers 2")
 NCU_TRAFFIC_BYTES = {
-    ("moe-layer-bf16-decode-T64", "auto"): (1506657792, 1499103232, _CAPTURE + " (gather + 2 tcgen05 launches)"),
-    ("moe-layer-bf16-decode-T8", "auto"): (584311040, 582889472, _CAPTURE + " --tokens 8 (gather + 2 tcgen05 launches)"),
-    ("moe-layer-bf16-decode-T1", "auto"): (95626240, 95163904, _CAPTURE + " --tokens 1 (2 one-token GEMV launches)"),
-    ("moe-layer-int8-decode-T64", "auto"): (309177344, 304539136,
+    ("moe-layer-bf16-decode-T64", "auto"): (1506674944, 1499103232, _CAPTURE + " (gather + 2 tcgen05 launches)"),
+    ("moe-layer-bf16-decode-T8", "auto"): (583954944, 582889472, _CAPTURE + " --tokens 8 (gather + 2 tcgen05 launches)"),
+    ("moe-layer-bf16-decode-T1", "auto"): (95784192, 95163904, _CAPTURE + " --tokens 1 (2 one-token GEMV launches)"),
+    ("moe-layer-int8-decode-T64", "auto"): (308761856, 304539136,
                                             _CAPTURE + " --config decode-int8 (gather + 2 tcgen05 launches)"),
-    ("moe-layer-int8-decode-T8", "auto"): (143899904, 143187968,
+    ("moe-layer-int8-decode-T8", "auto"): (144329472, 143187968,
                                            _CAPTURE + " --config decode-int8 --tokens 8 (gather + 2 tcgen05 launches)"),
-    ("moe-layer-int8-decode-T1", "auto"): (47792128, 47719936,
+    ("moe-layer-int8-decode-T1", "auto"): (47796224, 47719936,
                                            _CAPTURE + " --config decode-int8 --tokens 1 (2 one-token GEMV launches)"),
-    ("moe-layer-int4-decode-T64", "auto"): (404422144, 398464000,
+    ("moe-layer-int4-decode-T64", "auto"): (404659712, 398464000,
                                             _CAPTURE + " --config int4-decode (gather + 2 tcgen05 launches)"),
-    ("moe-layer-int4-prefill-T1024", "auto"): (522397440, 410189824,
+    ("moe-layer-int4-prefill-T1024", "auto"): (521776128, 410189824,
                                                _CAPTURE + " --config int4-prefill (gather + 2 tcgen05 launches)"),
 }
 

@@ -94,15 +94,26 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t *__restrict__ id
     int total = 0;
     if (tid < E)
         for (int w = 0; w < kWarps; ++w) total += s_w[w * E + tid];
-    s_scan[tid] = total;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-        int v = (tid >= off) ? s_scan[tid - off] : 0;
-        __syncthreads();
-        s_scan[tid] += v;
-        __syncthreads();
+    // inclusive scan: within each warp by shuffles, then over the 32 warp sums
+    int incl = total;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
     }
-    const int incl = s_scan[tid];
+    if (lane == 31) s_scan[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int ws = s_scan[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, ws, off);
+            if (lane >= off) ws += v;
+        }
+        s_scan[32 + lane] = ws - s_scan[lane];  // exclusive: the warps before
+    }
+    __syncthreads();
+    incl += s_scan[32 + warp];
     const int excl = incl - total;
     if (tid < E) {
         counts[tid] = total;

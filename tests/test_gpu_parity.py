@@ -748,3 +748,44 @@ def test_layer_forward_one_token_combine_on_a_slot_table(fmt):
     oi, ow, orows, oy = oracle.moe_layer(OL, lg, x, k)
     assert (slot_of[oi] >= 0).any() and (slot_of[oi] < 0).any()
     assert rel_err(bf16_dev_to_f64(y1), oy) <= FFN_TOL
+
+
+@pytest.mark.parametrize("case", ["ties", "nan", "inf", "neg_inf", "neg_zero"])
+def test_layer_forward_one_token_degenerate_logits(case):
+    """One token through moe_layer_forward (routing and combine inside the FFN's
+    launches) with degenerate router logits: all equal (ties to the lower id),
+    a NaN, +inf entries, all -inf but one, -0.0 entries.  ids and weights match
+    the oracle's routing bit for bit and y matches the separate calls bit for bit."""
+    E, H, I, k = 16, 512, 192, 4
+    w13, w2 = syn.expert_weights(E, H, I, seed=101)
+    L = moe.make_layer(0, *device_weights_from_host(w13, w2))
+    x = syn.activations(1, H, seed=102)
+    lg = syn.router_logits(1, E, "normal", seed=103)
+    if case == "ties":
+        lg[:] = 0.5
+    elif case == "nan":
+        lg[0, 3] = np.nan
+    elif case == "inf":
+        lg[0, [2, 9]] = np.inf
+    elif case == "neg_inf":
+        lg[:] = -np.inf
+        lg[0, 7] = 1.0
+    else:
+        lg[0, ::3] = -0.0
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    d_lg = torch.from_numpy(lg).to(DEV)
+    ids1 = torch.empty((1, k), dtype=torch.int32, device=DEV)
+    w1 = torch.empty((1, k), dtype=torch.float32, device=DEV)
+    y1 = moe.moe_layer_forward(L, d_lg, xd, k, ids_out=ids1, w_out=w1)
+    ids, w, counts, offsets, sr, rp, rows = moe.moe_route_ffn(L, d_lg, xd, k)
+    y2 = moe.moe_combine(rows, rp, w, torch.empty((1, H), dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert moe.moe_take_device_errors() == (0, 0)
+    oi, ow = oracle.route_topk(lg, k)
+    assert np.array_equal(ids1.cpu().numpy(), oi)
+    g = w1.cpu().numpy()
+    assert np.array_equal(np.isnan(g), np.isnan(ow))  # NaN weights where the oracle has them
+    fin = ~np.isnan(ow)
+    assert bits_equal(np.where(fin, g, 0), np.where(fin, ow, 0))
+    assert torch.equal(w1.view(torch.int32), w.view(torch.int32))
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
